@@ -1,0 +1,119 @@
+"""PyTorch-facing wrappers of the C ABI (argument marshalling only).
+
+PyTorch supplies device memory and the current stream; every step of the
+alpha-entmax attention runs inside libentattn.so.  Tensors are [B, H, N, d],
+contiguous, float32 or bfloat16, on one CUDA device.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import capi
+
+_DTYPES = {torch.float32: capi.ENT_F32, torch.bfloat16: capi.ENT_BF16}
+
+
+def _stream_handle(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(*ts):
+    t0 = ts[0]
+    if t0.dim() != 4:
+        raise ValueError(f"expected [B, H, N, d] tensors, got shape {tuple(t0.shape)}")
+    if t0.dtype not in _DTYPES:
+        raise ValueError(f"dtype {t0.dtype} not supported (float32 or bfloat16)")
+    for t in ts:
+        if t.shape != t0.shape or t.dtype != t0.dtype or t.device != t0.device:
+            raise ValueError("q, k, v (and o, dout) must share shape, dtype and device")
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _raise(st: int, where: str):
+    if st != capi.ENT_OK:
+        raise capi.EntAttnError(st, where, capi.ent_attn_last_error())
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A device workspace of at least ``nbytes`` bytes (256-byte aligned by torch)."""
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def entmax_attn_fwd(q, k, v, alpha: float = 1.5, causal: bool = False, *, with_iters=False,
+                    ws: torch.Tensor | None = None, out=None):
+    """Forward: returns (o, tau, block_mask, iters_or_None)."""
+    _check(q, k, v)
+    B, H, N, d = q.shape
+    dt = _DTYPES[q.dtype]
+    T = -(-N // capi.ent_attn_block_size()) if N else 0
+    if out is None:
+        o = torch.empty_like(q)
+        tau = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+        mask = torch.empty((B, H, T, T), dtype=torch.uint8, device=q.device)
+        iters = torch.empty((B, H, N), dtype=torch.uint8, device=q.device) if with_iters else None
+    else:
+        o, tau, mask, iters = out
+    need = capi.ent_attn_fwd_workspace_size(B, H, N, d, dt)
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, q.device)
+    st = capi.ent_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, dt, alpha,
+                           causal, o.data_ptr(), tau.data_ptr(), mask.data_ptr(),
+                           iters.data_ptr() if iters is not None else None, ws.data_ptr(),
+                           ws.numel(), _stream_handle(q.device))
+    _raise(st, "ent_attn_fwd")
+    return o, tau, mask, iters
+
+
+def entmax_attn_bwd(q, k, v, o, dout, tau, block_mask, alpha: float = 1.5, causal: bool = False,
+                    *, ws: torch.Tensor | None = None, out=None):
+    """Backward: returns (dq, dk, dv)."""
+    _check(q, k, v, dout)
+    B, H, N, d = q.shape
+    dt = _DTYPES[q.dtype]
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = out
+    need = capi.ent_attn_bwd_workspace_size(B, H, N, d, dt)
+    if ws is None or ws.numel() < need:
+        ws = workspace(need, q.device)
+    st = capi.ent_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                           o.data_ptr() if o is not None else None, dout.data_ptr(),
+                           tau.data_ptr(), block_mask.data_ptr(), B, H, N, d, dt, alpha, causal,
+                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(),
+                           _stream_handle(q.device))
+    _raise(st, "ent_attn_bwd")
+    return dq, dk, dv
+
+
+def read_status(ws: torch.Tensor) -> list[int]:
+    """Counters of the last call that used ``ws`` (synchronises); raises on a timeout flag."""
+    st, ctr = capi.ent_attn_read_status(ws.data_ptr(), _stream_handle(ws.device))
+    _raise(st, "ent_attn_read_status")
+    return ctr
+
+
+class EntmaxAttention(torch.autograd.Function):
+    """Autograd wrapper: O = entmax_alpha(Q K^T / sqrt(d)) V."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, alpha, causal):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, tau, mask, _ = entmax_attn_fwd(q, k, v, alpha, causal)
+        ctx.save_for_backward(q, k, v, o, tau, mask)
+        ctx.alpha, ctx.causal = alpha, causal
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, tau, mask = ctx.saved_tensors
+        dq, dk, dv = entmax_attn_bwd(q, k, v, o, do.contiguous(), tau, mask, ctx.alpha, ctx.causal)
+        return dq, dk, dv, None, None
+
+
+def entmax_attention(q, k, v, alpha: float = 1.5, causal: bool = False):
+    """Differentiable fused alpha-entmax attention."""
+    return EntmaxAttention.apply(q, k, v, alpha, causal)

@@ -1,0 +1,187 @@
+// common.cuh -- device-side pieces shared by every kernel of the library:
+// the alpha-entmax power terms, the per-row tau solver state and its
+// Halley-bisection update, the sliding score histogram, and the workspace
+// header layout.
+//
+// Method (AdaSplash pages, by title and section):
+//   "AdaSplash: Adaptive Sparse Flash Attention", Technical Deep Dive /
+//   Accelerated Alpha-Entmax Transformation: tau is the root of
+//   f(tau) = sum_j (x_j - tau)_+^gamma - 1, x = (alpha-1) s, gamma = 1/(alpha-1);
+//   f' and f'' are again shifted powers times constants; Halley's step is taken
+//   when it stays inside the bracket, otherwise the bracket is bisected.
+//   "AdaSplash-2: ...", Sparse Attention Makes Waves: the iteration starts from
+//   a coarse histogram of the row's scores kept on chip.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace ent {
+
+constexpr int kBlk = 128;          // query-tile rows and key-block columns
+constexpr int kBins = 64;          // histogram slots per row
+constexpr float kBinsPerUnit = 63.f;  // bin width 1/63: 64 slots cover [m-1, m]
+constexpr int kMaxPass = 24;       // solver pass cap (bisection alone needs ~20-23)
+
+// Workspace header (first 256 bytes of every workspace).
+struct WsHeader {
+    unsigned int status;           // 0 = ok, 1 = a bounded wait gave up
+    unsigned int timeout_site;     // where it gave up (debug)
+    unsigned int tile_counter;     // persistent-scheduler work counter
+    unsigned int pad0;
+    unsigned long long counters[8];
+    unsigned char pad1[256 - 16 - 64];
+};
+static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
+
+enum Counter { kCtrQkBlocks = 0, kCtrPvBlocks = 1, kCtrPasses = 2, kCtrTiles = 3,
+               kCtrBwdBlocks = 4 };
+
+__device__ __forceinline__ float load_f(const float* p, size_t i) { return p[i]; }
+__device__ __forceinline__ float load_f(const __nv_bfloat16* p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_f(float* p, size_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void store_f(__nv_bfloat16* p, size_t i, float v) {
+    p[i] = __float2bfloat16_rn(v);
+}
+
+// Power terms of u = x - tau > 0: t0 = u^gamma (the probability), t1 = u^(gamma-1)
+// (the backward's g and -f'/gamma), t2 = u^(gamma-2) (f''/(gamma(gamma-1))).
+// GM = 1..4 is an exact integer gamma (alpha = 2, 1.5, 4/3, 1.25); GM = 0 any
+// gamma >= 1 via exp2/log2.  u <= 0 gives zeros (strict support).
+template <int GM>
+__device__ __forceinline__ void entmax_terms(float u, float gamma, float& t0, float& t1,
+                                             float& t2) {
+    if (!(u > 0.f)) { t0 = t1 = t2 = 0.f; return; }
+    if (GM == 1) { t0 = u; t1 = 1.f; t2 = 0.f; }
+    else if (GM == 2) { t0 = u * u; t1 = u; t2 = 1.f; }
+    else if (GM == 3) { const float u2 = u * u; t0 = u2 * u; t1 = u2; t2 = u; }
+    else if (GM == 4) { const float u2 = u * u; t0 = u2 * u2; t1 = u2 * u; t2 = u2; }
+    else {
+        t2 = exp2f((gamma - 2.f) * __log2f(u));
+        t1 = t2 * u;
+        t0 = t1 * u;
+    }
+}
+
+template <int GM>
+__device__ __forceinline__ float entmax_p(float u, float gamma) {
+    if (!(u > 0.f)) return 0.f;
+    if (GM == 1) return u;
+    if (GM == 2) return u * u;
+    if (GM == 3) return u * u * u;
+    if (GM == 4) { const float u2 = u * u; return u2 * u2; }
+    return exp2f(gamma * __log2f(u));
+}
+
+template <int GM>
+__device__ __forceinline__ float entmax_g(float u, float gamma) {
+    if (!(u > 0.f)) return 0.f;
+    if (GM == 1) return 1.f;
+    if (GM == 2) return u;
+    if (GM == 3) return u * u;
+    if (GM == 4) return u * u * u;
+    return exp2f((gamma - 1.f) * __log2f(u));
+}
+
+// Per-row solver state.
+struct RowSolver {
+    float tau, lo, hi;
+    int done;
+    int iters;
+};
+
+// One Halley-bisection update after a pass evaluated F0 = sum u^gamma,
+// F1 = sum u^(gamma-1), F2 = sum u^(gamma-2) at the current tau.  Stops (keeping
+// the evaluated tau) when |f| <= ftol, when the proposed step is below
+// stol*max(1,|tau|), or at the pass cap.  The Halley point is taken when it lies
+// within the closed bracket [lo, hi] (a point that rounding put a few ulps
+// outside is clamped onto it: a root on a bracket end, such as tau = m - 1 for
+// a one-element support, must stay reachable); otherwise the bracket is bisected.
+__device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1, float F2,
+                                              float gamma, bool gamma_is_one, int pass,
+                                              float ftol, float stol) {
+    if (st.done) return;
+    const float f = F0 - 1.f;
+    if (fabsf(f) <= ftol || pass >= kMaxPass) { st.done = 1; st.iters = pass; return; }
+    if (f > 0.f) st.lo = st.tau; else st.hi = st.tau;
+    const float fp = -gamma * F1;
+    const float fpp = gamma_is_one ? 0.f : gamma * (gamma - 1.f) * F2;
+    const float h = st.tau - 2.f * f * fp / (2.f * fp * fp - f * fpp);
+    const float tol = stol * fmaxf(1.f, fabsf(st.tau));
+    const float next = (isfinite(h) && h >= st.lo - tol && h <= st.hi + tol)
+                           ? fminf(fmaxf(h, st.lo), st.hi)
+                           : 0.5f * (st.lo + st.hi);
+    if (fabsf(next - st.tau) <= tol) { st.done = 1; st.iters = pass; return; }
+    st.tau = next;
+}
+
+// ---------------------------------------------------------------- histogram
+// Absolute bin of x: a = floor(x * 63).  A row whose running maximum m has bin
+// A keeps the 64 bins A-63..A in slots (a & 63).  Anything below bin A-63 lies
+// under (A-63)/63 <= m - 1 <= tau and can never be in the support.
+__device__ __forceinline__ int abs_bin(float x) { return __float2int_rd(x * kBinsPerUnit); }
+
+constexpr int kNoBin = -(1 << 29);
+
+// Slots of hist (stride `stride` between slots of one row) that leave the
+// window when the top bin moves from A_old to A_new are cleared.
+__device__ __forceinline__ void hist_slide(unsigned int* hist, int stride, int A_old, int A_new) {
+    if (A_new <= A_old) return;
+    const int moved = A_new - A_old;
+    if (moved >= kBins) {
+        for (int s = 0; s < kBins; ++s) hist[s * stride] = 0u;
+    } else {
+        for (int k = 0; k < moved; ++k) hist[((A_old - (kBins - 1) + k) & (kBins - 1)) * stride] = 0u;
+    }
+}
+
+// Bracket and start for tau from a row histogram (slots as above, top bin A,
+// max m, n admissible keys), using ptab[k] = (k/63)^gamma, k = 0..64.
+// For an edge E = e/63 the counts c_a give rigorous bounds of f:
+//   F_low(e) = sum_{a > e} c_a ptab[a-e] - 1  <=  f(E)  <=  F_up(e) = sum_{a >= e} c_a ptab[a+1-e] - 1.
+// Scanning edges down from the top bin: hi = the lowest edge with F_up <= 0,
+// lo = the first (highest) edge with F_low >= 0 (both functions are monotone).
+// Both ends are widened by a few ulps of m against rounding in the bin
+// assignment and intersected with the plain bracket [m-1, m - n^(1-alpha)].
+// tau_0 is the root of the straight line through the bin-centre model
+// F_c(E) = sum_a c_a ((a+1/2)/63 - E)_+^gamma - 1 at E = lo and E = hi.
+template <int GM>
+__device__ __forceinline__ void hist_start(const unsigned int* hist, int stride, int A, float m,
+                                           int n, float alpha, float gamma, const float* ptab,
+                                           float& lo, float& hi, float& tau0) {
+    int h_ok = A + 1;
+    int l_ok = kNoBin;
+    for (int e = A; e >= A - (kBins - 1); --e) {
+        float fu = -1.f, fl = -1.f;
+        for (int a = e; a <= A; ++a) {
+            const float c = (float)hist[(a & (kBins - 1)) * stride];
+            fu = fmaf(c, ptab[a + 1 - e], fu);
+            fl = fmaf(c, ptab[a - e], fl);
+        }
+        if (fu <= 0.f) h_ok = e;
+        if (fl >= 0.f) { l_ok = e; break; }
+    }
+    const float slack = 4.f * 1.1920929e-7f * fmaxf(1.f, fabsf(m));
+    const float plain_lo = m - 1.f;
+    const float plain_hi = m - exp2f((1.f - alpha) * __log2f((float)n));
+    lo = (l_ok != kNoBin) ? fmaxf((float)l_ok / kBinsPerUnit - slack, plain_lo) : plain_lo;
+    hi = fminf((float)h_ok / kBinsPerUnit + slack, plain_hi);
+    if (hi < lo) hi = lo;
+    float fcl = -1.f, fch = -1.f;
+    for (int k = 0; k < kBins; ++k) {
+        const int a = A - k;
+        const unsigned int c = hist[(a & (kBins - 1)) * stride];
+        if (c) {
+            const float centre = ((float)a + 0.5f) / kBinsPerUnit;
+            fcl = fmaf((float)c, entmax_p<GM>(centre - lo, gamma), fcl);
+            fch = fmaf((float)c, entmax_p<GM>(centre - hi, gamma), fch);
+        }
+    }
+    float t0 = 0.5f * (lo + hi);
+    if (fcl > 0.f && fch < 0.f) t0 = lo + (hi - lo) * (fcl / (fcl - fch));
+    tau0 = fminf(fmaxf(t0, lo), hi);
+}
+
+}  // namespace ent

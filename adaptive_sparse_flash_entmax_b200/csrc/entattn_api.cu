@@ -1,0 +1,189 @@
+// entattn_api.cu -- the C ABI (include/entattn.h): argument validation,
+// workspace layout, and dispatch to the kernels.  No exception crosses it.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/entattn.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+ent_status fail(ent_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+ent_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(ENT_ECUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+constexpr size_t kHdr = sizeof(ent::WsHeader);
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int n_tiles(int N) { return (N + ent::kBlk - 1) / ent::kBlk; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Exact integer gamma = 1/(alpha-1) in {1,2,3,4} gets a specialised kernel
+// (alpha = 2, 1.5, 4/3, 1.25); any other alpha in (1, 2] uses exp2/log2.
+int gamma_mode(float alpha, float* gamma_out) {
+    const float gamma = 1.f / (alpha - 1.f);
+    const float r = nearbyintf(gamma);
+    if (r >= 1.f && r <= 4.f && fabsf(gamma - r) <= 1e-5f * r) {
+        *gamma_out = r;
+        return (int)r;
+    }
+    *gamma_out = gamma;
+    return 0;
+}
+
+// Backward workspace layout (after the 256-byte header).
+struct BwdLayout {
+    size_t delta, dq_acc, lists, total;
+};
+
+BwdLayout bwd_layout(int B, int H, int N, int d) {
+    const size_t BH = (size_t)B * H, T = (size_t)n_tiles(N);
+    BwdLayout L;
+    L.delta = kHdr;
+    L.dq_acc = L.delta + round_up(BH * N * sizeof(float), 256);
+    L.lists = L.dq_acc + round_up(BH * N * d * sizeof(float), 256);
+    L.total = L.lists + round_up(BH * 2 * T * (T + 1) * sizeof(int), 256);
+    return L;
+}
+
+ent_status check_common(int B, int H, int N, int d, int dtype, float alpha, int causal) {
+    if (B < 0 || H < 0 || N < 0) return fail(ENT_EINVAL, "negative size (B=%d H=%d N=%d)", B, H, N);
+    if (dtype != ENT_F32 && dtype != ENT_BF16) return fail(ENT_EINVAL, "unknown dtype %d", dtype);
+    if (!(alpha > 1.f && alpha <= 2.f)) return fail(ENT_EINVAL, "alpha=%g outside (1, 2]", (double)alpha);
+    if (causal != 0 && causal != 1) return fail(ENT_EINVAL, "causal must be 0 or 1 (got %d)", causal);
+    if (d != 64 && d != 128) return fail(ENT_EUNSUPPORTED, "head dim d=%d (supported: 64, 128)", d);
+    if ((long long)B * H > 65535) return fail(ENT_EUNSUPPORTED, "B*H=%lld exceeds 65535", (long long)B * H);
+    if (n_tiles(N) > 1024) return fail(ENT_EUNSUPPORTED, "N=%d exceeds 131072", N);
+    return ENT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ent_attn_block_size(void) { return ent::kBlk; }
+
+size_t ent_attn_fwd_workspace_size(int B, int H, int N, int d, int dtype) {
+    (void)B; (void)H; (void)N; (void)d; (void)dtype;
+    return kHdr;
+}
+
+size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype) {
+    (void)dtype;
+    if (B < 0 || H < 0 || N < 0 || d < 0) return 0;
+    return bwd_layout(B, H, N, d).total;
+}
+
+const char* ent_attn_last_error(void) { return g_err.c_str(); }
+
+ent_status ent_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                        int dtype, float alpha, int causal, void* o, float* tau,
+                        uint8_t* block_mask, uint8_t* iters, void* ws, size_t ws_bytes,
+                        void* stream) {
+    ent_status st = check_common(B, H, N, d, dtype, alpha, causal);
+    if (st != ENT_OK) return st;
+    if (!ws) return fail(ENT_EINVAL, "null workspace");
+    if (ws_bytes < ent_attn_fwd_workspace_size(B, H, N, d, dtype))
+        return fail(ENT_EINVAL, "workspace of %zu bytes is below the required %zu", ws_bytes,
+                    ent_attn_fwd_workspace_size(B, H, N, d, dtype));
+    if (!aligned16(ws)) return fail(ENT_EINVAL, "workspace pointer not 16-byte aligned");
+    const bool empty = (long long)B * H == 0 || N == 0;
+    if (!empty && (!q || !k || !v || !o || !tau || !block_mask))
+        return fail(ENT_EINVAL, "null q/k/v/o/tau/block_mask pointer");
+    if (!empty && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)))
+        return fail(ENT_EINVAL, "q/k/v/o must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace header");
+    if (empty) return ENT_OK;
+
+    ent::FwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.o = o; a.tau = tau; a.mask = block_mask; a.iters = iters;
+    a.hdr = static_cast<ent::WsHeader*>(ws);
+    a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal;
+    a.alpha = alpha;
+    const int gm = gamma_mode(alpha, &a.gamma);
+    a.scale = 1.f / sqrtf((float)d);
+    a.cx = (alpha - 1.f) * a.scale;
+    // Stop rule: bf16 outputs resolve ~4e-3 relative, so |sum p - 1| <= 1e-5 is
+    // far below their rounding; float32 outputs get 1e-6.
+    a.ftol = dtype == ENT_F32 ? 1e-6f : 1e-5f;
+    a.stol = dtype == ENT_F32 ? 4e-7f : 1e-6f;
+    e = dtype == ENT_F32 ? ent::simt_fwd_f32(a, d, gm, s) : ent::simt_fwd_bf16(a, d, gm, s);
+    if (e != cudaSuccess) return cuda_fail(e, "forward launch");
+    return ENT_OK;
+}
+
+ent_status ent_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* tau, const uint8_t* block_mask, int B,
+                        int H, int N, int d, int dtype, float alpha, int causal, void* dq,
+                        void* dk, void* dv, void* ws, size_t ws_bytes, void* stream) {
+    (void)o;
+    ent_status st = check_common(B, H, N, d, dtype, alpha, causal);
+    if (st != ENT_OK) return st;
+    if (!ws) return fail(ENT_EINVAL, "null workspace");
+    const BwdLayout L = bwd_layout(B, H, N, d);
+    if (ws_bytes < L.total)
+        return fail(ENT_EINVAL, "workspace of %zu bytes is below the required %zu", ws_bytes, L.total);
+    if (!aligned16(ws)) return fail(ENT_EINVAL, "workspace pointer not 16-byte aligned");
+    const bool empty = (long long)B * H == 0 || N == 0;
+    if (!empty && (!q || !k || !v || !dout || !tau || !block_mask || !dq || !dk || !dv))
+        return fail(ENT_EINVAL, "null q/k/v/dout/tau/block_mask/dq/dk/dv pointer");
+    if (!empty && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
+                   !aligned16(dq) || !aligned16(dk) || !aligned16(dv)))
+        return fail(ENT_EINVAL, "q/k/v/dout/dq/dk/dv must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace header");
+    if (empty) return ENT_OK;
+
+    ent::BwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.dout = dout; a.tau = tau; a.mask = block_mask;
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    char* base = static_cast<char*>(ws);
+    a.hdr = reinterpret_cast<ent::WsHeader*>(base);
+    a.delta = reinterpret_cast<float*>(base + L.delta);
+    a.dq_acc = reinterpret_cast<float*>(base + L.dq_acc);
+    a.lists = reinterpret_cast<int*>(base + L.lists);
+    a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal;
+    a.alpha = alpha;
+    const int gm = gamma_mode(alpha, &a.gamma);
+    a.scale = 1.f / sqrtf((float)d);
+    a.cx = (alpha - 1.f) * a.scale;
+    e = dtype == ENT_F32 ? ent::simt_bwd_f32(a, d, gm, s) : ent::simt_bwd_bf16(a, d, gm, s);
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return ENT_OK;
+}
+
+ent_status ent_attn_read_status(const void* ws, long long* counters, void* stream) {
+    if (!ws) return fail(ENT_EINVAL, "null workspace");
+    ent::WsHeader h;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the workspace header");
+    if (counters)
+        for (int i = 0; i < 8; ++i) counters[i] = (long long)h.counters[i];
+    if (h.status != 0)
+        return fail(ENT_ETIMEOUT, "a bounded device wait gave up (site %u)", h.timeout_site);
+    return ENT_OK;
+}
+
+}  // extern "C"

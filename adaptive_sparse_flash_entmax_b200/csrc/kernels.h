@@ -1,0 +1,50 @@
+// kernels.h -- host-side launch interface between the C ABI (entattn_api.cu)
+// and the kernel files.  Internal to the library.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include "common.cuh"
+
+namespace ent {
+
+struct FwdArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* o;
+    float* tau;
+    uint8_t* mask;
+    uint8_t* iters;        // nullable
+    WsHeader* hdr;         // workspace header (status, counters)
+    int BH, N, T, causal;
+    float alpha, gamma;    // gamma = 1/(alpha-1)
+    float cx;              // (alpha-1)/sqrt(d): x = cx * (q . k)
+    float scale;           // 1/sqrt(d)
+    float ftol, stol;      // solver stop rule: |f| <= ftol, or a step <= stol*max(1,|tau|)
+};
+
+struct BwdArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* dout;
+    const float* tau;
+    const uint8_t* mask;
+    void* dq;
+    void* dk;
+    void* dv;
+    float* delta;          // workspace [BH*N]
+    float* dq_acc;         // workspace [BH*N*d] fp32 (tensor-core path)
+    int* lists;            // workspace: per-tile / per-block live lists (tensor-core path)
+    WsHeader* hdr;
+    int BH, N, T, causal;
+    float alpha, gamma, cx, scale;
+};
+
+// FP32 CUDA-core path (any dtype; float32 inputs always use it).
+cudaError_t simt_fwd_f32(const FwdArgs& a, int d, int gm, cudaStream_t s);
+cudaError_t simt_fwd_bf16(const FwdArgs& a, int d, int gm, cudaStream_t s);
+cudaError_t simt_bwd_f32(const BwdArgs& a, int d, int gm, cudaStream_t s);
+cudaError_t simt_bwd_bf16(const BwdArgs& a, int d, int gm, cudaStream_t s);
+
+}  // namespace ent

@@ -1,0 +1,363 @@
+#!/usr/bin/env python
+"""Benchmark: fused alpha-entmax attention forward + backward on B200.
+
+One step = one forward and one backward over one batch of the workload
+(default: B4 H16 N4096 d128 bf16, causal, alpha 1.5, beta 1).  Prints one JSON
+line (rank 0).  ``--impl reference`` times the float64 CPU oracle instead, on a
+bounded sample of the same workload, on the host cores.
+
+Multi-GPU (torchrun): every rank runs its own independent batch (heads are
+independent problems; no data-path collective), the step time is the max over
+ranks, and ``value`` counts the work of all ranks (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from adaptive_sparse_flash_entmax_b200 import inputs  # noqa: E402
+
+METRIC = "entmax attn fwd+bwd ms & TFLOP/s (executed, % BF16 peak) vs block sparsity"
+UNIT = "TFLOP/s"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="iid", choices=sorted(inputs.WORKLOADS))
+    p.add_argument("--beta", type=float, default=None)
+    p.add_argument("--alpha", type=float, default=None)
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-heads", type=int, default=24,
+                   help="heads in the oracle sample of the cpu_baseline leg")
+    p.add_argument("--ref-heads-per-step", type=int, default=4,
+                   help="heads per step in the --impl reference arm")
+    return p.parse_args()
+
+
+def workload(args) -> inputs.Workload:
+    w = inputs.WORKLOADS[args.workload]
+    kw = {}
+    if args.beta is not None:
+        kw["beta"] = args.beta
+    if args.alpha is not None:
+        kw["alpha"] = args.alpha
+    return w.replace(**kw) if kw else w
+
+
+def config_of(w, n_gpus, extra=None):
+    c = {"workload": f"{w.name}: B{w.B} H{w.H} N{w.N} d{w.d} {w.dtype} "
+                     f"{'causal' if w.causal else 'non-causal'} alpha={w.alpha} beta={w.beta} "
+                     f"({w.kind} inputs)",
+         "B": w.B, "H": w.H, "N": w.N, "d": w.d, "alpha": w.alpha, "beta": w.beta,
+         "causal": w.causal, "global_batch": w.B * n_gpus, "seq_len": w.N,
+         "parallelism": f"replicas x{n_gpus} (independent batches per GPU)",
+         "l2": "inputs larger than L2: q, k, v, dO = %d MiB per GPU" % (
+             4 * w.B * w.H * w.N * w.d * (2 if w.dtype == 'bf16' else 4) >> 20)}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def dense_flops(w) -> float:
+    """Algorithmic (dense, FlashAttention convention) fwd+bwd flops: 14 B H N^2 d (/2 causal)."""
+    f = 14.0 * w.B * w.H * w.N * w.N * w.d
+    return f / 2 if w.causal else f
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0}, "fallback"
+
+
+# --------------------------------------------------------------------- oracle
+def oracle_sample(w, heads, seed):
+    """Time the oracle (fwd + bwd) on `heads` heads of the workload (host cores)."""
+    import oracle
+    oracle.build()
+    q, k, v, do = inputs.make_inputs(w.replace(B=1, H=max(1, heads)), seed)
+    cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, w.alpha, w.causal, nthreads=cores)
+    oracle.attn_bwd(q, k, v, do, w.alpha, w.causal, nthreads=cores)
+    dt = time.perf_counter() - t0
+    return dt, cores
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = workload(args)
+    heads = args.ref_heads_per_step
+    frac = heads / (w.B * w.H)
+    for _ in range(args.warmup):
+        oracle_sample(w, heads, args.seed)
+    times = []
+    for _ in range(args.steps):
+        dt, cores = oracle_sample(w, heads, args.seed)
+        times.append(dt)
+    tot = sum(times)
+    value = dense_flops(w) * frac * args.steps / tot / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot / args.steps / frac, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, 1, {"extrapolated_from": f"{heads} head(s) per step"}),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"float64 oracle fwd+bwd on {heads} of {w.B * w.H} heads "
+                                       "per step; dense-equivalent flops (14 N^2 d / 2 per head)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------- ours
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from adaptive_sparse_flash_entmax_b200 import attention as A
+    from adaptive_sparse_flash_entmax_b200 import capi
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    capi.load()
+    w = workload(args)
+    B, H, N, d = w.shape
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q, k, v, do = inputs.make_inputs(w, args.seed + rank)
+    host = [torch.from_numpy(a).to(tdt).pin_memory() for a in (q, k, v, do)]
+    qd, kd, vd, dod = (h.to(dev) for h in host)
+    del q, k, v, do
+    dt_code = capi.ENT_BF16 if w.dtype == "bf16" else capi.ENT_F32
+    T = -(-N // 128)
+    o = torch.empty_like(qd)
+    tau = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    mask = torch.empty((B, H, T, T), dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    wsf = A.workspace(capi.ent_attn_fwd_workspace_size(B, H, N, d, dt_code), dev)
+    wsb = A.workspace(capi.ent_attn_bwd_workspace_size(B, H, N, d, dt_code), dev)
+
+    def step():
+        A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, None))
+        A.entmax_attn_bwd(qd, kd, vd, o, dod, tau, mask, w.alpha, w.causal, ws=wsb,
+                          out=(dq, dk, dv))
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    # counters, sparsity and solver passes of one step (untimed)
+    it = torch.empty((B, H, N), dtype=torch.uint8, device=dev)
+    A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, it))
+    cf = A.read_status(wsf)
+    A.entmax_attn_bwd(qd, kd, vd, o, dod, tau, mask, w.alpha, w.causal, ws=wsb, out=(dq, dk, dv))
+    cb = A.read_status(wsb)
+    blk = 2.0 * 128 * 128 * d
+    fwd_flops = blk * (cf[0] + 2 * cf[1])
+    bwd_flops = blk * cb[4]
+    exec_flops = fwd_flops + bwd_flops
+    admissible = B * H * (T * (T + 1) // 2 if w.causal else T * T)
+    live = int(mask.sum().item())
+    iters = it.float()
+
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, None))
+            ev[s][1].record(stream)
+            A.entmax_attn_bwd(qd, kd, vd, o, dod, tau, mask, w.alpha, w.causal, ws=wsb,
+                              out=(dq, dk, dv))
+            ev[s][2].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed = t_start.elapsed_time(t_end)
+    ms_fwd = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    ms_bwd = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step = t.item() / args.steps
+
+    # end to end through the public API from pinned host memory
+    outs_host = [torch.empty(qd.shape, dtype=tdt).pin_memory() for _ in range(4)]
+    h2d = sum(h.numel() * h.element_size() for h in host)
+    d2h = sum(x.numel() * x.element_size() for x in outs_host)
+
+    def e2e_step():
+        qq, kk, vv, dd = (h.to(dev, non_blocking=True) for h in host)
+        oo, tt, mm, _ = A.entmax_attn_fwd(qq, kk, vv, w.alpha, w.causal, ws=wsf)
+        g = A.entmax_attn_bwd(qq, kk, vv, oo, dd, tt, mm, w.alpha, w.causal, ws=wsb)
+        for dst, src in zip(outs_host, (oo,) + tuple(g)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    ms_e2e = te.item()
+
+    peaks, peak_kind = measured_peaks()
+    sm_max = peaks.get("sm_max_mhz", 1965.0)
+    alu_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12   # FP32 FMA, all SMs, max clock
+    fwd_tflops = fwd_flops / (ms_fwd * 1e-3) / 1e12
+    value = world * exec_flops / (ms_step * 1e-3) / 1e12
+    line = None
+    if rank == 0:
+        clocks = clk.summary()
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            heads = min(args.cpu_heads, B * H)
+            dt_cpu, cores = oracle_sample(w, heads, args.seed)
+            frac = heads / (B * H)
+            cpu = {"value": exec_flops * frac / dt_cpu / 1e12, "unit": UNIT, "cores": cores,
+                   "kind": "oracle",
+                   "sample": f"float64 oracle fwd+bwd on {heads} of {B * H} heads of the same "
+                             f"workload ({dt_cpu:.1f} s); value = this workload's executed "
+                             "flops for those heads / oracle time"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if w.dtype == "f32" else "bf16 inputs, f32 accumulate",
+            "data": "synthetic",
+            "config": config_of(w, world),
+            "ms_fwd": ms_fwd, "ms_bwd": ms_bwd,
+            "executed_tflop_per_step": exec_flops / 1e12,
+            "effective_dense_tflops": world * dense_flops(w) / (ms_step * 1e-3) / 1e12,
+            "pct_bf16_peak_executed": 100 * value / world / peaks["bf16_tflops"],
+            "block_sparsity": 1.0 - live / admissible,
+            "tau_passes": {"row_mean": iters.mean().item(), "row_max": int(iters.max().item()),
+                           "tile_mean": cf[2] / max(1, cf[3])},
+            "roofline": {"kernel": "forward (statistics + solver + P.V), FP32 CUDA cores",
+                         "bound": "alu", "achieved": fwd_tflops, "peak": alu_peak,
+                         "unit": "TFLOP/s", "frac": fwd_tflops / alu_peak, "traffic": None,
+                         "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x %.0f MHz" % sm_max},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * exec_flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "peaks": {"source": peak_kind, "bf16_tflops": peaks["bf16_tflops"],
+                      "hbm_gbs": peaks["hbm_gbs"]},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

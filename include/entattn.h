@@ -1,0 +1,130 @@
+/*
+ * entattn.h -- C ABI of the B200 fused alpha-entmax attention library
+ * (libentattn.so).  Forward and backward of
+ *
+ *     s = Q K^T / sqrt(d),   P = alpha-entmax(s) row-wise,   O = P V,
+ *
+ * with alpha-entmax p_j = [(alpha-1) s_j - tau]_+^(1/(alpha-1)), tau such that
+ * sum_j p_j = 1 (support strict: p_j > 0 iff (alpha-1) s_j > tau).
+ *
+ * Defining passages (AdaSplash web pages, by title and section):
+ *  - "AdaSplash: Adaptive Sparse Flash Attention" (ICML 2025 talk summary):
+ *      Background -- alpha-entmax, alpha = 1 softmax, alpha = 2 sparsemax;
+ *      Technical Deep Dive / Accelerated Alpha-Entmax Transformation -- tau as
+ *        the root of f(tau) = 0, Halley-bisection;
+ *      Technical Deep Dive / AdaSplash: Fused GPU Kernel for Attention -- the
+ *        Q tile stays on chip, K tiles stream for the tau passes, a final pass
+ *        streams K and V and accumulates O = P V without materialising S or P;
+ *      Technical Deep Dive / Exploiting Sparsity -- all-zero tiles of P skip
+ *        their K/V loads and compute, in the forward and the backward;
+ *      Experimental Setup & Results / Backward Pass -- the backward skips the
+ *        same zero tiles.
+ *  - "AdaSplash-2: The Transformer Revolution We Didn't See Coming",
+ *      Sparse Attention Makes Waves -- a coarse on-chip histogram of the
+ *      scores starts the tau iteration (typically 1-2 further iterations).
+ *
+ * Conventions shared by every entry point:
+ *  - Tensors are contiguous row-major [B][H][N][d] (q, k, v, o, dout, dq, dk,
+ *    dv), all of one dtype: ENT_F32 (float) or ENT_BF16 (bfloat16 bits).
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    allocates no memory.  Pointers must be 16-byte aligned.
+ *  - The scale is fixed at 1/sqrt(d).  A score temperature beta is applied by
+ *    the caller pre-scaling q.
+ *  - tau is float32 [B][H][N], in units of x = (alpha-1) s (absolute, not
+ *    shifted by the row maximum).
+ *  - block_mask is uint8 [B][H][T][T], T = ceil(N/128): entry (t, b) is 1 iff
+ *    the 128x128 block of P for query tile t and key block b holds a nonzero
+ *    (blocks above the diagonal are 0 when causal).  The forward writes it;
+ *    the backward reads it and skips exactly the 0 blocks.
+ *  - Supported: 1 < alpha <= 2, d in {64, 128}, N >= 1 (any N; the last tile
+ *    may be ragged), B, H >= 0.  B*H == 0 or N == 0 is a no-op returning ENT_OK.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  Argument errors return synchronously before any
+ *    work is enqueued.  No exception crosses the ABI.
+ *  - ws / ws_bytes: caller-owned device workspace of at least the size that
+ *    the matching *_workspace_size() returns.  The library zeroes what it
+ *    needs on `stream`; its first 256 bytes hold a status word and counters
+ *    (see ent_attn_read_status).
+ *  - Device waits are bounded: a wait that gives up sets the status word in
+ *    ws; ent_attn_read_status then reports ENT_ETIMEOUT.
+ */
+#ifndef ENTATTN_H
+#define ENTATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ENT_OK = 0,
+    ENT_EINVAL = 1,        /* a bad argument (null pointer, bad size, alpha out of range) */
+    ENT_EUNSUPPORTED = 2,  /* a valid request this build does not implement (e.g. d = 96) */
+    ENT_ECUDA = 3,         /* a CUDA runtime call failed; see ent_attn_last_error() */
+    ENT_ETIMEOUT = 4       /* a bounded device wait gave up (reported by ent_attn_read_status) */
+} ent_status;
+
+typedef enum { ENT_F32 = 0, ENT_BF16 = 1 } ent_dtype;
+
+/* Query/key tile edge of the block mask (128). */
+int ent_attn_block_size(void);
+
+/* Bytes of device workspace the forward / backward need for this shape. */
+size_t ent_attn_fwd_workspace_size(int B, int H, int N, int d, int dtype);
+size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype);
+
+/*
+ * Forward.  Inputs q, k, v [B,H,N,d].  Outputs: o [B,H,N,d] (same dtype),
+ * tau float [B,H,N], block_mask uint8 [B,H,T,T] (all required) and iters
+ * uint8 [B,H,N] (nullable): the number of tau-solver passes each row took
+ * after the histogram pass.  Per 128-row query tile the kernel runs one
+ * statistics pass (row max and score histogram), solver passes until every
+ * row of the tile has converged, and one P.V pass over the live key blocks.
+ */
+ent_status ent_attn_fwd(const void *q, const void *k, const void *v,
+                        int B, int H, int N, int d, int dtype,
+                        float alpha, int causal,
+                        void *o, float *tau, uint8_t *block_mask, uint8_t *iters,
+                        void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Backward.  Inputs q, k, v, o, dout [B,H,N,d]; tau and block_mask as the
+ * forward wrote them.  Outputs dq, dk, dv [B,H,N,d] (same dtype), computed
+ * with g = (x - tau)_+^(1/(alpha-1) - 1), delta_i = sum_j g_ij dP_ij /
+ * sum_j g_ij, dS = g (dP - delta), dP = dO V^T:
+ *     dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d),  dV = P^T dO,
+ * visiting only blocks whose block_mask entry is 1.  `o` is accepted for
+ * interface symmetry and may be NULL (entmax has no O-based shortcut for
+ * delta; it is recomputed from the live blocks).
+ */
+ent_status ent_attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                        const void *dout, const float *tau, const uint8_t *block_mask,
+                        int B, int H, int N, int d, int dtype, float alpha, int causal,
+                        void *dq, void *dk, void *dv,
+                        void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronises `stream` and reads the status word and the work counters of a
+ * workspace that a forward or backward used.  counters (nullable, 8 entries):
+ *   [0] block products (128x128xd, 2*128*128*d flops each) in the forward's
+ *       statistics and solver passes (one S block per visited block and pass),
+ *   [1] live blocks in the forward P.V pass (two block products each: S, P V),
+ *   [2] solver passes summed over query tiles,
+ *   [3] query tiles processed,
+ *   [4] block products issued by the backward kernels (all of them),
+ *   [5]..[7] reserved (0).
+ * Executed flops of a call = 2*128*128*d * ([0] + 2*[1] + [4]).
+ * Returns ENT_OK, ENT_ETIMEOUT if a bounded wait gave up, ENT_ECUDA on a
+ * CUDA error.
+ */
+ent_status ent_attn_read_status(const void *ws, long long *counters, void *stream);
+
+/* Thread-local message describing the last non-OK status of this thread. */
+const char *ent_attn_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ENTATTN_H */

@@ -527,14 +527,17 @@ int orc_attn_bwd_head_sampled(const double *qh, const double *kh, const double *
  *     F_low(tau) = sum_b c_b (lower_b - tau)_+^gamma - 1 <= f(tau)
  *              <= F_up(tau)  = sum_b c_b (upper_b - tau)_+^gamma - 1.
  * lo = the largest edge with F_low >= 0, hi = the smallest edge with
- * F_up <= 0; both are rigorous.
+ * F_up <= 0; both are rigorous.  The start is the root of the straight line
+ * through the bin-centre model sum_b c_b (centre_b - tau)_+^gamma - 1 at lo and
+ * hi (the pages leave the start open; methods 0 and 1 start at the midpoint).
  *
  * Each pass evaluates f, f' = -gamma sum u^(gamma-1) and
  * f'' = gamma (gamma-1) sum u^(gamma-2) at the current tau (one sweep over
  * the row) and counts as one pass.  Stop when |f| <= ftol or hi-lo <= wtol
  * (tau = the last evaluated point).  Otherwise f > 0 moves lo up, else hi
- * down; the Halley point tau - 2 f f' / (2 f'^2 - f f'') is taken if it lies
- * strictly inside (lo, hi) and is finite, else the midpoint (bisection).
+ * down; the Halley point tau - 2 f f' / (2 f'^2 - f f'') is taken if it is
+ * finite and lies within the bounds [lo, hi] (ends included: the root can sit
+ * on an end, e.g. tau = m - 1 for a one-element support), else the midpoint.
  * Returns 0, or -1 on bad arguments.
  */
 int orc_entmax_tau_iterative(const double *s, int n, double alpha, int method, int nbins,
@@ -547,7 +550,7 @@ int orc_entmax_tau_iterative(const double *s, int n, double alpha, int method, i
     double *x = (double *)malloc(sizeof(double) * (size_t)n);
     double m = -INFINITY;
     for (int j = 0; j < n; ++j) { x[j] = (alpha - 1.0) * s[j]; if (x[j] > m) m = x[j]; }
-    double lo = m - 1.0, hi = m - pow((double)n, 1.0 - alpha);
+    double lo = m - 1.0, hi = m - pow((double)n, 1.0 - alpha), tau0 = 0.0;
 
     if (method == 2) {
         const double w = 1.0 / nbins;
@@ -571,12 +574,24 @@ int orc_entmax_tau_iterative(const double *s, int n, double alpha, int method, i
             if (flow >= 0.0 && e > hlo) hlo = e;
             if (fup <= 0.0 && e < hhi) hhi = e;
         }
-        free(cnt);
         if (hlo > lo) lo = hlo;
         if (hhi < hi) hi = hhi;
+        if (hi < lo) hi = lo;
+        /* start: root of the line through the bin-centre model at lo and hi */
+        double fcl = -1.0, fch = -1.0;
+        for (int b = 0; b < nbins; ++b) {
+            if (!cnt[b]) continue;
+            const double centre = m - 1.0 + (b + 0.5) * w;
+            fcl += cnt[b] * pos_pow(centre - lo, gamma);
+            fch += cnt[b] * pos_pow(centre - hi, gamma);
+        }
+        free(cnt);
+        tau0 = (fcl > 0.0 && fch < 0.0) ? lo + (hi - lo) * fcl / (fcl - fch) : 0.5 * (lo + hi);
+        if (tau0 < lo) tau0 = lo;
+        if (tau0 > hi) tau0 = hi;
     }
 
-    double tau = 0.5 * (lo + hi);
+    double tau = (method == 2) ? tau0 : 0.5 * (lo + hi);
     int passes = 0;
     for (;;) {
         if (hi - lo <= wtol && passes > 0) break;
@@ -597,7 +612,7 @@ int orc_entmax_tau_iterative(const double *s, int n, double alpha, int method, i
             const double fp = -gamma * F1;
             const double fpp = (gamma != 1.0) ? gamma * (gamma - 1.0) * F2 : 0.0;
             const double h = tau - 2.0 * f * fp / (2.0 * fp * fp - f * fpp);
-            if (isfinite(h) && h > lo && h < hi) next = h;
+            if (isfinite(h) && h >= lo && h <= hi) next = h;
         }
         tau = next;
     }

@@ -1,0 +1,92 @@
+"""The C-ABI library on a machine without a GPU: it builds, loads, exports every
+symbol the header declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+
+import pytest
+
+from adaptive_sparse_flash_entmax_b200 import build, capi
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return capi.load()
+
+
+def test_exports_every_header_symbol(lib):
+    names = capi.header_symbols()
+    assert {"ent_attn_fwd", "ent_attn_bwd", "ent_attn_fwd_workspace_size",
+            "ent_attn_bwd_workspace_size", "ent_attn_read_status", "ent_attn_last_error",
+            "ent_attn_block_size"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert ctypes.cast(getattr(lib, n), ctypes.c_void_p).value
+
+
+def test_sizes(lib):
+    assert capi.ent_attn_block_size() == 128
+    assert capi.ent_attn_fwd_workspace_size(4, 16, 4096, 128, capi.ENT_BF16) >= 256
+    B, H, N, d = 4, 16, 4096, 128
+    ws = capi.ent_attn_bwd_workspace_size(B, H, N, d, capi.ENT_BF16)
+    assert ws >= 256 + B * H * N * 4 + B * H * N * d * 4
+
+
+FAKE = 1 << 20   # a 16-byte-aligned non-null value; never dereferenced on argument errors
+
+
+def fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, B=1, H=1, N=128, d=64, dtype=capi.ENT_BF16, alpha=1.5,
+             causal=1, o=FAKE, tau=FAKE, block_mask=FAKE, iters=None, ws=FAKE, ws_bytes=256,
+             stream=None)
+    a.update(kw)
+    return capi.ent_attn_fwd(**a)
+
+
+def bwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=None, dout=FAKE, tau=FAKE, block_mask=FAKE, B=1, H=1,
+             N=128, d=64, dtype=capi.ENT_BF16, alpha=1.5, causal=1, dq=FAKE, dk=FAKE, dv=FAKE,
+             ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return capi.ent_attn_bwd(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(alpha=1.0), capi.ENT_EINVAL),
+    (dict(alpha=2.5), capi.ENT_EINVAL),
+    (dict(alpha=float("nan")), capi.ENT_EINVAL),
+    (dict(d=96), capi.ENT_EUNSUPPORTED),
+    (dict(dtype=7), capi.ENT_EINVAL),
+    (dict(N=-1), capi.ENT_EINVAL),
+    (dict(causal=2), capi.ENT_EINVAL),
+    (dict(q=None), capi.ENT_EINVAL),
+    (dict(o=FAKE + 4), capi.ENT_EINVAL),
+    (dict(ws=None), capi.ENT_EINVAL),
+    (dict(ws_bytes=16), capi.ENT_EINVAL),
+    (dict(N=200000), capi.ENT_EUNSUPPORTED),
+])
+def test_fwd_argument_errors(lib, kw, code):
+    assert fwd(**kw) == code
+    assert capi.ent_attn_last_error()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(alpha=0.5), capi.ENT_EINVAL),
+    (dict(d=32), capi.ENT_EUNSUPPORTED),
+    (dict(tau=None), capi.ENT_EINVAL),
+    (dict(dq=FAKE + 8), capi.ENT_EINVAL),
+    (dict(ws_bytes=1024), capi.ENT_EINVAL),
+])
+def test_bwd_argument_errors(lib, kw, code):
+    assert bwd(**kw) == code
+    assert capi.ent_attn_last_error()
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = capi._lib
+    try:
+        capi._lib = None
+        with pytest.raises(RuntimeError, match="not built"):
+            capi.load(str(tmp_path / "libentattn.so"))
+    finally:
+        capi._lib = saved

@@ -126,7 +126,13 @@ ent_status ent_attn_fwd(const void* q, const void* k, const void* v, int B, int 
     // far below their rounding; float32 outputs get 1e-6.
     a.ftol = dtype == ENT_F32 ? 1e-6f : 1e-5f;
     a.stol = dtype == ENT_F32 ? 4e-7f : 1e-6f;
-    e = dtype == ENT_F32 ? ent::simt_fwd_f32(a, d, gm, s) : ent::simt_fwd_bf16(a, d, gm, s);
+    if (dtype == ENT_F32) {
+        e = ent::simt_fwd_f32(a, d, gm, s);
+    } else {
+        const char* why = nullptr;
+        e = ent::tc_fwd(a, d, gm, s, &why);
+        if (e != cudaSuccess && why) return fail(ENT_ECUDA, "forward launch: %s", why);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "forward launch");
     return ENT_OK;
 }
@@ -167,7 +173,13 @@ ent_status ent_attn_bwd(const void* q, const void* k, const void* v, const void*
     const int gm = gamma_mode(alpha, &a.gamma);
     a.scale = 1.f / sqrtf((float)d);
     a.cx = (alpha - 1.f) * a.scale;
-    e = dtype == ENT_F32 ? ent::simt_bwd_f32(a, d, gm, s) : ent::simt_bwd_bf16(a, d, gm, s);
+    if (dtype == ENT_F32) {
+        e = ent::simt_bwd_f32(a, d, gm, s);
+    } else {
+        const char* why = nullptr;
+        e = ent::tc_bwd(a, d, gm, s, &why);
+        if (e != cudaSuccess && why) return fail(ENT_ECUDA, "backward launch: %s", why);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return ENT_OK;
 }

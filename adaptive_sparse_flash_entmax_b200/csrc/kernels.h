@@ -41,10 +41,12 @@ struct BwdArgs {
     float alpha, gamma, cx, scale;
 };
 
-// FP32 CUDA-core path (any dtype; float32 inputs always use it).
+// FP32 CUDA-core path: float32 inputs (scores by FFMA, no TF32 rounding).
 cudaError_t simt_fwd_f32(const FwdArgs& a, int d, int gm, cudaStream_t s);
-cudaError_t simt_fwd_bf16(const FwdArgs& a, int d, int gm, cudaStream_t s);
 cudaError_t simt_bwd_f32(const BwdArgs& a, int d, int gm, cudaStream_t s);
-cudaError_t simt_bwd_bf16(const BwdArgs& a, int d, int gm, cudaStream_t s);
+
+// bf16 tensor-core path (tcgen05 + TMEM + TMA).  `why` names a host-side failure.
+cudaError_t tc_fwd(const FwdArgs& a, int d, int gm, cudaStream_t s, const char** why);
+cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char** why);
 
 }  // namespace ent

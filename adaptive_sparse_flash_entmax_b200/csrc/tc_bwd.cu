@@ -1,0 +1,638 @@
+// tc_bwd.cu -- the bf16 backward on sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// Entmax Jacobian (derived from the definition; the pages state that the
+// backward skips the zero tiles, "AdaSplash: Adaptive Sparse Flash Attention",
+// Experimental Setup & Results / Backward Pass, and Technical Deep Dive /
+// Exploiting Sparsity): with u = x - tau, g = u^(gamma-1) on u > 0,
+//     delta_i = sum_j g_ij dP_ij / sum_j g_ij,   dS = g (dP - delta),   dP = dO V^T,
+//     dQ = dS K / sqrt(d),   dK = dS^T Q / sqrt(d),   dV = P^T dO.
+// Only the 128 x 128 blocks marked live by the forward's block mask are visited.
+//
+// Two kernels, both with warp roles (warp 0 TMA, warp 1 MMA issuer, warps 2-5
+// elementwise, thread = TMEM lane) and 64-wide sub-tiles so that two stages,
+// double-buffered TMEM accumulators and the bf16 operand written by the
+// elementwise warps fit on chip:
+//   dq kernel   one CTA per 128-row query tile, K/V in 64-key sub-blocks of
+//               the live blocks.  Phase A: S = Q K^T, dP = dO V^T -> delta per
+//               row (also written to the workspace).  Phase B: again S and dP,
+//               dS as a pair of bf16 parts (hi + lo, shared memory) and
+//               dQ += dS K (K read MN-major).
+//   dkv kernel  one CTA per 128-key block, Q/dO in 64-row sub-tiles of the
+//               live query tiles.  S^T = K Q^T, dP^T = V dO^T, then P^T and
+//               dS^T (bf16, shared memory) and dV += P^T dO, dK += dS^T Q (dO
+//               and Q read MN-major from the same tiles that fed S^T and dP^T).
+// All waits are bounded as in the forward.
+#include <cudaTypedefs.h>
+
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace ent {
+using namespace tc;
+
+bool make_tmap_bf16_rows(CUtensorMap* map, const void* base, int BH, int N, int D, int box_rows);
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kEw = 128;
+constexpr int kNst = 2;
+constexpr int kTmemCols = 512;
+constexpr int kSub = 64;                       // sub-tile width (keys or query rows)
+constexpr int kAtom128 = 128 * 128;            // [128 rows x 64 bf16] atom
+constexpr int kAtom64 = 64 * 128;              // [64 rows x 64 bf16] atom
+
+struct Misc {
+    uint32_t tmem_base;
+    int njobs;      // sub-tile jobs per phase
+    int abort;
+    int pad;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Write 64 bf16 values (32 packed words) as one 128-byte row `row` of a
+// K-major 128-byte-swizzled atom starting at `atom`.
+__device__ __forceinline__ void store_row_sw128(uint8_t* atom, int row, const uint32_t* w) {
+    uint8_t* base = atom + row * 128;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<uint4*>(base + ((ch ^ (row & 7)) << 4)) =
+            make_uint4(w[ch * 4], w[ch * 4 + 1], w[ch * 4 + 2], w[ch * 4 + 3]);
+}
+
+__device__ __forceinline__ void store_out_row(void* out, size_t off, const float* v, int D, float sc) {
+    __nv_bfloat16* p = static_cast<__nv_bfloat16*>(out) + off;
+    for (int c = 0; c < D; c += 8) {
+        uint4 val = make_uint4(pack_bf16(v[c] * sc, v[c + 1] * sc), pack_bf16(v[c + 2] * sc, v[c + 3] * sc),
+                               pack_bf16(v[c + 4] * sc, v[c + 5] * sc), pack_bf16(v[c + 6] * sc, v[c + 7] * sc));
+        *reinterpret_cast<uint4*>(p + c) = val;
+    }
+}
+
+}  // namespace
+
+// =========================================================================
+// dq kernel: delta and dQ for one 128-row query tile.
+// =========================================================================
+template <int D>
+struct DqLayout {
+    static constexpr int kTile = D / 64 * kAtom128;     // Q or dO [128 x D]
+    static constexpr int kSubT = D / 64 * kAtom64;      // K or V sub-block [64 x D]
+    static constexpr int kQ = 0;
+    static constexpr int kDO = kQ + kTile;
+    static constexpr int kStage0 = kDO + kTile;
+    static constexpr int kStageBytes = 2 * kSubT;       // K_sub, V_sub
+    static constexpr int kDS = kStage0 + kNst * kStageBytes;   // dS hi, dS lo: [128 x 64] bf16 atoms
+    static constexpr int kBars = kDS + 2 * kAtom128;
+    static constexpr int kMisc = kBars + 8 * 16;
+    static constexpr int kList = kMisc + 16;            // int job list [2*T]
+    static size_t bytes(int T) { return (size_t)kList + 8 * (size_t)T + 1024; }
+};
+
+template <int D, int GM>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v64,
+                 const BwdArgs a) {
+    using L = DqLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+    uint64_t* full = bars;               // [2]
+    uint64_t* empty = bars + 2;          // [2]
+    uint64_t* s_full = bars + 4;         // [2]
+    uint64_t* s_empty = bars + 6;        // [2]
+    uint64_t* ds_full = bars + 8;
+    uint64_t* ds_empty = bars + 9;
+    uint64_t* acc_full = bars + 10;
+    uint64_t* in_full = bars + 11;       // Q and dO tiles
+    uint64_t* mma_done = bars + 12;
+    Misc* misc = reinterpret_cast<Misc*>(smem + L::kMisc);
+    int* jobs = reinterpret_cast<int*>(smem + L::kList);   // key offsets of the 64-key sub-blocks
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = a.T, N = a.N;
+    const int t = a.causal ? (T - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+    const int bh = blockIdx.y;
+    const int nblk = a.causal ? t + 1 : T;
+    const int last_row = min(t * kBlk + kBlk - 1, N - 1);
+    const Abort ab{&misc->abort, a.hdr};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&full[s], 1); mbar_init(&empty[s], 1);
+            mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 4);
+        }
+        mbar_init(ds_full, 4);
+        mbar_init(ds_empty, 1);
+        mbar_init(acc_full, 1);
+        mbar_init(in_full, 1);
+        mbar_init(mma_done, 1);
+        misc->abort = 0;
+        // sub-block list of the live key blocks of this tile
+        const uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
+        int n = 0;
+        for (int b = 0; b < nblk; ++b) {
+            if (!mrow[b]) continue;
+            for (int h = 0; h < 2; ++h) {
+                const int j0 = b * kBlk + h * kSub;
+                if (j0 >= N || (a.causal && j0 > last_row)) continue;
+                jobs[n++] = j0;
+            }
+        }
+        misc->njobs = n;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&misc->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+    const int njobs = misc->njobs;
+    const int total = 2 * njobs;     // phase A then phase B
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tm_q); prefetch_tmap(&tm_do); prefetch_tmap(&tm_k64); prefetch_tmap(&tm_v64);
+            mbar_arrive_expect_tx(in_full, 2 * L::kTile);
+            for (int at = 0; at < D / 64; ++at) {
+                tma_load_3d(smem + L::kQ + at * kAtom128, &tm_q, at * 64, t * kBlk, bh, in_full);
+                tma_load_3d(smem + L::kDO + at * kAtom128, &tm_do, at * 64, t * kBlk, bh, in_full);
+            }
+            int job = 0;
+            bool ok = true;
+            for (; job < total && ok; ++job) {
+                const int j0 = jobs[job % njobs];
+                const int st = job & 1;
+                if (!(ok = mbar_wait(&empty[st], ((job >> 1) & 1) ^ 1, ab, 21))) break;
+                uint8_t* sb = smem + L::kStage0 + st * L::kStageBytes;
+                mbar_arrive_expect_tx(&full[st], 2 * L::kSubT);
+                for (int at = 0; at < D / 64; ++at) {
+                    tma_load_3d(sb + at * kAtom64, &tm_k64, at * 64, j0, bh, &full[st]);
+                    tma_load_3d(sb + L::kSubT + at * kAtom64, &tm_v64, at * 64, j0, bh, &full[st]);
+                }
+            }
+            drain_wait(in_full, 0);
+            for (int j = job - 1; j >= 0 && j >= job - kNst; --j) drain_wait(&full[j & 1], (j >> 1) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16(128, kSub, 0, 0);   // [128 x 64], K = d
+            constexpr uint32_t idesc_dq = idesc_bf16(128, D, 0, 1);     // dQ += dS K, K MN-major
+            const uint32_t qb = smem_u32(smem + L::kQ), dob = smem_u32(smem + L::kDO);
+            const uint32_t dsb = smem_u32(smem + L::kDS);
+            bool ok = mbar_wait(in_full, 0, ab, 22);
+            tc_fence_after();
+            // issue S and dP of job j into TMEM buffer j & 1
+            auto issue_sdp = [&](int j) -> bool {
+                const int st = j & 1, sbuf = j & 1;
+                if (!mbar_wait(&full[st], (j >> 1) & 1, ab, 23)) return false;
+                if (!mbar_wait(&s_empty[sbuf], ((j >> 1) & 1) ^ 1, ab, 24)) return false;
+                tc_fence_after();
+                const uint32_t kb = smem_u32(smem + L::kStage0 + st * L::kStageBytes);
+                const uint32_t vb = kb + L::kSubT;
+                const uint32_t dS = tmem + sbuf * 128, dPc = tmem + sbuf * 128 + 64;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t oa = (kk >> 2) * kAtom128 + (kk & 3) * 32;
+                    const uint32_t ob = (kk >> 2) * kAtom64 + (kk & 3) * 32;
+                    umma_bf16(dS, sdesc_sw128(qb + oa, 16, 1024), sdesc_sw128(kb + ob, 16, 1024), idesc_s, kk > 0);
+                    umma_bf16(dPc, sdesc_sw128(dob + oa, 16, 1024), sdesc_sw128(vb + ob, 16, 1024), idesc_s, kk > 0);
+                }
+                umma_commit(&s_full[sbuf]);
+                return true;
+            };
+            if (ok && total > 0) ok = issue_sdp(0);
+            for (int j = 0; j < total && ok; ++j) {
+                if (j + 1 < total && !(ok = issue_sdp(j + 1))) break;
+                const int st = j & 1;
+                if (j < njobs) {                 // phase A: K/V stage only fed S and dP
+                    umma_commit(&empty[st]);
+                    continue;
+                }
+                const int bj = j - njobs;        // phase B job: dQ += dS K
+                if (!(ok = mbar_wait(ds_full, bj & 1, ab, 25))) break;
+                tc_fence_after();
+                const uint32_t kb = smem_u32(smem + L::kStage0 + st * L::kStageBytes);
+                // dQ += (dS_hi + dS_lo) K: the two bf16 parts carry dS to ~16 bits, which
+                // the cancellation in sum_j dS_ij k_j (rows of dS sum to 0) needs.
+#pragma unroll
+                for (int kk = 0; kk < kSub / 16; ++kk) {
+                    const uint64_t bdesc = sdesc_sw128(kb + kk * 16 * 128, kAtom64, 1024);
+                    umma_bf16(tmem + 256, sdesc_sw128(dsb + kk * 32, 16, 1024), bdesc, idesc_dq,
+                              (bj > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16(tmem + 256, sdesc_sw128(dsb + kAtom128 + kk * 32, 16, 1024), bdesc,
+                              idesc_dq, 1u);
+                }
+                umma_commit(ds_empty);
+                umma_commit(&empty[st]);
+            }
+            if (ok) umma_commit(acc_full);
+            umma_commit(mma_done);
+            drain_wait(mma_done, 0);
+        }
+    } else {
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int i = t * kBlk + row;
+        const bool row_valid = i < N;
+        const int key_end = !row_valid ? 0 : (a.causal ? i + 1 : N);
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const float gamma = a.gamma, cx = a.cx;
+        const float tau = row_valid ? a.tau[(size_t)bh * N + i] : 0.f;
+        float sg = 0.f, sgdp = 0.f, delta = 0.f;
+        bool ok = true;
+        for (int j = 0; j < total && ok; ++j) {
+            const int sbuf = j & 1;
+            if (!(ok = mbar_wait(&s_full[sbuf], (j >> 1) & 1, ab, 26))) break;
+            tc_fence_after();
+            float s[64], dp[64];
+            tmem_ld32(lane_base + sbuf * 128, &s[0]);
+            tmem_ld32(lane_base + sbuf * 128 + 32, &s[32]);
+            tmem_ld32(lane_base + sbuf * 128 + 64, &dp[0]);
+            tmem_ld32(lane_base + sbuf * 128 + 96, &dp[32]);
+            tmem_wait_ld();
+            reg_fence<64>(s);
+            reg_fence<64>(dp);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sbuf]);
+            const int nv = key_end - jobs[j < njobs ? j : j - njobs];
+            if (j < njobs) {
+                float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const float g0 = (c < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c], -tau), gamma) : 0.f;
+                    const float g1 = (c + 1 < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c + 1], -tau), gamma) : 0.f;
+                    a0 += g0; a1 += g1;
+                    b0 = fmaf(g0, dp[c], b0); b1 = fmaf(g1, dp[c + 1], b1);
+                }
+                sg += a0 + a1;
+                sgdp += b0 + b1;
+                if (j == njobs - 1) {
+                    delta = (sg > 0.f) ? sgdp / sg : 0.f;
+                    if (row_valid) a.delta[(size_t)bh * N + i] = delta;
+                }
+            } else {
+                if (njobs == 0) break;
+                uint32_t whi[32], wlo[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const float g0 = (c < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c], -tau), gamma) : 0.f;
+                    const float g1 = (c + 1 < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c + 1], -tau), gamma) : 0.f;
+                    const float d0 = g0 * (dp[c] - delta), d1 = g1 * (dp[c + 1] - delta);
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(d0, d1);
+                    const float2 hf = __bfloat1622float2(h);
+                    whi[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+                    wlo[c >> 1] = pack_bf16(d0 - hf.x, d1 - hf.y);
+                }
+                const int bj = j - njobs;
+                if (!(ok = mbar_wait(ds_empty, (bj & 1) ^ 1, ab, 27))) break;
+                store_row_sw128(smem + L::kDS, row, whi);
+                store_row_sw128(smem + L::kDS + kAtom128, row, wlo);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(ds_full);
+            }
+        }
+        if (njobs == 0 && row_valid) a.delta[(size_t)bh * N + i] = 0.f;
+        float acc[D];
+        if (ok && njobs > 0) {
+            ok = mbar_wait(acc_full, 0, ab, 28);
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + 256 + c * 32, &acc[c * 32]);
+            tmem_wait_ld();
+            reg_fence<D>(acc);
+        } else {
+#pragma unroll
+            for (int c = 0; c < D; ++c) acc[c] = 0.f;
+        }
+        if (row_valid) store_out_row(a.dq, ((size_t)bh * N + i) * D, acc, D, a.scale);
+        if (threadIdx.x == 64)   // block products: phase A S,dP (2) + phase B S,dP,dQ hi,lo (4), per 64-key half
+            atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(3 * njobs));
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// =========================================================================
+// dkv kernel: dK and dV for one 128-key block.
+// =========================================================================
+template <int D>
+struct DkvLayout {
+    static constexpr int kTile = D / 64 * kAtom128;     // K or V block [128 x D]
+    static constexpr int kSubT = D / 64 * kAtom64;      // Q or dO sub-tile [64 x D]
+    static constexpr int kK = 0;
+    static constexpr int kV = kK + kTile;
+    static constexpr int kStage0 = kV + kTile;
+    static constexpr int kStageBytes = 2 * kSubT;       // Q_sub, dO_sub
+    static constexpr int kPT = kStage0 + kNst * kStageBytes;   // P^T [128 keys x 64] bf16: one atom
+    static constexpr int kDST = kPT + kAtom128;                 // dS^T
+    static constexpr int kTauDelta = kDST + kAtom128;           // [2][2][64] floats
+    static constexpr int kBars = kTauDelta + 4 * 64 * 4;
+    static constexpr int kMisc = kBars + 8 * 16;
+    static constexpr int kList = kMisc + 16;
+    static size_t bytes(int T) { return (size_t)kList + 8 * (size_t)T + 1024; }
+};
+
+template <int D, int GM>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_do64,
+                  const BwdArgs a) {
+    using L = DkvLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + 2;
+    uint64_t* s_full = bars + 4;
+    uint64_t* s_empty = bars + 6;
+    uint64_t* p_full = bars + 8;
+    uint64_t* p_empty = bars + 9;
+    uint64_t* acc_full = bars + 10;
+    uint64_t* in_full = bars + 11;
+    uint64_t* mma_done = bars + 12;
+    Misc* misc = reinterpret_cast<Misc*>(smem + L::kMisc);
+    int* jobs = reinterpret_cast<int*>(smem + L::kList);   // row offsets of the 64-row sub-tiles
+    float* td = reinterpret_cast<float*>(smem + L::kTauDelta);   // [buf][tau|delta][64]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = a.T, N = a.N;
+    const int b = blockIdx.x;
+    const int bh = blockIdx.y;
+    const Abort ab{&misc->abort, a.hdr};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&full[s], 1); mbar_init(&empty[s], 1);
+            mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 4);
+        }
+        mbar_init(p_full, 4);
+        mbar_init(p_empty, 1);
+        mbar_init(acc_full, 1);
+        mbar_init(in_full, 1);
+        mbar_init(mma_done, 1);
+        misc->abort = 0;
+        int n = 0;
+        for (int t = a.causal ? b : 0; t < T; ++t) {
+            if (!a.mask[((size_t)bh * T + t) * T + b]) continue;
+            for (int h = 0; h < 2; ++h) {
+                const int i0 = t * kBlk + h * kSub;
+                if (i0 >= N || (a.causal && i0 + kSub - 1 < b * kBlk)) continue;
+                jobs[n++] = i0;
+            }
+        }
+        misc->njobs = n;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&misc->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc->tmem_base;
+    const int njobs = misc->njobs;
+    const uint32_t tm_dv = tmem + 256, tm_dk = tmem + 256 + D;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_q64); prefetch_tmap(&tm_do64);
+            mbar_arrive_expect_tx(in_full, 2 * L::kTile);
+            for (int at = 0; at < D / 64; ++at) {
+                tma_load_3d(smem + L::kK + at * kAtom128, &tm_k, at * 64, b * kBlk, bh, in_full);
+                tma_load_3d(smem + L::kV + at * kAtom128, &tm_v, at * 64, b * kBlk, bh, in_full);
+            }
+            int job = 0;
+            bool ok = true;
+            for (; job < njobs && ok; ++job) {
+                const int i0 = jobs[job];
+                const int st = job & 1;
+                if (!(ok = mbar_wait(&empty[st], ((job >> 1) & 1) ^ 1, ab, 31))) break;
+                uint8_t* sb = smem + L::kStage0 + st * L::kStageBytes;
+                mbar_arrive_expect_tx(&full[st], 2 * L::kSubT);
+                for (int at = 0; at < D / 64; ++at) {
+                    tma_load_3d(sb + at * kAtom64, &tm_q64, at * 64, i0, bh, &full[st]);
+                    tma_load_3d(sb + L::kSubT + at * kAtom64, &tm_do64, at * 64, i0, bh, &full[st]);
+                }
+            }
+            drain_wait(in_full, 0);
+            for (int j = job - 1; j >= 0 && j >= job - kNst; --j) drain_wait(&full[j & 1], (j >> 1) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16(128, kSub, 0, 0);   // S^T, dP^T [128 keys x 64]
+            constexpr uint32_t idesc_acc = idesc_bf16(128, D, 0, 1);    // dV, dK: B (dO, Q) MN-major
+            const uint32_t kb = smem_u32(smem + L::kK), vb = smem_u32(smem + L::kV);
+            const uint32_t ptb = smem_u32(smem + L::kPT), dstb = smem_u32(smem + L::kDST);
+            bool ok = mbar_wait(in_full, 0, ab, 32);
+            tc_fence_after();
+            auto issue_sdp = [&](int j) -> bool {
+                const int st = j & 1, sbuf = j & 1;
+                if (!mbar_wait(&full[st], (j >> 1) & 1, ab, 33)) return false;
+                if (!mbar_wait(&s_empty[sbuf], ((j >> 1) & 1) ^ 1, ab, 34)) return false;
+                tc_fence_after();
+                const uint32_t qs = smem_u32(smem + L::kStage0 + st * L::kStageBytes);
+                const uint32_t dos = qs + L::kSubT;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t oa = (kk >> 2) * kAtom128 + (kk & 3) * 32;
+                    const uint32_t ob = (kk >> 2) * kAtom64 + (kk & 3) * 32;
+                    umma_bf16(tmem + sbuf * 128, sdesc_sw128(kb + oa, 16, 1024),
+                              sdesc_sw128(qs + ob, 16, 1024), idesc_s, kk > 0);
+                    umma_bf16(tmem + sbuf * 128 + 64, sdesc_sw128(vb + oa, 16, 1024),
+                              sdesc_sw128(dos + ob, 16, 1024), idesc_s, kk > 0);
+                }
+                umma_commit(&s_full[sbuf]);
+                return true;
+            };
+            if (ok && njobs > 0) ok = issue_sdp(0);
+            for (int j = 0; j < njobs && ok; ++j) {
+                if (j + 1 < njobs && !(ok = issue_sdp(j + 1))) break;
+                if (!(ok = mbar_wait(p_full, j & 1, ab, 35))) break;
+                tc_fence_after();
+                const int st = j & 1;
+                const uint32_t qs = smem_u32(smem + L::kStage0 + st * L::kStageBytes);
+                const uint32_t dos = qs + L::kSubT;
+#pragma unroll
+                for (int kk = 0; kk < kSub / 16; ++kk) {
+                    const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+                    umma_bf16(tm_dv, sdesc_sw128(ptb + kk * 32, 16, 1024),
+                              sdesc_sw128(dos + kk * 16 * 128, kAtom64, 1024), idesc_acc, acc);
+                    umma_bf16(tm_dk, sdesc_sw128(dstb + kk * 32, 16, 1024),
+                              sdesc_sw128(qs + kk * 16 * 128, kAtom64, 1024), idesc_acc, acc);
+                }
+                umma_commit(p_empty);
+                umma_commit(&empty[st]);
+            }
+            if (ok) umma_commit(acc_full);
+            umma_commit(mma_done);
+            drain_wait(mma_done, 0);
+        }
+    } else {
+        const int ew = threadIdx.x - 64;
+        const int quarter = warp & 3;
+        const int krow = quarter * 32 + lane;         // key row == TMEM lane
+        const int jkey = b * kBlk + krow;
+        const bool key_valid = jkey < N;
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const float gamma = a.gamma, cx = a.cx;
+        bool ok = true;
+        for (int j = 0; j < njobs && ok; ++j) {
+            const int i0 = jobs[j];
+            float* tdb = td + (j & 1) * 128;
+            if (ew < 64) {
+                const int ii = i0 + ew;
+                tdb[ew] = ii < N ? a.tau[(size_t)bh * N + ii] : 0.f;
+                tdb[64 + ew] = ii < N ? a.delta[(size_t)bh * N + ii] : 0.f;
+            }
+            named_bar(1, kEw);
+            const int sbuf = j & 1;
+            if (!(ok = mbar_wait(&s_full[sbuf], (j >> 1) & 1, ab, 36))) break;
+            tc_fence_after();
+            float s[64], dp[64];
+            tmem_ld32(lane_base + sbuf * 128, &s[0]);
+            tmem_ld32(lane_base + sbuf * 128 + 32, &s[32]);
+            tmem_ld32(lane_base + sbuf * 128 + 64, &dp[0]);
+            tmem_ld32(lane_base + sbuf * 128 + 96, &dp[32]);
+            tmem_wait_ld();
+            reg_fence<64>(s);
+            reg_fence<64>(dp);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sbuf]);
+            // column c is query i0 + c: admissible iff i < N, key valid, and key <= i if causal
+            const int cmin = a.causal ? jkey - i0 : 0;       // c >= cmin
+            const int cmax = min(kSub, N - i0);              // c < cmax
+            uint32_t wp[32], wd[32];
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+                float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
+                if (key_valid && c >= cmin && c < cmax) {
+                    const float u = __fmaf_rn(cx, s[c], -tdb[c]);
+                    p0 = entmax_p<GM>(u, gamma);
+                    d0 = entmax_g<GM>(u, gamma) * (dp[c] - tdb[64 + c]);
+                }
+                if (key_valid && c + 1 >= cmin && c + 1 < cmax) {
+                    const float u = __fmaf_rn(cx, s[c + 1], -tdb[c + 1]);
+                    p1 = entmax_p<GM>(u, gamma);
+                    d1 = entmax_g<GM>(u, gamma) * (dp[c + 1] - tdb[64 + c + 1]);
+                }
+                wp[c >> 1] = pack_bf16(p0, p1);
+                wd[c >> 1] = pack_bf16(d0, d1);
+            }
+            if (!(ok = mbar_wait(p_empty, (j & 1) ^ 1, ab, 37))) break;
+            store_row_sw128(smem + L::kPT, krow, wp);
+            store_row_sw128(smem + L::kDST, krow, wd);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        float acc[D];
+        if (ok && njobs > 0) {
+            ok = mbar_wait(acc_full, 0, ab, 38);
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) tmem_ld32(tm_dv + ((uint32_t)(quarter * 32) << 16) + c * 32, &acc[c * 32]);
+            tmem_wait_ld();
+            reg_fence<D>(acc);
+        } else {
+#pragma unroll
+            for (int c = 0; c < D; ++c) acc[c] = 0.f;
+        }
+        if (key_valid) store_out_row(a.dv, ((size_t)bh * N + jkey) * D, acc, D, 1.f);
+        if (ok && njobs > 0) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) tmem_ld32(tm_dk + ((uint32_t)(quarter * 32) << 16) + c * 32, &acc[c * 32]);
+            tmem_wait_ld();
+            reg_fence<D>(acc);
+        }
+        if (key_valid) store_out_row(a.dk, ((size_t)bh * N + jkey) * D, acc, D, a.scale);
+        if (ew == 0)   // block products: S^T, dP^T, dV, dK (4) per 64-row half
+            atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(2 * njobs));
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+template <int D, int GM>
+static cudaError_t launch_tc_bwd(const BwdArgs& a, cudaStream_t s, const CUtensorMap* m) {
+    // m: q128, do128, k64, v64, k128, v128, q64, do64
+    {
+        const size_t sm = DqLayout<D>::bytes(a.T);
+        auto kern = tc_bwd_dq_kernel<D, GM>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(m[0], m[1], m[2], m[3], a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    const size_t sm = DkvLayout<D>::bytes(a.T);
+    auto kern = tc_bwd_dkv_kernel<D, GM>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(m[4], m[5], m[6], m[7], a);
+    return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t tc_bwd_d(const BwdArgs& a, int gm, cudaStream_t s, const CUtensorMap* m) {
+    switch (gm) {
+        case 1: return launch_tc_bwd<D, 1>(a, s, m);
+        case 2: return launch_tc_bwd<D, 2>(a, s, m);
+        case 4: return launch_tc_bwd<D, 4>(a, s, m);
+        default: return launch_tc_bwd<D, 0>(a, s, m);
+    }
+}
+
+cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char** why) {
+    CUtensorMap m[8];
+    const bool ok = make_tmap_bf16_rows(&m[0], a.q, a.BH, a.N, d, 128) &&
+                    make_tmap_bf16_rows(&m[1], a.dout, a.BH, a.N, d, 128) &&
+                    make_tmap_bf16_rows(&m[2], a.k, a.BH, a.N, d, 64) &&
+                    make_tmap_bf16_rows(&m[3], a.v, a.BH, a.N, d, 64) &&
+                    make_tmap_bf16_rows(&m[4], a.k, a.BH, a.N, d, 128) &&
+                    make_tmap_bf16_rows(&m[5], a.v, a.BH, a.N, d, 128) &&
+                    make_tmap_bf16_rows(&m[6], a.q, a.BH, a.N, d, 64) &&
+                    make_tmap_bf16_rows(&m[7], a.dout, a.BH, a.N, d, 64);
+    if (!ok) {
+        *why = "cuTensorMapEncodeTiled failed";
+        return cudaErrorInvalidValue;
+    }
+    return d == 64 ? tc_bwd_d<64>(a, gm, s, m) : tc_bwd_d<128>(a, gm, s, m);
+}
+
+}  // namespace ent

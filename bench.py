@@ -42,6 +42,8 @@ def parse():
     p.add_argument("--beta", type=float, default=None)
     p.add_argument("--alpha", type=float, default=None)
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--B", type=int, default=None, help="override the batch (profiling cases)")
+    p.add_argument("--H", type=int, default=None, help="override the head count")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-heads", type=int, default=24,
@@ -58,6 +60,10 @@ def workload(args) -> inputs.Workload:
         kw["beta"] = args.beta
     if args.alpha is not None:
         kw["alpha"] = args.alpha
+    if args.B is not None:
+        kw["B"] = args.B
+    if args.H is not None:
+        kw["H"] = args.H
     return w.replace(**kw) if kw else w
 
 
@@ -146,6 +152,31 @@ def measured_peaks():
     except (OSError, ValueError):
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                 "sm_max_mhz": 1965.0}, "fallback"
+
+
+def profiled_traffic(w, kernel):
+    """DRAM bytes per launch of `kernel` on this workload from the committed ncu
+    summary (profiles/traffic.json), or None when the kernel source changed since
+    the capture (the summary stores a hash of the source file)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    for r in rec.get("captures", []):
+        if r.get("kernel") != kernel or r.get("workload") != w.name:
+            continue
+        if any(r.get(k) != getattr(w, k) for k in ("B", "H", "N", "d", "alpha", "beta")):
+            continue
+        src = os.path.join(ROOT, r["source"])
+        try:
+            digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        except OSError:
+            return None
+        if digest == r.get("sha256"):
+            return r["dram_bytes_per_launch"]
+    return None
 
 
 # --------------------------------------------------------------------- oracle
@@ -302,8 +333,24 @@ def run_ours(args):
 
     peaks, peak_kind = measured_peaks()
     sm_max = peaks.get("sm_max_mhz", 1965.0)
-    alu_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12   # FP32 FMA, all SMs, max clock
     fwd_tflops = fwd_flops / (ms_fwd * 1e-3) / 1e12
+    if w.dtype == "bf16":
+        # tcgen05 forward: executed MMA flops against the sustained bf16 tensor peak
+        # (the kernel is timed inside a long step)
+        roof = {"kernel": "tc_fwd_kernel: statistics + solver + P.V passes (tcgen05/TMEM/TMA)",
+                "bound": "tensor", "achieved": fwd_tflops,
+                "peak": peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
+                "unit": "TFLOP/s",
+                "peak_source": f"{peak_kind} bf16_tflops_sustained"}
+        launches = 3    # forward + two backward kernels
+    else:
+        alu_peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12   # FP32 FMA, all SMs, max clock
+        roof = {"kernel": "simt_fwd_kernel: FP32 CUDA-core forward", "bound": "alu",
+                "achieved": fwd_tflops, "peak": alu_peak, "unit": "TFLOP/s",
+                "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x %.0f MHz" % sm_max}
+        launches = 4    # forward + three backward kernels
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = profiled_traffic(w, roof["kernel"].split(":")[0])
     value = world * exec_flops / (ms_step * 1e-3) / 1e12
     line = None
     if rank == 0:
@@ -332,14 +379,11 @@ def run_ours(args):
             "block_sparsity": 1.0 - live / admissible,
             "tau_passes": {"row_mean": iters.mean().item(), "row_max": int(iters.max().item()),
                            "tile_mean": cf[2] / max(1, cf[3])},
-            "roofline": {"kernel": "forward (statistics + solver + P.V), FP32 CUDA cores",
-                         "bound": "alu", "achieved": fwd_tflops, "peak": alu_peak,
-                         "unit": "TFLOP/s", "frac": fwd_tflops / alu_peak, "traffic": None,
-                         "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x %.0f MHz" % sm_max},
+            "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": world * exec_flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": launches * args.steps,
             "clocks": clocks,
             "peaks": {"source": peak_kind, "bf16_tflops": peaks["bf16_tflops"],
                       "hbm_gbs": peaks["hbm_gbs"]},

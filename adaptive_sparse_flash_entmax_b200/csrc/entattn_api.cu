@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "../../include/entattn.h"
@@ -199,3 +200,99 @@ ent_status ent_attn_read_status(const void* ws, long long* counters, void* strea
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward with library-owned scratch (no workspace argument).
+//
+// Some callers cannot call cudaMalloc at the point where they run the
+// backward: serving and training stacks that plan all device memory up front
+// and treat any later allocation as an error (a cudaMalloc may synchronise the
+// device and fragments a pre-sized pool), and plain-C callers with no device
+// allocator of their own.  For them the backward's scratch (a 256-byte status
+// and counter header plus delta, one float per query row) lives in the
+// fixed-size array below, compiled into the library.  Every GPU that loads the
+// library holds this array until the process exits.
+namespace {
+
+constexpr size_t kFixedScratchBytes = size_t(4) << 20;   // 4 MiB: header + 1,048,512 rows of delta
+constexpr int kMaxScratchDevices = 64;
+
+static __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
+
+std::mutex g_fixed_scratch_mu;
+void* g_fixed_scratch_addr[kMaxScratchDevices] = {};
+
+// Device address of g_fixed_scratch on the current device.  The first call on
+// a device looks it up with cudaGetSymbolAddress (the host-side name is only a
+// stand-in, never a device address) and caches it.
+cudaError_t fixed_scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_fixed_scratch_mu);
+    if (!g_fixed_scratch_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_fixed_scratch);
+        if (e != cudaSuccess) return e;
+        g_fixed_scratch_addr[dev] = p;
+    }
+    *out = g_fixed_scratch_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" ent_status ent_attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                                           const void* o, const void* dout, const float* tau,
+                                           const uint8_t* block_mask, int B, int H, int N, int d,
+                                           int dtype, float alpha, int causal, void* dq, void* dk,
+                                           void* dv, void* stream) {
+    (void)o;
+    ent_status st = check_common(B, H, N, d, dtype, alpha, causal);
+    if (st != ENT_OK) return st;
+    const bool empty = (long long)B * H == 0 || N == 0;
+    const size_t need = kHdr + round_up((size_t)B * H * N * sizeof(float), 256);
+    if (need > kFixedScratchBytes)
+        return fail(ENT_EUNSUPPORTED,
+                    "ent_attn_bwd_noalloc: B*H*N = %lld rows exceed the %zu rows its fixed "
+                    "scratch holds; use ent_attn_bwd with a workspace",
+                    (long long)B * H * N, (kFixedScratchBytes - kHdr) / sizeof(float));
+    if (!empty && (!q || !k || !v || !dout || !tau || !block_mask || !dq || !dk || !dv))
+        return fail(ENT_EINVAL, "null q/k/v/dout/tau/block_mask/dq/dk/dv pointer");
+    if (!empty && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
+                   !aligned16(dq) || !aligned16(dk) || !aligned16(dv)))
+        return fail(ENT_EINVAL, "q/k/v/dout/dq/dk/dv must be 16-byte aligned");
+    void* base = nullptr;
+    cudaError_t e = fixed_scratch_address(&base);
+    if (e != cudaSuccess) return cuda_fail(e, "looking up the fixed scratch address");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // The scratch keeps the previous call's contents: the header (status and
+    // counters) must start at zero; delta is fully rewritten before it is read.
+    e = cudaMemsetAsync(base, 0, kHdr, s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the fixed scratch header");
+    if (empty) return ENT_OK;
+
+    ent::BwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.dout = dout; a.tau = tau; a.mask = block_mask;
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    char* b = static_cast<char*>(base);
+    a.hdr = reinterpret_cast<ent::WsHeader*>(b);
+    a.delta = reinterpret_cast<float*>(b + kHdr);
+    a.dq_acc = nullptr;
+    a.lists = nullptr;
+    a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal;
+    a.alpha = alpha;
+    const int gm = gamma_mode(alpha, &a.gamma);
+    a.scale = 1.f / sqrtf((float)d);
+    a.cx = (alpha - 1.f) * a.scale;
+    if (dtype == ENT_F32) {
+        e = ent::simt_bwd_f32(a, d, gm, s);
+    } else {
+        const char* why = nullptr;
+        e = ent::tc_bwd(a, d, gm, s, &why);
+        if (e != cudaSuccess && why) return fail(ENT_ECUDA, "backward launch: %s", why);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return ENT_OK;
+}

@@ -106,6 +106,35 @@ ent_status ent_attn_bwd(const void *q, const void *k, const void *v, const void 
                         void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Backward without a workspace argument.  The pages have no counterpart: this
+ * is a library convenience.  It computes exactly what ent_attn_bwd computes
+ * (same kernels, same arguments minus ws / ws_bytes) for callers that cannot
+ * allocate device memory when they run the backward -- stacks that plan all
+ * device memory ahead of time and forbid later cudaMalloc calls (an
+ * allocation can synchronise the device and fragments a fixed pool), or plain
+ * C code with no device allocator to size and own a workspace.
+ *  - Scratch: a fixed 4 MiB device array inside the library (a 256-byte header
+ *    plus one float per query row), held on every GPU that loads the library
+ *    until the process exits.  B*H*N above 1,048,512 rows returns
+ *    ENT_EUNSUPPORTED with a message; use ent_attn_bwd then.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *    first call before any stream capture.
+ *  - All calls share the one array, and it keeps the previous call's contents
+ *    (the call clears the header itself): calls whose work overlaps on the GPU
+ *    (concurrent streams, or other host threads) race and must be ordered by
+ *    the caller.
+ *  - A bounded device wait that gives up is not reported (there is no
+ *    workspace to pass to ent_attn_read_status); use ent_attn_bwd when the
+ *    timeout status is needed.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+ent_status ent_attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                                const void *dout, const float *tau, const uint8_t *block_mask,
+                                int B, int H, int N, int d, int dtype, float alpha, int causal,
+                                void *dq, void *dk, void *dv, void *stream);
+
+/*
  * Synchronises `stream` and reads the status word and the work counters of a
  * workspace that a forward or backward used.  counters (nullable, 8 entries):
  *   [0] block products (128x128xd, 2*128*128*d flops each) in the forward's

@@ -147,16 +147,17 @@ __device__ __forceinline__ void hist_slide(unsigned int* hist, int stride, int A
 // assignment and intersected with the plain bracket [m-1, m - n^(1-alpha)].
 // tau_0 is the root of the straight line through the bin-centre model
 // F_c(E) = sum_a c_a ((a+1/2)/63 - E)_+^gamma - 1 at E = lo and E = hi.
-template <int GM>
-__device__ __forceinline__ void hist_start(const unsigned int* hist, int stride, int A, float m,
-                                           int n, float alpha, float gamma, const float* ptab,
-                                           float& lo, float& hi, float& tau0) {
+// `count(a)` returns the number of elements in absolute bin a (a in [A-63, A]).
+template <int GM, typename CountFn>
+__device__ __forceinline__ void hist_start_fn(CountFn count, int A, float m, int n, float alpha,
+                                              float gamma, const float* ptab, float& lo, float& hi,
+                                              float& tau0) {
     int h_ok = A + 1;
     int l_ok = kNoBin;
     for (int e = A; e >= A - (kBins - 1); --e) {
         float fu = -1.f, fl = -1.f;
         for (int a = e; a <= A; ++a) {
-            const float c = (float)hist[(a & (kBins - 1)) * stride];
+            const float c = (float)count(a);
             fu = fmaf(c, ptab[a + 1 - e], fu);
             fl = fmaf(c, ptab[a - e], fl);
         }
@@ -172,7 +173,7 @@ __device__ __forceinline__ void hist_start(const unsigned int* hist, int stride,
     float fcl = -1.f, fch = -1.f;
     for (int k = 0; k < kBins; ++k) {
         const int a = A - k;
-        const unsigned int c = hist[(a & (kBins - 1)) * stride];
+        const unsigned int c = count(a);
         if (c) {
             const float centre = ((float)a + 0.5f) / kBinsPerUnit;
             fcl = fmaf((float)c, entmax_p<GM>(centre - lo, gamma), fcl);
@@ -182,6 +183,44 @@ __device__ __forceinline__ void hist_start(const unsigned int* hist, int stride,
     float t0 = 0.5f * (lo + hi);
     if (fcl > 0.f && fch < 0.f) t0 = lo + (hi - lo) * (fcl / (fcl - fch));
     tau0 = fminf(fmaxf(t0, lo), hi);
+}
+
+// Single histogram with slots hist[(a & 63) * stride].
+template <int GM>
+__device__ __forceinline__ void hist_start(const unsigned int* hist, int stride, int A, float m,
+                                           int n, float alpha, float gamma, const float* ptab,
+                                           float& lo, float& hi, float& tau0) {
+    hist_start_fn<GM>([&](int a) { return hist[(a & (kBins - 1)) * stride]; }, A, m, n, alpha,
+                      gamma, ptab, lo, hi, tau0);
+}
+
+// Branch-free power terms for the streaming passes: u <= 0 gives zeros through
+// max(u, 0) and selects instead of branches.
+template <int GM>
+__device__ __forceinline__ void entmax_terms_bf(float u, float gamma, float& t0, float& t1,
+                                                float& t2) {
+    const float up = fmaxf(u, 0.f);
+    if (GM == 1) { t0 = up; t1 = (u > 0.f) ? 1.f : 0.f; t2 = 0.f; }
+    else if (GM == 2) { t0 = up * up; t1 = up; t2 = (u > 0.f) ? 1.f : 0.f; }
+    else if (GM == 3) { t2 = up; t1 = up * up; t0 = t1 * up; }
+    else if (GM == 4) { t2 = up * up; t1 = t2 * up; t0 = t2 * t2; }
+    else {
+        const float l = __log2f(up);                      // -inf at up = 0
+        const float v = exp2f((gamma - 2.f) * l);         // inf at up = 0 when gamma < 2
+        t2 = (u > 0.f) ? v : 0.f;
+        t1 = t2 * up;
+        t0 = t1 * up;
+    }
+}
+
+template <int GM>
+__device__ __forceinline__ float entmax_p_bf(float u, float gamma) {
+    const float up = fmaxf(u, 0.f);
+    if (GM == 1) return up;
+    if (GM == 2) return up * up;
+    if (GM == 3) return up * up * up;
+    if (GM == 4) { const float u2 = up * up; return u2 * u2; }
+    return exp2f(gamma * __log2f(up));                    // 0 at up = 0 (gamma > 0)
 }
 
 }  // namespace ent

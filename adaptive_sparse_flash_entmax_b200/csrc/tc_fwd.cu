@@ -8,7 +8,8 @@
 //            two-stage ring;
 //   warp 1   MMA issuer: S = Q K^T into a double-buffered TMEM accumulator
 //            (128 x 128 fp32), and O += P V (P from shared memory, V MN-major);
-//   warps 2-5 elementwise: thread = query row = TMEM lane.  Pass 0 builds the
+//   warps 2-9 elementwise: two threads per query row (= TMEM lane), 64 columns
+//            each.  Pass 0 builds the
 //            row max and the sliding 64-bin histogram ("AdaSplash-2: ...",
 //            Sparse Attention Makes Waves); solver passes accumulate
 //            F0, F1, F2 and take a Halley-bisection step (Accelerated Alpha-Entmax
@@ -30,8 +31,9 @@ using namespace tc;
 namespace {
 
 constexpr int kNst = 2;            // K/V ring stages
-constexpr int kThreads = 192;      // 6 warps
-constexpr int kEw = 128;           // elementwise threads (warps 2-5)
+constexpr int kThreads = 320;      // 10 warps
+constexpr int kEw = 256;           // elementwise threads (warps 2-9): two per query row
+constexpr int kEwWarps = 8;
 constexpr int kAtom = 128 * 128;   // bytes of a [128 rows x 64 bf16] swizzled atom
 constexpr int kTmemCols = 512;     // S0 [0,128), S1 [128,256), O [256, 256+D)
 constexpr int kDecSolve = 1, kDecPv = 2;
@@ -43,8 +45,14 @@ struct Layout {
     static constexpr int kStage0 = kQ + kTile;
     static constexpr int kStageBytes = 2 * kTile;         // K, then V
     static constexpr int kP = kStage0 + kNst * kStageBytes;
-    static constexpr int kPBytes = 2 * kAtom;             // P [128 x 128] bf16, or hist [64][128] u32
-    static constexpr int kBars = kP + kPBytes;
+    static constexpr int kPBytes = 2 * kAtom;             // P [128 x 128] bf16
+    // Row histograms ([64 slots][128 rows] u32 per column half) live in memory that
+    // is idle during the score passes: the V halves of the two stages when they
+    // are 32 KB (D = 128), else P and a region of their own.
+    static constexpr int kHist0 = (D == 128) ? kStage0 + kTile : kP;
+    static constexpr int kHist1 = (D == 128) ? kStage0 + kStageBytes + kTile : kP + kPBytes;
+    static constexpr int kXch = (D == 128) ? kP + kPBytes : kP + 2 * kPBytes;   // [4][2][128] f32
+    static constexpr int kBars = kXch + 4 * 2 * 128 * 4;
     static constexpr int kNumBars = 16;
     static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, decision, nlive, abort
     static constexpr int kPtab = kMisc + 16;              // 68 floats
@@ -105,8 +113,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kNst; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 4); }
-        mbar_init(p_full, 4);
+        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps); }
+        mbar_init(p_full, kEwWarps);
         mbar_init(p_empty, 1);
         mbar_init(o_full, 1);
         mbar_init(q_full, 1);
@@ -225,17 +233,24 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
     } else {
         // ------------------------------------------------------------ elementwise
-        const int ew = threadIdx.x - 64;          // 0..127
+        // Two threads per query row: `half` selects columns [64*half, 64*half + 64)
+        // of every 128-key block.  Row state (tau, bracket) is kept identically in
+        // both; per-pass partial sums are combined through shared memory.
+        const int ew = threadIdx.x - 64;          // 0..255
+        const int half = ew >> 7;
         const int quarter = warp & 3;             // TMEM lane quarter of this warp
         const int row = quarter * 32 + lane;      // tile row == TMEM lane
+        const int c0 = half * 64;                 // first column of this thread
         const int i = t * kBlk + row;
         const bool row_valid = i < N;
         const int key_end = !row_valid ? 0 : (a.causal ? i + 1 : N);
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const float gamma = a.gamma, cx = a.cx;
-        unsigned int* hist = reinterpret_cast<unsigned int*>(smem + L::kP) + row;   // stride 128
+        unsigned int* hist = reinterpret_cast<unsigned int*>(smem + (half ? L::kHist1 : L::kHist0)) + row;
+        float* xch = reinterpret_cast<float*>(smem + L::kXch);   // [k][half][row]
+        auto X = [&](int k, int h) -> float& { return xch[(k * 2 + h) * 128 + row]; };
         if (ew < 65) ptab[ew] = entmax_p<GM>((float)ew / kBinsPerUnit, gamma);
-        for (int s = 0; s < kBins; ++s) hist[s * 128] = 0u;
+        for (int sl = 0; sl < kBins; ++sl) hist[sl * 128] = 0u;
         named_bar(1, kEw);
 
         float m = -INFINITY;
@@ -249,80 +264,104 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (;; ++pass) {
             float F0 = 0.f, F1 = 0.f, F2 = 0.f;
             if (pass > 0) {
-                for (int b = ew; b < nblk; b += kEw) live[b] = 0;
+                for (int bb = ew; bb < nblk; bb += kEw) live[bb] = 0;
                 named_bar(1, kEw);
             }
             for (int b = 0; b < nblk; ++b, ++job) {
                 const int sb = job & 1;
                 if (!(ok = mbar_wait(&s_full[sb], (job >> 1) & 1, ab, 8))) break;
                 tc_fence_after();
-                float s[128];
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    tmem_ld32(lane_base + sb * 128 + c * 32, &s[c * 32]);
+                float s[64];
+                tmem_ld32(lane_base + sb * 128 + c0, &s[0]);
+                tmem_ld32(lane_base + sb * 128 + c0 + 32, &s[32]);
                 tmem_wait_ld();
-                reg_fence<128>(s);
+                reg_fence<64>(s);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_empty[sb]);
-                const int nv = key_end - b * kBlk;   // valid columns: c < nv
+                const int nv = key_end - b * kBlk - c0;   // valid columns of this thread: c < nv
+                const bool full_blk = __all_sync(0xffffffffu, nv >= 64);
+                if (!full_blk) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
+                }
                 if (pass == 0) {
-                    if (nv > 0) {
-                        float bm = -INFINITY;
+                    float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-                        for (int c = 0; c < 128; ++c)
-                            if (c < nv) bm = fmaxf(bm, s[c]);
-                        const float xm = __fmul_rn(cx, bm);
-                        if (xm > m) {
-                            m = xm;
-                            const int An = abs_bin(m);
-                            hist_slide(hist, 128, A, An);
-                            A = An;
-                        }
-                        // candidates: x >= (A-63)/63 (an exact integer test follows)
-                        const float thr = (float)(A - (kBins - 1)) / kBinsPerUnit;
+                    for (int c = 4; c < 64; c += 4) {
+                        m0 = fmaxf(m0, s[c]); m1 = fmaxf(m1, s[c + 1]);
+                        m2 = fmaxf(m2, s[c + 2]); m3 = fmaxf(m3, s[c + 3]);
+                    }
+                    const float xm = __fmul_rn(cx, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
+                    if (xm > m) {
+                        m = xm;
+                        const int An = abs_bin(m);
+                        hist_slide(hist, 128, A, An);
+                        A = An;
+                    }
+                    // candidates: x >= (A-63)/63 (an exact integer test follows)
+                    const float thr = (float)(A - (kBins - 1)) / kBinsPerUnit - 1e-3f;
 #pragma unroll
-                        for (int c = 0; c < 128; ++c) {
-                            if (c < nv) {
-                                const float x = __fmul_rn(cx, s[c]);
-                                if (x >= thr - 1e-3f) {
-                                    const int ab2 = abs_bin(x);
-                                    if (ab2 >= A - (kBins - 1)) hist[(ab2 & (kBins - 1)) * 128] += 1u;
-                                }
-                            }
+                    for (int c = 0; c < 64; ++c) {
+                        const float x = __fmul_rn(cx, s[c]);
+                        if (x >= thr) {
+                            const int ab2 = abs_bin(x);
+                            if (ab2 >= A - (kBins - 1)) hist[(ab2 & (kBins - 1)) * 128] += 1u;
                         }
                     }
                 } else {
-                    float f1b = 0.f;
+                    float f0a = 0.f, f0b = 0.f, f1a = 0.f, f1b = 0.f, f2a = 0.f, f2b = 0.f;
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        if (c < nv) {
-                            const float u = __fmaf_rn(cx, s[c], -sv.tau);
-                            float t0, t1, t2;
-                            entmax_terms<GM>(u, gamma, t0, t1, t2);
-                            F0 += t0; f1b += t1; F2 += t2;
-                        }
+                    for (int c = 0; c < 64; c += 2) {
+                        float t0, t1, t2, q0, q1, q2;
+                        entmax_terms_bf<GM>(__fmaf_rn(cx, s[c], -sv.tau), gamma, t0, t1, t2);
+                        entmax_terms_bf<GM>(__fmaf_rn(cx, s[c + 1], -sv.tau), gamma, q0, q1, q2);
+                        f0a += t0; f1a += t1; f2a += t2;
+                        f0b += q0; f1b += q1; f2b += q2;
                     }
+                    const float f1 = f1a + f1b;
+                    F0 += f0a + f0b; F1 += f1; F2 += f2a + f2b;
                     // liveness: t1 = u^(gamma-1) > 0 exactly where u > 0 (up to underflow,
                     // where p = u^gamma is 0 as well)
-                    F1 += f1b;
-                    if (__any_sync(0xffffffffu, f1b > 0.f) && lane == 0) live[b] = 1;
+                    if (__any_sync(0xffffffffu, f1 > 0.f) && lane == 0) live[b] = 1;
                 }
             }
             if (!ok) break;
             if (pass == 0) {
-                if (row_valid)
-                    hist_start<GM>(hist, 128, A, m, key_end, a.alpha, gamma, ptab, sv.lo, sv.hi,
-                                   sv.tau);
+                // merge the two half-row histograms; the half-0 thread computes the start
+                X(3, half) = m;
+                named_bar(1, kEw);
+                const float m_other = X(3, half ^ 1);
+                if (half == 0 && row_valid) {
+                    const int A0 = A;
+                    const int A1 = (m_other == -INFINITY) ? kNoBin : abs_bin(m_other);
+                    const unsigned int* h0 = hist;
+                    const unsigned int* h1 = reinterpret_cast<const unsigned int*>(smem + L::kHist1) + row;
+                    const float mr = fmaxf(m, m_other);
+                    const int Ar = abs_bin(mr);
+                    auto count = [&](int ab2) -> unsigned int {
+                        unsigned int c = 0;
+                        if (ab2 <= A0 && ab2 >= A0 - (kBins - 1)) c += h0[(ab2 & (kBins - 1)) * 128];
+                        if (ab2 <= A1 && ab2 >= A1 - (kBins - 1)) c += h1[(ab2 & (kBins - 1)) * 128];
+                        return c;
+                    };
+                    hist_start_fn<GM>(count, Ar, mr, key_end, a.alpha, gamma, ptab, sv.lo, sv.hi, sv.tau);
+                    X(0, 0) = sv.lo; X(1, 0) = sv.hi; X(2, 0) = sv.tau;
+                }
+                named_bar(1, kEw);
+                if (half == 1 && row_valid) { sv.lo = X(0, 0); sv.hi = X(1, 0); sv.tau = X(2, 0); }
             } else {
-                solver_update(sv, F0, F1, F2, gamma, gamma == 1.f, pass, a.ftol, a.stol);
+                X(0, half) = F0; X(1, half) = F1; X(2, half) = F2;
+                named_bar(1, kEw);
+                const float G0 = F0 + X(0, half ^ 1), G1 = F1 + X(1, half ^ 1), G2 = F2 + X(2, half ^ 1);
+                solver_update(sv, G0, G1, G2, gamma, gamma == 1.f, pass, a.ftol, a.stol);
             }
             const int all = named_bar_and(1, kEw, sv.done) && pass > 0;
             if (ew == 0) {
                 if (all) {
                     int n = 0;
-                    for (int b = 0; b < nblk; ++b)
-                        if (live[b]) live_list[n++] = b;
+                    for (int bb = 0; bb < nblk; ++bb)
+                        if (live[bb]) live_list[n++] = bb;
                     misc->nlive = n;
                 }
                 misc->decision = all ? kDecPv : kDecSolve;
@@ -340,55 +379,54 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const int sb = job & 1;
                 if (!(ok = mbar_wait(&s_full[sb], (job >> 1) & 1, ab, 9))) break;
                 tc_fence_after();
-                float s[128];
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    tmem_ld32(lane_base + sb * 128 + c * 32, &s[c * 32]);
+                float s[64];
+                tmem_ld32(lane_base + sb * 128 + c0, &s[0]);
+                tmem_ld32(lane_base + sb * 128 + c0 + 32, &s[32]);
                 tmem_wait_ld();
-                reg_fence<128>(s);
+                reg_fence<64>(s);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_empty[sb]);
-                const int nv = key_end - b * kBlk;
-                uint32_t pk[64];
+                const int nv = key_end - b * kBlk - c0;
+                uint32_t pk[32];
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const float p0 = (2 * c < nv) ? entmax_p<GM>(__fmaf_rn(cx, s[2 * c], -sv.tau), gamma) : 0.f;
-                    const float p1 = (2 * c + 1 < nv) ? entmax_p<GM>(__fmaf_rn(cx, s[2 * c + 1], -sv.tau), gamma) : 0.f;
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                    pk[c] = *reinterpret_cast<const uint32_t*>(&h2);
+                for (int c = 0; c < 64; c += 2) {
+                    const float u0 = (c < nv) ? __fmaf_rn(cx, s[c], -sv.tau) : -1.f;
+                    const float u1 = (c + 1 < nv) ? __fmaf_rn(cx, s[c + 1], -sv.tau) : -1.f;
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(entmax_p_bf<GM>(u0, gamma),
+                                                                    entmax_p_bf<GM>(u1, gamma));
+                    pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
                 }
                 if (!(ok = mbar_wait(p_empty, (pvjob & 1) ^ 1, ab, 10))) break;
-                uint8_t* prow = smem + L::kP + row * 128;
+                uint8_t* prow = smem + L::kP + half * kAtom + row * 128;
 #pragma unroll
-                for (int ch = 0; ch < 16; ++ch) {   // 16-byte chunk = 8 keys
-                    const int atom = ch >> 3, cin = ch & 7;
-                    uint4 val = make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-                    *reinterpret_cast<uint4*>(prow + atom * kAtom + ((cin ^ (row & 7)) << 4)) = val;
-                }
+                for (int ch = 0; ch < 8; ++ch)   // 16-byte chunk = 8 keys
+                    *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
+                        make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(p_full);
             }
         }
-        // epilogue: O row from TMEM, tau, iters, mask row, counters
-        float o[D];
+        // epilogue: this thread's half of the O row, tau, iters, mask row, counters
+        constexpr int DH = D / 2;
+        float o[DH];
         if (ok && nlive > 0) {
             ok = mbar_wait(o_full, 0, ab, 11);
             tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c)
-                tmem_ld32(lane_base + 256 + c * 32, &o[c * 32]);
+            for (int c = 0; c < DH / 32; ++c)
+                tmem_ld32(lane_base + 256 + half * DH + c * 32, &o[c * 32]);
             tmem_wait_ld();
-            reg_fence<D>(o);
+            reg_fence<DH>(o);
         } else {
 #pragma unroll
-            for (int c = 0; c < D; ++c) o[c] = 0.f;
+            for (int c = 0; c < DH; ++c) o[c] = 0.f;
         }
         if (row_valid) {
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + ((size_t)bh * N + i) * D;
+            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + ((size_t)bh * N + i) * D + half * DH;
 #pragma unroll
-            for (int c = 0; c < D; c += 8) {
+            for (int c = 0; c < DH; c += 8) {
                 uint4 val;
                 __nv_bfloat162 h;
                 h = __floats2bfloat162_rn(o[c], o[c + 1]); val.x = *reinterpret_cast<uint32_t*>(&h);
@@ -397,11 +435,13 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 h = __floats2bfloat162_rn(o[c + 6], o[c + 7]); val.w = *reinterpret_cast<uint32_t*>(&h);
                 *reinterpret_cast<uint4*>(orow + c) = val;
             }
-            a.tau[(size_t)bh * N + i] = sv.tau;
-            if (a.iters) a.iters[(size_t)bh * N + i] = (uint8_t)sv.iters;
+            if (half == 0) {
+                a.tau[(size_t)bh * N + i] = sv.tau;
+                if (a.iters) a.iters[(size_t)bh * N + i] = (uint8_t)sv.iters;
+            }
         }
         uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
-        for (int b = ew; b < T; b += kEw) mrow[b] = (b < nblk) ? live[b] : 0;
+        for (int bb = ew; bb < T; bb += kEw) mrow[bb] = (bb < nblk) ? live[bb] : 0;
         if (ew == 0) {
             atomicAdd(&a.hdr->counters[kCtrQkBlocks], (unsigned long long)nblk * (npass + 1));
             atomicAdd(&a.hdr->counters[kCtrPvBlocks], (unsigned long long)nlive);

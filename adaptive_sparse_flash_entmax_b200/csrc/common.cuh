@@ -127,13 +127,14 @@ constexpr int kNoBin = -(1 << 29);
 
 // Slots of hist (stride `stride` between slots of one row) that leave the
 // window when the top bin moves from A_old to A_new are cleared.
-__device__ __forceinline__ void hist_slide(unsigned int* hist, int stride, int A_old, int A_new) {
+template <typename C>
+__device__ __forceinline__ void hist_slide(C* hist, int stride, int A_old, int A_new) {
     if (A_new <= A_old) return;
     const int moved = A_new - A_old;
     if (moved >= kBins) {
-        for (int s = 0; s < kBins; ++s) hist[s * stride] = 0u;
+        for (int s = 0; s < kBins; ++s) hist[s * stride] = 0;
     } else {
-        for (int k = 0; k < moved; ++k) hist[((A_old - (kBins - 1) + k) & (kBins - 1)) * stride] = 0u;
+        for (int k = 0; k < moved; ++k) hist[((A_old - (kBins - 1) + k) & (kBins - 1)) * stride] = 0;
     }
 }
 

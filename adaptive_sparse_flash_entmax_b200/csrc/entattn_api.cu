@@ -71,7 +71,7 @@ ent_status check_common(int B, int H, int N, int d, int dtype, float alpha, int 
     if (causal != 0 && causal != 1) return fail(ENT_EINVAL, "causal must be 0 or 1 (got %d)", causal);
     if (d != 64 && d != 128) return fail(ENT_EUNSUPPORTED, "head dim d=%d (supported: 64, 128)", d);
     if ((long long)B * H > 65535) return fail(ENT_EUNSUPPORTED, "B*H=%lld exceeds 65535", (long long)B * H);
-    if (n_tiles(N) > 1024) return fail(ENT_EUNSUPPORTED, "N=%d exceeds 131072", N);
+    if (N > 130944) return fail(ENT_EUNSUPPORTED, "N=%d exceeds 130944", N);
     return ENT_OK;
 }
 

@@ -38,14 +38,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  : "memory");
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is
+// suspended by the hardware (it issues nothing) until the phase completes or
+// about 0.1 ms pass, so waiting warps leave the issue slots to working ones.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(100000u)
         : "memory");
     return ok != 0;
 }
@@ -68,7 +71,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0u) {
+        if ((it & 7u) == 0u) {
             if (*ab.flag) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 *ab.flag = 1;
@@ -109,6 +112,14 @@ __device__ __forceinline__ int named_bar_and(uint32_t id, uint32_t nthreads, int
         : "r"(id), "r"(nthreads), "r"(pred)
         : "memory");
     return (int)out;
+}
+
+// Shared-memory add without a returned value (no load-use dependency).
+__device__ __forceinline__ void red_shared_add_u32(uint32_t saddr, uint32_t v) {
+    asm volatile("red.shared::cta.add.u32 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_shared_and_b32(uint32_t saddr, uint32_t v) {
+    asm volatile("red.shared::cta.and.b32 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
 }
 
 // ------------------------------------------------------------------ TMA

@@ -4,10 +4,11 @@
 // Technical Deep Dive / AdaSplash: Fused GPU Kernel for Attention: the Q tile is
 // loaded once and stays on chip; K tiles stream for the tau passes; a final pass
 // streams K and V and accumulates O = P V).  Warp roles:
-//   warp 0   TMA producer: Q once, then K (and V in the P.V pass) blocks into a
-//            two-stage ring;
-//   warp 1   MMA issuer: S = Q K^T into a double-buffered TMEM accumulator
-//            (128 x 128 fp32), and O += P V (P from shared memory, V MN-major);
+//   warp 0   TMA producer: Q once, then K blocks into a four-slot ring during
+//            the score passes, or (K, V) pairs into two stages (the same memory)
+//            in the P.V pass;
+//   warp 1   MMA issuer: S = Q K^T into three TMEM accumulators (128 x 128
+//            fp32), and O += P V (P from shared memory, V MN-major);
 //   warps 2-9 elementwise: two threads per query row (= TMEM lane), 64 columns
 //            each.  Pass 0 builds the
 //            row max and the sliding 64-bin histogram ("AdaSplash-2: ...",
@@ -15,6 +16,10 @@
 //            F0, F1, F2 and take a Halley-bisection step (Accelerated Alpha-Entmax
 //            Transformation); the last solver pass marks live key blocks
 //            (Exploiting Sparsity); the P.V pass writes P (bf16) for live blocks.
+// Solver passes visit only candidate blocks: pass 0 records each warp's block
+// maximum of x, and a block is streamed again only if some warp's maximum
+// exceeds that warp's smallest current tau (otherwise no row of the tile has
+// u > 0 there, so the skipped block adds nothing to the sums or the mask).
 // After each score pass the elementwise group publishes a decision (another
 // solver pass, or the P.V pass with its live-block list) that the producer and
 // the MMA issuer wait on.  Every wait is bounded (2 s); a wait that gives up
@@ -30,40 +35,41 @@ using namespace tc;
 
 namespace {
 
-constexpr int kNst = 2;            // K/V ring stages
+constexpr int kSlots = 4;          // K slots of the score-pass ring
+constexpr int kPvStages = 2;       // (K, V) stages of the P.V pass (same memory as the slots)
+constexpr int kSbuf = 3;           // S accumulators in TMEM
 constexpr int kThreads = 320;      // 10 warps
 constexpr int kEw = 256;           // elementwise threads (warps 2-9): two per query row
 constexpr int kEwWarps = 8;
 constexpr int kAtom = 128 * 128;   // bytes of a [128 rows x 64 bf16] swizzled atom
-constexpr int kTmemCols = 512;     // S0 [0,128), S1 [128,256), O [256, 256+D)
+constexpr int kTmemCols = 512;     // S0 [0,128), S1 [128,256), O [256, 256+D), S2 [384, 512)
 constexpr int kDecSolve = 1, kDecPv = 2;
+
+__host__ __device__ constexpr uint32_t sbuf_col(int sb) { return sb < 2 ? sb * 128 : 384; }
 
 template <int D>
 struct Layout {
     static constexpr int kTile = D / 64 * kAtom;          // [128 x D] bf16
     static constexpr int kQ = 0;
-    static constexpr int kStage0 = kQ + kTile;
-    static constexpr int kStageBytes = 2 * kTile;         // K, then V
-    static constexpr int kP = kStage0 + kNst * kStageBytes;
-    static constexpr int kPBytes = 2 * kAtom;             // P [128 x 128] bf16
-    // Row histograms ([64 slots][128 rows] u32 per column half) live in memory that
-    // is idle during the score passes: the V halves of the two stages when they
-    // are 32 KB (D = 128), else P and a region of their own.
-    static constexpr int kHist0 = (D == 128) ? kStage0 + kTile : kP;
-    static constexpr int kHist1 = (D == 128) ? kStage0 + kStageBytes + kTile : kP + kPBytes;
-    static constexpr int kXch = (D == 128) ? kP + kPBytes : kP + 2 * kPBytes;   // [4][2][128] f32
+    static constexpr int kRing = kQ + kTile;              // kSlots tiles: score-pass K slots,
+                                                          // or two (K, V) stages in the P.V pass
+    static constexpr int kP = kRing + kSlots * kTile;     // P [128 x 128] bf16; in pass 0 the two
+    static constexpr int kPBytes = 2 * kAtom;             // half-row histograms [64][128] u16
+    static constexpr int kXch = kP + kPBytes;             // [4][2][128] f32 exchange
     static constexpr int kBars = kXch + 4 * 2 * 128 * 4;
-    static constexpr int kNumBars = 16;
-    static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, decision, nlive, abort
+    static constexpr int kNumBars = 24;
+    static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, decision, njobs, abort
     static constexpr int kPtab = kMisc + 16;              // 68 floats
-    static constexpr int kLive = kPtab + 68 * 4;          // T bytes
-    static size_t bytes(int T) { return (size_t)kLive + (size_t)((T + 15) / 16) * 16 + 4 * (size_t)T + 1024; }
+    static constexpr int kLive = kPtab + 68 * 4;          // live[T], cand[T] (bytes), list[T] (int),
+                                                          // per-warp block maxima [T][8] (bf16)
+    __host__ __device__ static size_t r16(int T) { return (size_t)((T + 15) / 16) * 16; }
+    static size_t bytes(int T) { return (size_t)kLive + 2 * r16(T) + 4 * (size_t)T + 16 * (size_t)T + 1024; }
 };
 
 struct Misc {
     uint32_t tmem_base;
     int decision;
-    int nlive;
+    int njobs;      // blocks in job_list for the next pass
     int abort;
 };
 
@@ -89,20 +95,24 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-    uint64_t* full = bars;                 // [kNst]  TMA -> MMA
-    uint64_t* empty = bars + kNst;         // [kNst]  MMA -> TMA
-    uint64_t* s_full = bars + 2 * kNst;    // [2]     MMA -> elementwise
-    uint64_t* s_empty = s_full + 2;        // [2]     elementwise -> MMA
-    uint64_t* p_full = s_empty + 2;        //         elementwise -> MMA
-    uint64_t* p_empty = p_full + 1;        //         MMA -> elementwise
-    uint64_t* o_full = p_empty + 1;        //         MMA -> elementwise
-    uint64_t* q_full = o_full + 1;         //         TMA -> MMA
-    uint64_t* dec_bar = q_full + 1;        //         elementwise -> TMA, MMA
-    uint64_t* mma_done = dec_bar + 1;      //         MMA -> MMA (all issued MMAs retired)
+    uint64_t* kfull = bars;                    // [kSlots]     TMA -> MMA (score passes)
+    uint64_t* kempty = kfull + kSlots;         // [kSlots]     MMA -> TMA
+    uint64_t* pvfull = kempty + kSlots;        // [kPvStages]  TMA -> MMA (P.V pass)
+    uint64_t* pvempty = pvfull + kPvStages;    // [kPvStages]  MMA -> TMA
+    uint64_t* s_full = pvempty + kPvStages;    // [kSbuf]      MMA -> elementwise
+    uint64_t* s_empty = s_full + kSbuf;        // [kSbuf]      elementwise -> MMA
+    uint64_t* p_full = s_empty + kSbuf;        //              elementwise -> MMA
+    uint64_t* p_empty = p_full + 1;            //              MMA -> elementwise
+    uint64_t* o_full = p_empty + 1;            //              MMA -> elementwise
+    uint64_t* q_full = o_full + 1;             //              TMA -> MMA
+    uint64_t* dec_bar = q_full + 1;            //              elementwise -> TMA, MMA
+    uint64_t* mma_done = dec_bar + 1;          //              MMA -> MMA (all MMAs retired)
     Misc* misc = reinterpret_cast<Misc*>(smem + L::kMisc);
     float* ptab = reinterpret_cast<float*>(smem + L::kPtab);
-    uint8_t* live = smem + L::kLive;
-    int* live_list = reinterpret_cast<int*>(smem + L::kLive + ((a.T + 15) / 16) * 16);
+    uint8_t* live = smem + L::kLive;                       // live blocks of the current pass
+    uint8_t* cand = live + L::r16(a.T);                    // candidate blocks, tagged by pass
+    int* job_list = reinterpret_cast<int*>(cand + L::r16(a.T));   // blocks of the next pass
+    __nv_bfloat16* bmw = reinterpret_cast<__nv_bfloat16*>(job_list + a.T);   // [T][8]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, N = a.N;
@@ -112,8 +122,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const Abort ab{&misc->abort, a.hdr};
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kNst; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps); }
+        for (int s = 0; s < kSlots; ++s) { mbar_init(&kfull[s], 1); mbar_init(&kempty[s], 1); }
+        for (int s = 0; s < kPvStages; ++s) { mbar_init(&pvfull[s], 1); mbar_init(&pvempty[s], 1); }
+        for (int s = 0; s < kSbuf; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps); }
         mbar_init(p_full, kEwWarps);
         mbar_init(p_empty, 1);
         mbar_init(o_full, 1);
@@ -121,7 +132,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_init(dec_bar, 1);
         mbar_init(mma_done, 1);
         misc->decision = 0;
-        misc->nlive = 0;
+        misc->njobs = 0;
         misc->abort = 0;
         fence_barrier_init();
     }
@@ -129,7 +140,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tmem_alloc(&misc->tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    for (int b = threadIdx.x; b < T; b += kThreads) live[b] = 0;
+    for (int b = threadIdx.x; b < T; b += kThreads) { live[b] = 0; cand[b] = 0; }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -144,25 +155,36 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_arrive_expect_tx(q_full, L::kTile);
             for (int at = 0; at < D / 64; ++at)
                 tma_load_3d(smem + L::kQ + at * kAtom, &tm_q, at * 64, t * kBlk, bh, q_full);
-            int job = 0, kind = kDecSolve;
+            int sj = 0, pj = 0, kind = kDecSolve;   // score-pass and P.V-pass load counters
             uint32_t dec_phase = 0;
-            bool ok = true;
+            bool ok = true, first = true;
             while (ok) {
                 const bool pv = kind == kDecPv;
-                const int njobs = pv ? misc->nlive : nblk;
-                for (int i = 0; i < njobs && ok; ++i, ++job) {
-                    const int b = pv ? live_list[i] : i;
-                    const int st = job % kNst;
-                    if (!(ok = mbar_wait(&empty[st], ((job / kNst) & 1) ^ 1, ab, 1))) break;
-                    uint8_t* kb = smem + L::kStage0 + st * L::kStageBytes;
-                    mbar_arrive_expect_tx(&full[st], pv ? 2 * L::kTile : L::kTile);
-                    for (int at = 0; at < D / 64; ++at)
-                        tma_load_3d(kb + at * kAtom, &tm_k, at * 64, b * kBlk, bh, &full[st]);
-                    if (pv)
+                const int njobs = first ? nblk : misc->njobs;
+                for (int i = 0; i < njobs && ok; ++i) {
+                    const int b = first ? i : job_list[i];
+                    if (!pv) {
+                        const int sl = sj % kSlots;
+                        if (!(ok = mbar_wait(&kempty[sl], ((sj / kSlots) & 1) ^ 1, ab, 1))) break;
+                        mbar_arrive_expect_tx(&kfull[sl], L::kTile);
+                        uint8_t* kb = smem + L::kRing + sl * L::kTile;
                         for (int at = 0; at < D / 64; ++at)
+                            tma_load_3d(kb + at * kAtom, &tm_k, at * 64, b * kBlk, bh, &kfull[sl]);
+                        ++sj;
+                    } else {
+                        const int st = pj % kPvStages;
+                        if (!(ok = mbar_wait(&pvempty[st], ((pj / kPvStages) & 1) ^ 1, ab, 1))) break;
+                        mbar_arrive_expect_tx(&pvfull[st], 2 * L::kTile);
+                        uint8_t* kb = smem + L::kRing + st * 2 * L::kTile;
+                        for (int at = 0; at < D / 64; ++at) {
+                            tma_load_3d(kb + at * kAtom, &tm_k, at * 64, b * kBlk, bh, &pvfull[st]);
                             tma_load_3d(kb + L::kTile + at * kAtom, &tm_v, at * 64, b * kBlk, bh,
-                                        &full[st]);
+                                        &pvfull[st]);
+                        }
+                        ++pj;
+                    }
                 }
+                first = false;
                 if (!ok || pv) break;
                 if (!(ok = mbar_wait(dec_bar, dec_phase, ab, 2))) break;
                 dec_phase ^= 1;
@@ -170,53 +192,69 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             // Copies issued but possibly not consumed land before the CTA ends.
             drain_wait(q_full, 0);
-            for (int j = job - 1; j >= 0 && j >= job - kNst; --j)
-                drain_wait(&full[j % kNst], (j / kNst) & 1);
+            for (int j = sj - 1; j >= 0 && j >= sj - kSlots; --j) drain_wait(&kfull[j % kSlots], (j / kSlots) & 1);
+            for (int j = pj - 1; j >= 0 && j >= pj - kPvStages; --j)
+                drain_wait(&pvfull[j % kPvStages], (j / kPvStages) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
-            const uint32_t qb = smem_u32(smem + L::kQ);
-            const uint32_t pb = smem_u32(smem + L::kP);
+            // Descriptors differ only in the start-address field (bits 0-13, address >> 4),
+            // so each operand's base descriptor is built once and offsets are added.
+            const uint64_t dq = sdesc_sw128(smem_u32(smem + L::kQ), 16, 1024);
+            const uint64_t dp = sdesc_sw128(smem_u32(smem + L::kP), 16, 1024);
+            const uint64_t dring = sdesc_sw128(smem_u32(smem + L::kRing), 16, 1024);
+            const uint64_t dring_mn = sdesc_sw128(smem_u32(smem + L::kRing), kAtom, 1024);
             bool ok = mbar_wait(q_full, 0, ab, 3);
             tc_fence_after();
-            int job = 0, pvjob = 0, kind = kDecSolve;
+            int job = 0, sj = 0, pj = 0, kind = kDecSolve;
             uint32_t dec_phase = 0;
+            bool first = true;
             while (ok) {
                 const bool pv = kind == kDecPv;
-                const int njobs = pv ? misc->nlive : nblk;
+                const int njobs = first ? nblk : misc->njobs;
+                first = false;
                 for (int i = 0; i < njobs && ok; ++i, ++job) {
-                    const int st = job % kNst, sb = job & 1;
-                    if (!(ok = mbar_wait(&full[st], (job / kNst) & 1, ab, 4))) break;
-                    if (!(ok = mbar_wait(&s_empty[sb], ((job >> 1) & 1) ^ 1, ab, 5))) break;
+                    const int sb = job % kSbuf;
+                    uint32_t kofs;   // byte offset of the K tile from the ring start
+                    if (!pv) {
+                        const int sl = sj % kSlots;
+                        if (!(ok = mbar_wait(&kfull[sl], (sj / kSlots) & 1, ab, 4))) break;
+                        kofs = sl * L::kTile;
+                    } else {
+                        const int st = pj % kPvStages;
+                        if (!(ok = mbar_wait(&pvfull[st], (pj / kPvStages) & 1, ab, 4))) break;
+                        kofs = st * 2 * L::kTile;
+                    }
+                    if (!(ok = mbar_wait(&s_empty[sb], ((job / kSbuf) & 1) ^ 1, ab, 5))) break;
                     tc_fence_after();
-                    const uint32_t kb = smem_u32(smem + L::kStage0 + st * L::kStageBytes);
+                    const uint64_t dk = dring + (kofs >> 4);
+                    const uint32_t dS = tmem + sbuf_col(sb);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-                        umma_bf16(tmem + sb * 128, sdesc_sw128(qb + off, 16, 1024),
-                                  sdesc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0);
+                        const uint32_t off = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
+                        umma_bf16(dS, dq + off, dk + off, idesc_qk, kk > 0);
                     }
                     umma_commit(&s_full[sb]);
                     if (!pv) {
-                        umma_commit(&empty[st]);
+                        umma_commit(&kempty[sj % kSlots]);
+                        ++sj;
                         continue;
                     }
-                    if (!(ok = mbar_wait(p_full, pvjob & 1, ab, 6))) break;
+                    if (!(ok = mbar_wait(p_full, pj & 1, ab, 6))) break;
                     tc_fence_after();
-                    const uint32_t vb = kb + L::kTile;
+                    const uint64_t dv = dring_mn + ((kofs + L::kTile) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < kBlk / 16; ++kk) {
-                        const uint32_t aoff = (kk >> 2) * kAtom + (kk & 3) * 32;
-                        umma_bf16(tmem + 256, sdesc_sw128(pb + aoff, 16, 1024),
-                                  sdesc_sw128(vb + kk * 16 * 128, kAtom, 1024), idesc_pv,
-                                  (pvjob > 0 || kk > 0) ? 1u : 0u);
+                        const uint32_t aoff = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
+                        umma_bf16(tmem + 256, dp + aoff, dv + ((kk * 16 * 128) >> 4), idesc_pv,
+                                  (pj > 0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(p_empty);
-                    umma_commit(&empty[st]);
-                    ++pvjob;
+                    umma_commit(&pvempty[pj % kPvStages]);
+                    ++pj;
                 }
                 if (!ok) break;
                 if (pv) {
@@ -246,11 +284,19 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int key_end = !row_valid ? 0 : (a.causal ? i + 1 : N);
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const float gamma = a.gamma, cx = a.cx;
-        unsigned int* hist = reinterpret_cast<unsigned int*>(smem + (half ? L::kHist1 : L::kHist0)) + row;
+        // Row histograms in the (then idle) P region: [64 slots][128 rows] u32 words,
+        // the low 16 bits counting half 0's columns and the high 16 bits half 1's.
+        // Updates are shared-memory reductions (no load-use chain, no lost updates).
+        uint32_t* histw = reinterpret_cast<uint32_t*>(smem + L::kP) + row;
+        const uint32_t hist_saddr = smem_u32(histw);
+        const uint32_t hinc = half ? 65536u : 1u;
+        const uint32_t hkeep = half ? 0x0000FFFFu : 0xFFFF0000u;   // red.and mask clearing my half
+        const float c63 = cx * kBinsPerUnit;
         float* xch = reinterpret_cast<float*>(smem + L::kXch);   // [k][half][row]
         auto X = [&](int k, int h) -> float& { return xch[(k * 2 + h) * 128 + row]; };
         if (ew < 65) ptab[ew] = entmax_p<GM>((float)ew / kBinsPerUnit, gamma);
-        for (int sl = 0; sl < kBins; ++sl) hist[sl * 128] = 0u;
+        if (half == 0)
+            for (int sl = 0; sl < kBins; ++sl) histw[sl * 128] = 0u;
         named_bar(1, kEw);
 
         float m = -INFINITY;
@@ -259,21 +305,27 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         sv.tau = 0.f; sv.lo = 0.f; sv.hi = 0.f;
         sv.done = row_valid ? 0 : 1;
         sv.iters = 0;
+        const int wi = warp - 2;                  // elementwise warp index 0..7
         int job = 0, pass = 0, nlive = 0;
+        long long qk_blocks = nblk;
         bool ok = true;
         for (;; ++pass) {
             float F0 = 0.f, F1 = 0.f, F2 = 0.f;
+            int npj = nblk;
             if (pass > 0) {
                 for (int bb = ew; bb < nblk; bb += kEw) live[bb] = 0;
-                named_bar(1, kEw);
+                named_bar(1, kEw);   // also publishes job_list / njobs of this pass
+                npj = misc->njobs;
+                qk_blocks += npj;
             }
-            for (int b = 0; b < nblk; ++b, ++job) {
-                const int sb = job & 1;
-                if (!(ok = mbar_wait(&s_full[sb], (job >> 1) & 1, ab, 8))) break;
+            for (int jj = 0; jj < npj; ++jj, ++job) {
+                const int b = (pass == 0) ? jj : job_list[jj];
+                const int sb = job % kSbuf;
+                if (!(ok = mbar_wait(&s_full[sb], (job / kSbuf) & 1, ab, 8))) break;
                 tc_fence_after();
                 float s[64];
-                tmem_ld32(lane_base + sb * 128 + c0, &s[0]);
-                tmem_ld32(lane_base + sb * 128 + c0 + 32, &s[32]);
+                tmem_ld32(lane_base + sbuf_col(sb) + c0, &s[0]);
+                tmem_ld32(lane_base + sbuf_col(sb) + c0 + 32, &s[32]);
                 tmem_wait_ld();
                 reg_fence<64>(s);
                 tc_fence_before();
@@ -293,20 +345,39 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         m2 = fmaxf(m2, s[c + 2]); m3 = fmaxf(m3, s[c + 3]);
                     }
                     const float xm = __fmul_rn(cx, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
+                    // per-warp block maximum (rounded up) for skipping in the solver passes
+                    float xw = xm;
+#pragma unroll
+                    for (int o2 = 16; o2 > 0; o2 >>= 1) xw = fmaxf(xw, __shfl_xor_sync(0xffffffffu, xw, o2));
+                    if (lane == 0) bmw[b * 8 + wi] = __float2bfloat16_ru(xw);
                     if (xm > m) {
                         m = xm;
                         const int An = abs_bin(m);
-                        hist_slide(hist, 128, A, An);
+                        // slots leaving the window: clear this half's 16 bits
+                        if (An > A) {
+                            const int moved = An - A;
+                            if (moved >= kBins) {
+                                for (int sl = 0; sl < kBins; ++sl) red_shared_and_b32(hist_saddr + sl * 512, hkeep);
+                            } else {
+                                for (int k2 = 0; k2 < moved; ++k2)
+                                    red_shared_and_b32(hist_saddr + ((A - (kBins - 1) + k2) & (kBins - 1)) * 512, hkeep);
+                            }
+                        }
                         A = An;
                     }
-                    // candidates: x >= (A-63)/63 (an exact integer test follows)
-                    const float thr = (float)(A - (kBins - 1)) / kBinsPerUnit - 1e-3f;
+                    // Elements below the window's lowest bin (A-63)/63 <= m-1 are never in the
+                    // support; blocks whose maximum is below it are skipped as a whole.
+                    const float thr_x = (float)(A - (kBins - 1)) / kBinsPerUnit - 1e-3f;
+                    if (__any_sync(0xffffffffu, xm >= thr_x)) {
+                        // bin = floor(x*63) via the 1.5*2^23 rounding trick: rint(x*63 - 1/2)
+                        // (an element exactly on an edge may land one bin low, which keeps
+                        // the edge bounds valid)
+                        const int lo_bin = A - (kBins - 1);
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        const float x = __fmul_rn(cx, s[c]);
-                        if (x >= thr) {
-                            const int ab2 = abs_bin(x);
-                            if (ab2 >= A - (kBins - 1)) hist[(ab2 & (kBins - 1)) * 128] += 1u;
+                        for (int c = 0; c < 64; ++c) {
+                            const float y = __fmaf_rn(s[c], c63, -0.5f) + 12582912.0f;
+                            const int ab2 = __float_as_int(y) - 0x4B400000;
+                            if (ab2 >= lo_bin) red_shared_add_u32(hist_saddr + (ab2 & (kBins - 1)) * 512, hinc);
                         }
                     }
                 } else {
@@ -335,14 +406,13 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (half == 0 && row_valid) {
                     const int A0 = A;
                     const int A1 = (m_other == -INFINITY) ? kNoBin : abs_bin(m_other);
-                    const unsigned int* h0 = hist;
-                    const unsigned int* h1 = reinterpret_cast<const unsigned int*>(smem + L::kHist1) + row;
                     const float mr = fmaxf(m, m_other);
                     const int Ar = abs_bin(mr);
                     auto count = [&](int ab2) -> unsigned int {
+                        const uint32_t w = histw[(ab2 & (kBins - 1)) * 128];
                         unsigned int c = 0;
-                        if (ab2 <= A0 && ab2 >= A0 - (kBins - 1)) c += h0[(ab2 & (kBins - 1)) * 128];
-                        if (ab2 <= A1 && ab2 >= A1 - (kBins - 1)) c += h1[(ab2 & (kBins - 1)) * 128];
+                        if (ab2 <= A0 && ab2 >= A0 - (kBins - 1)) c += w & 0xFFFFu;
+                        if (ab2 <= A1 && ab2 >= A1 - (kBins - 1)) c += w >> 16;
                         return c;
                     };
                     hist_start_fn<GM>(count, Ar, mr, key_end, a.alpha, gamma, ptab, sv.lo, sv.hi, sv.tau);
@@ -357,31 +427,48 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 solver_update(sv, G0, G1, G2, gamma, gamma == 1.f, pass, a.ftol, a.stol);
             }
             const int all = named_bar_and(1, kEw, sv.done) && pass > 0;
-            if (ew == 0) {
-                if (all) {
-                    int n = 0;
-                    for (int bb = 0; bb < nblk; ++bb)
-                        if (live[bb]) live_list[n++] = bb;
-                    misc->nlive = n;
+            const uint8_t tag = (uint8_t)(pass + 2);
+            if (!all) {
+                // Candidates for the next pass: a block can hold u > 0 for a row of this
+                // warp only if the warp's block maximum exceeds the warp's smallest tau.
+                float th = row_valid ? sv.tau : INFINITY;
+#pragma unroll
+                for (int o2 = 16; o2 > 0; o2 >>= 1) th = fminf(th, __shfl_xor_sync(0xffffffffu, th, o2));
+                th -= 4e-7f * fmaxf(1.f, fabsf(th));
+                for (int bb = lane; bb < nblk; bb += 32)
+                    if (__bfloat162float(bmw[bb * 8 + wi]) > th) cand[bb] = tag;
+                named_bar(1, kEw);
+            }
+            if (warp == 2) {
+                // compact the next pass's blocks: live ones for P.V, else the candidates
+                int n = 0;
+                for (int base = 0; base < nblk; base += 32) {
+                    const int bb = base + lane;
+                    const bool f = bb < nblk && (all ? live[bb] != 0 : cand[bb] == tag);
+                    const unsigned int msk = __ballot_sync(0xffffffffu, f);
+                    if (f) job_list[n + __popc(msk & ((1u << lane) - 1u))] = bb;
+                    n += __popc(msk);
                 }
-                misc->decision = all ? kDecPv : kDecSolve;
-                mbar_arrive(dec_bar);
+                if (lane == 0) {
+                    misc->njobs = n;
+                    misc->decision = all ? kDecPv : kDecSolve;
+                    mbar_arrive(dec_bar);
+                }
             }
             if (all) break;
         }
         const int npass = pass;
         if (ok) {
-            named_bar(1, kEw);   // live_list / nlive visible to the group
-            nlive = misc->nlive;
-            int pvjob = 0;
-            for (int li = 0; li < nlive; ++li, ++job, ++pvjob) {
-                const int b = live_list[li];
-                const int sb = job & 1;
-                if (!(ok = mbar_wait(&s_full[sb], (job >> 1) & 1, ab, 9))) break;
+            named_bar(1, kEw);   // job_list / njobs of the P.V pass visible to the group
+            nlive = misc->njobs;
+            for (int li = 0; li < nlive; ++li, ++job) {
+                const int b = job_list[li];
+                const int sb = job % kSbuf;
+                if (!(ok = mbar_wait(&s_full[sb], (job / kSbuf) & 1, ab, 9))) break;
                 tc_fence_after();
                 float s[64];
-                tmem_ld32(lane_base + sb * 128 + c0, &s[0]);
-                tmem_ld32(lane_base + sb * 128 + c0 + 32, &s[32]);
+                tmem_ld32(lane_base + sbuf_col(sb) + c0, &s[0]);
+                tmem_ld32(lane_base + sbuf_col(sb) + c0 + 32, &s[32]);
                 tmem_wait_ld();
                 reg_fence<64>(s);
                 tc_fence_before();
@@ -397,7 +484,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                                                     entmax_p_bf<GM>(u1, gamma));
                     pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
                 }
-                if (!(ok = mbar_wait(p_empty, (pvjob & 1) ^ 1, ab, 10))) break;
+                if (!(ok = mbar_wait(p_empty, (li & 1) ^ 1, ab, 10))) break;
                 uint8_t* prow = smem + L::kP + half * kAtom + row * 128;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)   // 16-byte chunk = 8 keys
@@ -443,7 +530,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
         for (int bb = ew; bb < T; bb += kEw) mrow[bb] = (bb < nblk) ? live[bb] : 0;
         if (ew == 0) {
-            atomicAdd(&a.hdr->counters[kCtrQkBlocks], (unsigned long long)nblk * (npass + 1));
+            atomicAdd(&a.hdr->counters[kCtrQkBlocks], (unsigned long long)qk_blocks);
             atomicAdd(&a.hdr->counters[kCtrPvBlocks], (unsigned long long)nlive);
             atomicAdd(&a.hdr->counters[kCtrPasses], (unsigned long long)npass);
             atomicAdd(&a.hdr->counters[kCtrTiles], 1ull);

@@ -36,8 +36,8 @@
  *    the 128x128 block of P for query tile t and key block b holds a nonzero
  *    (blocks above the diagonal are 0 when causal).  The forward writes it;
  *    the backward reads it and skips exactly the 0 blocks.
- *  - Supported: 1 < alpha <= 2, d in {64, 128}, N >= 1 (any N; the last tile
- *    may be ragged), B, H >= 0.  B*H == 0 or N == 0 is a no-op returning ENT_OK.
+ *  - Supported: 1 < alpha <= 2, d in {64, 128}, 1 <= N <= 130944 (any N; the
+ *    last tile may be ragged), B, H >= 0, B*H <= 65535.  B*H == 0 or N == 0 is a no-op returning ENT_OK.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
  *    legacy default stream).  Argument errors return synchronously before any
  *    work is enqueued.  No exception crosses the ABI.

@@ -148,14 +148,16 @@ __device__ __forceinline__ void hist_slide(C* hist, int stride, int A_old, int A
 // assignment and intersected with the plain bracket [m-1, m - n^(1-alpha)].
 // tau_0 is the root of the straight line through the bin-centre model
 // F_c(E) = sum_a c_a ((a+1/2)/63 - E)_+^gamma - 1 at E = lo and E = hi.
-// `count(a)` returns the number of elements in absolute bin a (a in [A-63, A]).
+// `count(a)` returns the number of elements in absolute bin a (a in [ebot, A]);
+// every element at or above edge ebot/63 is counted (the window may be narrower
+// than 64 bins; edges below ebot are not used).
 template <int GM, typename CountFn>
-__device__ __forceinline__ void hist_start_fn(CountFn count, int A, float m, int n, float alpha,
-                                              float gamma, const float* ptab, float& lo, float& hi,
-                                              float& tau0) {
+__device__ __forceinline__ void hist_start_fn(CountFn count, int A, int ebot, float m, int n,
+                                              float alpha, float gamma, const float* ptab,
+                                              float& lo, float& hi, float& tau0) {
     int h_ok = A + 1;
     int l_ok = kNoBin;
-    for (int e = A; e >= A - (kBins - 1); --e) {
+    for (int e = A; e >= ebot; --e) {
         float fu = -1.f, fl = -1.f;
         for (int a = e; a <= A; ++a) {
             const float c = (float)count(a);
@@ -172,8 +174,7 @@ __device__ __forceinline__ void hist_start_fn(CountFn count, int A, float m, int
     hi = fminf((float)h_ok / kBinsPerUnit + slack, plain_hi);
     if (hi < lo) hi = lo;
     float fcl = -1.f, fch = -1.f;
-    for (int k = 0; k < kBins; ++k) {
-        const int a = A - k;
+    for (int a = A; a >= ebot; --a) {
         const unsigned int c = count(a);
         if (c) {
             const float centre = ((float)a + 0.5f) / kBinsPerUnit;
@@ -191,8 +192,8 @@ template <int GM>
 __device__ __forceinline__ void hist_start(const unsigned int* hist, int stride, int A, float m,
                                            int n, float alpha, float gamma, const float* ptab,
                                            float& lo, float& hi, float& tau0) {
-    hist_start_fn<GM>([&](int a) { return hist[(a & (kBins - 1)) * stride]; }, A, m, n, alpha,
-                      gamma, ptab, lo, hi, tau0);
+    hist_start_fn<GM>([&](int a) { return hist[(a & (kBins - 1)) * stride]; }, A,
+                      A - (kBins - 1), m, n, alpha, gamma, ptab, lo, hi, tau0);
 }
 
 // Branch-free power terms for the streaming passes: u <= 0 gives zeros through

@@ -8,8 +8,8 @@
 //     dQ = dS K / sqrt(d),   dK = dS^T Q / sqrt(d),   dV = P^T dO.
 // Only the 128 x 128 blocks marked live by the forward's block mask are visited.
 //
-// Two kernels, both with warp roles (warp 0 TMA, warp 1 MMA issuer, warps 2-5
-// elementwise, thread = TMEM lane) and 64-wide sub-tiles so that two stages,
+// Two kernels, both with warp roles (warp 0 TMA, warp 1 MMA issuer, warps 2-9
+// elementwise, two threads per TMEM lane) and 64-wide sub-tiles so that two stages,
 // double-buffered TMEM accumulators and the bf16 operand written by the
 // elementwise warps fit on chip:
 //   dq kernel   one CTA per 128-row query tile, K/V in 64-key sub-blocks of
@@ -34,8 +34,9 @@ bool make_tmap_bf16_rows(CUtensorMap* map, const void* base, int BH, int N, int 
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kEw = 128;
+constexpr int kThreads = 320;                  // warp 0 TMA, warp 1 MMA, warps 2-9 elementwise
+constexpr int kEw = 256;                       // two threads per TMEM lane, 32 columns each
+constexpr int kEwWarps = 8;
 constexpr int kNst = 2;
 constexpr int kTmemCols = 512;
 constexpr int kSub = 64;                       // sub-tile width (keys or query rows)
@@ -75,6 +76,17 @@ __device__ __forceinline__ void store_row_sw128(uint8_t* atom, int row, const ui
             make_uint4(w[ch * 4], w[ch * 4 + 1], w[ch * 4 + 2], w[ch * 4 + 3]);
 }
 
+// Write 32 bf16 values (16 packed words): chunks 4*half .. 4*half+3 of row `row`.
+__device__ __forceinline__ void store_half_row_sw128(uint8_t* atom, int row, int half, const uint32_t* w) {
+    uint8_t* base = atom + row * 128;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int ch = half * 4 + q;
+        *reinterpret_cast<uint4*>(base + ((ch ^ (row & 7)) << 4)) =
+            make_uint4(w[q * 4], w[q * 4 + 1], w[q * 4 + 2], w[q * 4 + 3]);
+    }
+}
+
 __device__ __forceinline__ void store_out_row(void* out, size_t off, const float* v, int D, float sc) {
     __nv_bfloat16* p = static_cast<__nv_bfloat16*>(out) + off;
     for (int c = 0; c < D; c += 8) {
@@ -98,7 +110,8 @@ struct DqLayout {
     static constexpr int kStage0 = kDO + kTile;
     static constexpr int kStageBytes = 2 * kSubT;       // K_sub, V_sub
     static constexpr int kDS = kStage0 + kNst * kStageBytes;   // dS hi, dS lo: [128 x 64] bf16 atoms
-    static constexpr int kBars = kDS + 2 * kAtom128;
+    static constexpr int kXch = kDS + 2 * kAtom128;            // [2][2][128] f32
+    static constexpr int kBars = kXch + 2 * 2 * 128 * 4;
     static constexpr int kMisc = kBars + 8 * 16;
     static constexpr int kList = kMisc + 16;            // int job list [2*T]
     static size_t bytes(int T) { return (size_t)kList + 8 * (size_t)T + 1024; }
@@ -136,9 +149,9 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1); mbar_init(&empty[s], 1);
-            mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 4);
+            mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps);
         }
-        mbar_init(ds_full, 4);
+        mbar_init(ds_full, kEwWarps);
         mbar_init(ds_empty, 1);
         mbar_init(acc_full, 1);
         mbar_init(in_full, 1);
@@ -197,8 +210,12 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(128, kSub, 0, 0);   // [128 x 64], K = d
             constexpr uint32_t idesc_dq = idesc_bf16(128, D, 0, 1);     // dQ += dS K, K MN-major
-            const uint32_t qb = smem_u32(smem + L::kQ), dob = smem_u32(smem + L::kDO);
-            const uint32_t dsb = smem_u32(smem + L::kDS);
+            // base descriptors; operands differ only by start-address offsets
+            const uint64_t dq_ = sdesc_sw128(smem_u32(smem + L::kQ), 16, 1024);
+            const uint64_t ddo = sdesc_sw128(smem_u32(smem + L::kDO), 16, 1024);
+            const uint64_t dds = sdesc_sw128(smem_u32(smem + L::kDS), 16, 1024);
+            const uint64_t dst = sdesc_sw128(smem_u32(smem + L::kStage0), 16, 1024);
+            const uint64_t dst_mn = sdesc_sw128(smem_u32(smem + L::kStage0), kAtom64, 1024);
             bool ok = mbar_wait(in_full, 0, ab, 22);
             tc_fence_after();
             // issue S and dP of job j into TMEM buffer j & 1
@@ -207,15 +224,15 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (!mbar_wait(&full[st], (j >> 1) & 1, ab, 23)) return false;
                 if (!mbar_wait(&s_empty[sbuf], ((j >> 1) & 1) ^ 1, ab, 24)) return false;
                 tc_fence_after();
-                const uint32_t kb = smem_u32(smem + L::kStage0 + st * L::kStageBytes);
-                const uint32_t vb = kb + L::kSubT;
+                const uint64_t dk = dst + ((st * L::kStageBytes) >> 4);
+                const uint64_t dv = dk + (L::kSubT >> 4);
                 const uint32_t dS = tmem + sbuf * 128, dPc = tmem + sbuf * 128 + 64;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t oa = (kk >> 2) * kAtom128 + (kk & 3) * 32;
-                    const uint32_t ob = (kk >> 2) * kAtom64 + (kk & 3) * 32;
-                    umma_bf16(dS, sdesc_sw128(qb + oa, 16, 1024), sdesc_sw128(kb + ob, 16, 1024), idesc_s, kk > 0);
-                    umma_bf16(dPc, sdesc_sw128(dob + oa, 16, 1024), sdesc_sw128(vb + ob, 16, 1024), idesc_s, kk > 0);
+                    const uint32_t oa = ((kk >> 2) * kAtom128 + (kk & 3) * 32) >> 4;
+                    const uint32_t ob = ((kk >> 2) * kAtom64 + (kk & 3) * 32) >> 4;
+                    umma_bf16(dS, dq_ + oa, dk + ob, idesc_s, kk > 0);
+                    umma_bf16(dPc, ddo + oa, dv + ob, idesc_s, kk > 0);
                 }
                 umma_commit(&s_full[sbuf]);
                 return true;
@@ -231,16 +248,15 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int bj = j - njobs;        // phase B job: dQ += dS K
                 if (!(ok = mbar_wait(ds_full, bj & 1, ab, 25))) break;
                 tc_fence_after();
-                const uint32_t kb = smem_u32(smem + L::kStage0 + st * L::kStageBytes);
+                const uint64_t dkmn = dst_mn + ((st * L::kStageBytes) >> 4);
                 // dQ += (dS_hi + dS_lo) K: the two bf16 parts carry dS to ~16 bits, which
                 // the cancellation in sum_j dS_ij k_j (rows of dS sum to 0) needs.
 #pragma unroll
                 for (int kk = 0; kk < kSub / 16; ++kk) {
-                    const uint64_t bdesc = sdesc_sw128(kb + kk * 16 * 128, kAtom64, 1024);
-                    umma_bf16(tmem + 256, sdesc_sw128(dsb + kk * 32, 16, 1024), bdesc, idesc_dq,
+                    const uint64_t bdesc = dkmn + ((kk * 16 * 128) >> 4);
+                    umma_bf16(tmem + 256, dds + ((kk * 32) >> 4), bdesc, idesc_dq,
                               (bj > 0 || kk > 0) ? 1u : 0u);
-                    umma_bf16(tmem + 256, sdesc_sw128(dsb + kAtom128 + kk * 32, 16, 1024), bdesc,
-                              idesc_dq, 1u);
+                    umma_bf16(tmem + 256, dds + ((kAtom128 + kk * 32) >> 4), bdesc, idesc_dq, 1u);
                 }
                 umma_commit(ds_empty);
                 umma_commit(&empty[st]);
@@ -250,36 +266,39 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             drain_wait(mma_done, 0);
         }
     } else {
+        // two threads per query row: `half` takes columns [32*half, 32*half + 32)
+        // of each 64-key sub-block; delta's partial sums meet in shared memory
+        const int ew = threadIdx.x - 64;
+        const int half = ew >> 7;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int i = t * kBlk + row;
         const bool row_valid = i < N;
         const int key_end = !row_valid ? 0 : (a.causal ? i + 1 : N);
-        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + half * 32;
         const float gamma = a.gamma, cx = a.cx;
         const float tau = row_valid ? a.tau[(size_t)bh * N + i] : 0.f;
+        float* xch = reinterpret_cast<float*>(smem + L::kXch);   // [2][2][128]
         float sg = 0.f, sgdp = 0.f, delta = 0.f;
         bool ok = true;
         for (int j = 0; j < total && ok; ++j) {
             const int sbuf = j & 1;
             if (!(ok = mbar_wait(&s_full[sbuf], (j >> 1) & 1, ab, 26))) break;
             tc_fence_after();
-            float s[64], dp[64];
+            float s[32], dp[32];
             tmem_ld32(lane_base + sbuf * 128, &s[0]);
-            tmem_ld32(lane_base + sbuf * 128 + 32, &s[32]);
             tmem_ld32(lane_base + sbuf * 128 + 64, &dp[0]);
-            tmem_ld32(lane_base + sbuf * 128 + 96, &dp[32]);
             tmem_wait_ld();
-            reg_fence<64>(s);
-            reg_fence<64>(dp);
+            reg_fence<32>(s);
+            reg_fence<32>(dp);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[sbuf]);
-            const int nv = key_end - jobs[j < njobs ? j : j - njobs];
+            const int nv = key_end - jobs[j < njobs ? j : j - njobs] - half * 32;
             if (j < njobs) {
                 float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
+                for (int c = 0; c < 32; c += 2) {
                     const float g0 = (c < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c], -tau), gamma) : 0.f;
                     const float g1 = (c + 1 < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c + 1], -tau), gamma) : 0.f;
                     a0 += g0; a1 += g1;
@@ -288,14 +307,18 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 sg += a0 + a1;
                 sgdp += b0 + b1;
                 if (j == njobs - 1) {
-                    delta = (sg > 0.f) ? sgdp / sg : 0.f;
-                    if (row_valid) a.delta[(size_t)bh * N + i] = delta;
+                    xch[(0 * 2 + half) * 128 + row] = sg;
+                    xch[(1 * 2 + half) * 128 + row] = sgdp;
+                    named_bar(1, kEw);
+                    const float SG = sg + xch[(0 * 2 + (half ^ 1)) * 128 + row];
+                    const float SGDP = sgdp + xch[(1 * 2 + (half ^ 1)) * 128 + row];
+                    delta = (SG > 0.f) ? SGDP / SG : 0.f;
+                    if (row_valid && half == 0) a.delta[(size_t)bh * N + i] = delta;
                 }
             } else {
-                if (njobs == 0) break;
-                uint32_t whi[32], wlo[32];
+                uint32_t whi[16], wlo[16];
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
+                for (int c = 0; c < 32; c += 2) {
                     const float g0 = (c < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c], -tau), gamma) : 0.f;
                     const float g1 = (c + 1 < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c + 1], -tau), gamma) : 0.f;
                     const float d0 = g0 * (dp[c] - delta), d1 = g1 * (dp[c + 1] - delta);
@@ -306,27 +329,29 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 const int bj = j - njobs;
                 if (!(ok = mbar_wait(ds_empty, (bj & 1) ^ 1, ab, 27))) break;
-                store_row_sw128(smem + L::kDS, row, whi);
-                store_row_sw128(smem + L::kDS + kAtom128, row, wlo);
+                store_half_row_sw128(smem + L::kDS, row, half, whi);
+                store_half_row_sw128(smem + L::kDS + kAtom128, row, half, wlo);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ds_full);
             }
         }
-        if (njobs == 0 && row_valid) a.delta[(size_t)bh * N + i] = 0.f;
-        float acc[D];
+        if (njobs == 0 && row_valid && half == 0) a.delta[(size_t)bh * N + i] = 0.f;
+        constexpr int DH = D / 2;
+        float acc[DH];
         if (ok && njobs > 0) {
             ok = mbar_wait(acc_full, 0, ab, 28);
             tc_fence_after();
+            const uint32_t ob = tmem + ((uint32_t)(quarter * 32) << 16) + 256 + half * DH;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + 256 + c * 32, &acc[c * 32]);
+            for (int c = 0; c < DH / 32; ++c) tmem_ld32(ob + c * 32, &acc[c * 32]);
             tmem_wait_ld();
-            reg_fence<D>(acc);
+            reg_fence<DH>(acc);
         } else {
 #pragma unroll
-            for (int c = 0; c < D; ++c) acc[c] = 0.f;
+            for (int c = 0; c < DH; ++c) acc[c] = 0.f;
         }
-        if (row_valid) store_out_row(a.dq, ((size_t)bh * N + i) * D, acc, D, a.scale);
+        if (row_valid) store_out_row(a.dq, ((size_t)bh * N + i) * D + half * DH, acc, DH, a.scale);
         if (threadIdx.x == 64)   // block products: phase A S,dP (2) + phase B S,dP,dQ hi,lo (4), per 64-key half
             atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(3 * njobs));
     }
@@ -391,9 +416,9 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1); mbar_init(&empty[s], 1);
-            mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 4);
+            mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps);
         }
-        mbar_init(p_full, 4);
+        mbar_init(p_full, kEwWarps);
         mbar_init(p_empty, 1);
         mbar_init(acc_full, 1);
         mbar_init(in_full, 1);
@@ -450,8 +475,12 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(128, kSub, 0, 0);   // S^T, dP^T [128 keys x 64]
             constexpr uint32_t idesc_acc = idesc_bf16(128, D, 0, 1);    // dV, dK: B (dO, Q) MN-major
-            const uint32_t kb = smem_u32(smem + L::kK), vb = smem_u32(smem + L::kV);
-            const uint32_t ptb = smem_u32(smem + L::kPT), dstb = smem_u32(smem + L::kDST);
+            const uint64_t dkk = sdesc_sw128(smem_u32(smem + L::kK), 16, 1024);
+            const uint64_t dvv = sdesc_sw128(smem_u32(smem + L::kV), 16, 1024);
+            const uint64_t dpt = sdesc_sw128(smem_u32(smem + L::kPT), 16, 1024);
+            const uint64_t ddst = sdesc_sw128(smem_u32(smem + L::kDST), 16, 1024);
+            const uint64_t dst = sdesc_sw128(smem_u32(smem + L::kStage0), 16, 1024);
+            const uint64_t dst_mn = sdesc_sw128(smem_u32(smem + L::kStage0), kAtom64, 1024);
             bool ok = mbar_wait(in_full, 0, ab, 32);
             tc_fence_after();
             auto issue_sdp = [&](int j) -> bool {
@@ -459,16 +488,14 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 if (!mbar_wait(&full[st], (j >> 1) & 1, ab, 33)) return false;
                 if (!mbar_wait(&s_empty[sbuf], ((j >> 1) & 1) ^ 1, ab, 34)) return false;
                 tc_fence_after();
-                const uint32_t qs = smem_u32(smem + L::kStage0 + st * L::kStageBytes);
-                const uint32_t dos = qs + L::kSubT;
+                const uint64_t dqs = dst + ((st * L::kStageBytes) >> 4);
+                const uint64_t dos = dqs + (L::kSubT >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t oa = (kk >> 2) * kAtom128 + (kk & 3) * 32;
-                    const uint32_t ob = (kk >> 2) * kAtom64 + (kk & 3) * 32;
-                    umma_bf16(tmem + sbuf * 128, sdesc_sw128(kb + oa, 16, 1024),
-                              sdesc_sw128(qs + ob, 16, 1024), idesc_s, kk > 0);
-                    umma_bf16(tmem + sbuf * 128 + 64, sdesc_sw128(vb + oa, 16, 1024),
-                              sdesc_sw128(dos + ob, 16, 1024), idesc_s, kk > 0);
+                    const uint32_t oa = ((kk >> 2) * kAtom128 + (kk & 3) * 32) >> 4;
+                    const uint32_t ob = ((kk >> 2) * kAtom64 + (kk & 3) * 32) >> 4;
+                    umma_bf16(tmem + sbuf * 128, dkk + oa, dqs + ob, idesc_s, kk > 0);
+                    umma_bf16(tmem + sbuf * 128 + 64, dvv + oa, dos + ob, idesc_s, kk > 0);
                 }
                 umma_commit(&s_full[sbuf]);
                 return true;
@@ -479,15 +506,14 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 if (!(ok = mbar_wait(p_full, j & 1, ab, 35))) break;
                 tc_fence_after();
                 const int st = j & 1;
-                const uint32_t qs = smem_u32(smem + L::kStage0 + st * L::kStageBytes);
-                const uint32_t dos = qs + L::kSubT;
+                const uint64_t qmn = dst_mn + ((st * L::kStageBytes) >> 4);
+                const uint64_t domn = qmn + (L::kSubT >> 4);
 #pragma unroll
                 for (int kk = 0; kk < kSub / 16; ++kk) {
                     const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-                    umma_bf16(tm_dv, sdesc_sw128(ptb + kk * 32, 16, 1024),
-                              sdesc_sw128(dos + kk * 16 * 128, kAtom64, 1024), idesc_acc, acc);
-                    umma_bf16(tm_dk, sdesc_sw128(dstb + kk * 32, 16, 1024),
-                              sdesc_sw128(qs + kk * 16 * 128, kAtom64, 1024), idesc_acc, acc);
+                    const uint32_t ok_ = (kk * 16 * 128) >> 4;
+                    umma_bf16(tm_dv, dpt + ((kk * 32) >> 4), domn + ok_, idesc_acc, acc);
+                    umma_bf16(tm_dk, ddst + ((kk * 32) >> 4), qmn + ok_, idesc_acc, acc);
                 }
                 umma_commit(p_empty);
                 umma_commit(&empty[st]);
@@ -497,12 +523,14 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             drain_wait(mma_done, 0);
         }
     } else {
+        // two threads per key row: `half` takes query columns [32*half, 32*half + 32)
         const int ew = threadIdx.x - 64;
+        const int half = ew >> 7;
         const int quarter = warp & 3;
         const int krow = quarter * 32 + lane;         // key row == TMEM lane
         const int jkey = b * kBlk + krow;
         const bool key_valid = jkey < N;
-        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + half * 32;
         const float gamma = a.gamma, cx = a.cx;
         bool ok = true;
         for (int j = 0; j < njobs && ok; ++j) {
@@ -517,64 +545,66 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             const int sbuf = j & 1;
             if (!(ok = mbar_wait(&s_full[sbuf], (j >> 1) & 1, ab, 36))) break;
             tc_fence_after();
-            float s[64], dp[64];
+            float s[32], dp[32];
             tmem_ld32(lane_base + sbuf * 128, &s[0]);
-            tmem_ld32(lane_base + sbuf * 128 + 32, &s[32]);
             tmem_ld32(lane_base + sbuf * 128 + 64, &dp[0]);
-            tmem_ld32(lane_base + sbuf * 128 + 96, &dp[32]);
             tmem_wait_ld();
-            reg_fence<64>(s);
-            reg_fence<64>(dp);
+            reg_fence<32>(s);
+            reg_fence<32>(dp);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[sbuf]);
-            // column c is query i0 + c: admissible iff i < N, key valid, and key <= i if causal
-            const int cmin = a.causal ? jkey - i0 : 0;       // c >= cmin
-            const int cmax = min(kSub, N - i0);              // c < cmax
-            uint32_t wp[32], wd[32];
+            // column c is query i0 + 32*half + c: admissible iff i < N, key valid, key <= i if causal
+            const int ib = i0 + half * 32;
+            const int cmin = a.causal ? jkey - ib : 0;       // c >= cmin
+            const int cmax = min(32, N - ib);                // c < cmax
+            const float* tcol = tdb + half * 32;
+            uint32_t wp[16], wd[16];
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
+            for (int c = 0; c < 32; c += 2) {
                 float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
                 if (key_valid && c >= cmin && c < cmax) {
-                    const float u = __fmaf_rn(cx, s[c], -tdb[c]);
+                    const float u = __fmaf_rn(cx, s[c], -tcol[c]);
                     p0 = entmax_p<GM>(u, gamma);
-                    d0 = entmax_g<GM>(u, gamma) * (dp[c] - tdb[64 + c]);
+                    d0 = entmax_g<GM>(u, gamma) * (dp[c] - tcol[64 + c]);
                 }
                 if (key_valid && c + 1 >= cmin && c + 1 < cmax) {
-                    const float u = __fmaf_rn(cx, s[c + 1], -tdb[c + 1]);
+                    const float u = __fmaf_rn(cx, s[c + 1], -tcol[c + 1]);
                     p1 = entmax_p<GM>(u, gamma);
-                    d1 = entmax_g<GM>(u, gamma) * (dp[c + 1] - tdb[64 + c + 1]);
+                    d1 = entmax_g<GM>(u, gamma) * (dp[c + 1] - tcol[64 + c + 1]);
                 }
                 wp[c >> 1] = pack_bf16(p0, p1);
                 wd[c >> 1] = pack_bf16(d0, d1);
             }
             if (!(ok = mbar_wait(p_empty, (j & 1) ^ 1, ab, 37))) break;
-            store_row_sw128(smem + L::kPT, krow, wp);
-            store_row_sw128(smem + L::kDST, krow, wd);
+            store_half_row_sw128(smem + L::kPT, krow, half, wp);
+            store_half_row_sw128(smem + L::kDST, krow, half, wd);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_full);
         }
-        float acc[D];
+        constexpr int DH = D / 2;
+        float acc[DH];
+        const uint32_t qoff = ((uint32_t)(quarter * 32) << 16) + half * DH;
         if (ok && njobs > 0) {
             ok = mbar_wait(acc_full, 0, ab, 38);
             tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) tmem_ld32(tm_dv + ((uint32_t)(quarter * 32) << 16) + c * 32, &acc[c * 32]);
+            for (int c = 0; c < DH / 32; ++c) tmem_ld32(tm_dv + qoff + c * 32, &acc[c * 32]);
             tmem_wait_ld();
-            reg_fence<D>(acc);
+            reg_fence<DH>(acc);
         } else {
 #pragma unroll
-            for (int c = 0; c < D; ++c) acc[c] = 0.f;
+            for (int c = 0; c < DH; ++c) acc[c] = 0.f;
         }
-        if (key_valid) store_out_row(a.dv, ((size_t)bh * N + jkey) * D, acc, D, 1.f);
+        if (key_valid) store_out_row(a.dv, ((size_t)bh * N + jkey) * D + half * DH, acc, DH, 1.f);
         if (ok && njobs > 0) {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) tmem_ld32(tm_dk + ((uint32_t)(quarter * 32) << 16) + c * 32, &acc[c * 32]);
+            for (int c = 0; c < DH / 32; ++c) tmem_ld32(tm_dk + qoff + c * 32, &acc[c * 32]);
             tmem_wait_ld();
-            reg_fence<D>(acc);
+            reg_fence<DH>(acc);
         }
-        if (key_valid) store_out_row(a.dk, ((size_t)bh * N + jkey) * D, acc, D, a.scale);
+        if (key_valid) store_out_row(a.dk, ((size_t)bh * N + jkey) * D + half * DH, acc, DH, a.scale);
         if (ew == 0)   // block products: S^T, dP^T, dV, dK (4) per 64-row half
             atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(2 * njobs));
     }

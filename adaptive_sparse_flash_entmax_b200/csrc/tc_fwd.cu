@@ -292,6 +292,17 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t hinc = half ? 65536u : 1u;
         const uint32_t hkeep = half ? 0x0000FFFFu : 0xFFFF0000u;   // red.and mask clearing my half
         const float c63 = cx * kBinsPerUnit;
+        // Insert budget per half-row: a row whose window keeps filling with scores
+        // (a dense row) stops building its histogram after kInsertBudget inserts and
+        // starts from the plain bracket [m-1, m - n^(1-alpha)]: on such rows the
+        // inserts cost more than the solver pass the histogram saves (measured;
+        // narrowing the window instead of stopping was slower still).  The window
+        // width `wbins` is kept general: counts are complete for every bin inside
+        // it, so any bracket taken from it is rigorous.
+        constexpr int kInsertBudget = 48;
+        int n_ins = 0;
+        int wbins = kBins;                        // window width in bins (0: stopped)
+        auto clear_bin = [&](int ab2) { red_shared_and_b32(hist_saddr + (ab2 & (kBins - 1)) * 512, hkeep); };
         float* xch = reinterpret_cast<float*>(smem + L::kXch);   // [k][half][row]
         auto X = [&](int k, int h) -> float& { return xch[(k * 2 + h) * 128 + row]; };
         if (ew < 65) ptab[ew] = entmax_p<GM>((float)ew / kBinsPerUnit, gamma);
@@ -353,31 +364,38 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     if (xm > m) {
                         m = xm;
                         const int An = abs_bin(m);
-                        // slots leaving the window: clear this half's 16 bits
-                        if (An > A) {
+                        // bins leaving the window [A-w+1, A]: clear this half's 16 bits
+                        if (An > A && wbins > 0) {
                             const int moved = An - A;
-                            if (moved >= kBins) {
-                                for (int sl = 0; sl < kBins; ++sl) red_shared_and_b32(hist_saddr + sl * 512, hkeep);
+                            if (moved >= wbins) {
+                                for (int sl = 0; sl < kBins; ++sl) clear_bin(sl);
                             } else {
-                                for (int k2 = 0; k2 < moved; ++k2)
-                                    red_shared_and_b32(hist_saddr + ((A - (kBins - 1) + k2) & (kBins - 1)) * 512, hkeep);
+                                for (int k2 = 0; k2 < moved; ++k2) clear_bin(A - wbins + 1 + k2);
                             }
                         }
                         A = An;
                     }
                     // Elements below the window's lowest bin (A-63)/63 <= m-1 are never in the
-                    // support; blocks whose maximum is below it are skipped as a whole.
-                    const float thr_x = (float)(A - (kBins - 1)) / kBinsPerUnit - 1e-3f;
-                    if (__any_sync(0xffffffffu, xm >= thr_x)) {
+                    // support; blocks whose maximum is below the window are skipped as a whole.
+                    const float thr_x = (float)(A - (wbins - 1)) / kBinsPerUnit - 1e-3f;
+                    if (__any_sync(0xffffffffu, xm >= thr_x && wbins > 0)) {
                         // bin = floor(x*63) via the 1.5*2^23 rounding trick: rint(x*63 - 1/2)
                         // (an element exactly on an edge may land one bin low, which keeps
                         // the edge bounds valid)
-                        const int lo_bin = A - (kBins - 1);
+                        const int lo_bin = (wbins > 0) ? A - (wbins - 1) : 0x7FFFFFFF;
 #pragma unroll
                         for (int c = 0; c < 64; ++c) {
                             const float y = __fmaf_rn(s[c], c63, -0.5f) + 12582912.0f;
                             const int ab2 = __float_as_int(y) - 0x4B400000;
-                            if (ab2 >= lo_bin) red_shared_add_u32(hist_saddr + (ab2 & (kBins - 1)) * 512, hinc);
+                            const bool q = ab2 >= lo_bin;
+                            if (q) red_shared_add_u32(hist_saddr + (ab2 & (kBins - 1)) * 512, hinc);
+                            n_ins += q;
+                        }
+                        const int want = n_ins > kInsertBudget ? 0 : kBins;
+                        if (want < wbins) {
+                            // narrow the window: bins [A-w+1, A-want] leave (all of it when stopping)
+                            for (int ab2 = A - wbins + 1; ab2 <= A - want; ++ab2) clear_bin(ab2);
+                            wbins = want;
                         }
                     }
                 } else {
@@ -401,21 +419,38 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (pass == 0) {
                 // merge the two half-row histograms; the half-0 thread computes the start
                 X(3, half) = m;
+                X(2, half) = (float)wbins;
                 named_bar(1, kEw);
                 const float m_other = X(3, half ^ 1);
-                if (half == 0 && row_valid) {
-                    const int A0 = A;
-                    const int A1 = (m_other == -INFINITY) ? kNoBin : abs_bin(m_other);
+                const int w_other = (int)X(2, half ^ 1);
+                const bool over = (wbins == 0) || (w_other == 0);
+                if (half == 0 && row_valid && over) {
+                    // plain bracket [m-1, m - n^(1-alpha)], start at its midpoint
+                    const float mr = fmaxf(m, m_other);
+                    sv.lo = mr - 1.f;
+                    sv.hi = fmaxf(sv.lo, mr - exp2f((1.f - a.alpha) * __log2f((float)key_end)));
+                    sv.tau = 0.5f * (sv.lo + sv.hi);
+                }
+                named_bar(1, kEw);
+                if (half == 0 && row_valid && over) {
+                    X(0, 0) = sv.lo; X(1, 0) = sv.hi; X(2, 0) = sv.tau;
+                } else if (half == 0 && row_valid) {
+                    const int A0 = A, w0 = wbins;
+                    const int A1 = (m_other == -INFINITY) ? kNoBin : abs_bin(m_other), w1 = w_other;
                     const float mr = fmaxf(m, m_other);
                     const int Ar = abs_bin(mr);
+                    // edges are usable only where both halves count every element above them
+                    const int ebot = max(A0 == kNoBin ? kNoBin : A0 - w0 + 1,
+                                         A1 == kNoBin ? kNoBin : A1 - w1 + 1);
                     auto count = [&](int ab2) -> unsigned int {
                         const uint32_t w = histw[(ab2 & (kBins - 1)) * 128];
                         unsigned int c = 0;
-                        if (ab2 <= A0 && ab2 >= A0 - (kBins - 1)) c += w & 0xFFFFu;
-                        if (ab2 <= A1 && ab2 >= A1 - (kBins - 1)) c += w >> 16;
+                        if (ab2 <= A0 && ab2 >= A0 - (w0 - 1)) c += w & 0xFFFFu;
+                        if (ab2 <= A1 && ab2 >= A1 - (w1 - 1)) c += w >> 16;
                         return c;
                     };
-                    hist_start_fn<GM>(count, Ar, mr, key_end, a.alpha, gamma, ptab, sv.lo, sv.hi, sv.tau);
+                    hist_start_fn<GM>(count, Ar, max(ebot, Ar - (kBins - 1)), mr, key_end, a.alpha,
+                                      gamma, ptab, sv.lo, sv.hi, sv.tau);
                     X(0, 0) = sv.lo; X(1, 0) = sv.hi; X(2, 0) = sv.tau;
                 }
                 named_bar(1, kEw);

@@ -216,6 +216,17 @@ __device__ __forceinline__ void entmax_terms_bf(float u, float gamma, float& t0,
 }
 
 template <int GM>
+__device__ __forceinline__ float entmax_g_bf(float u, float gamma) {
+    const float up = fmaxf(u, 0.f);
+    if (GM == 1) return (u > 0.f) ? 1.f : 0.f;
+    if (GM == 2) return up;
+    if (GM == 3) return up * up;
+    if (GM == 4) return up * up * up;
+    const float v = exp2f((gamma - 1.f) * __log2f(up));   // inf at up = 0 when gamma < 1 (not used)
+    return (u > 0.f) ? v : 0.f;
+}
+
+template <int GM>
 __device__ __forceinline__ float entmax_p_bf(float u, float gamma) {
     const float up = fmaxf(u, 0.f);
     if (GM == 1) return up;

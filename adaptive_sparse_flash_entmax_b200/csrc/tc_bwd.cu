@@ -37,11 +37,14 @@ namespace {
 constexpr int kThreads = 320;                  // warp 0 TMA, warp 1 MMA, warps 2-9 elementwise
 constexpr int kEw = 256;                       // two threads per TMEM lane, 32 columns each
 constexpr int kEwWarps = 8;
-constexpr int kNst = 2;
+constexpr int kNst = 3;                        // K/V (dq) or Q/dO (dkv) sub-tile stages
 constexpr int kTmemCols = 512;
 constexpr int kSub = 64;                       // sub-tile width (keys or query rows)
 constexpr int kAtom128 = 128 * 128;            // [128 rows x 64 bf16] atom
 constexpr int kAtom64 = 64 * 128;              // [64 rows x 64 bf16] atom
+constexpr int kSbufDq = 3;                     // S/dP accumulator pairs of the dq kernel
+// TMEM column of S/dP pair `sb` in the dq kernel (dQ lives at columns 256..383)
+__host__ __device__ constexpr uint32_t dq_sbuf_col(int sb) { return sb < 2 ? sb * 128 : 384; }
 
 struct Misc {
     uint32_t tmem_base;
@@ -126,15 +129,15 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-    uint64_t* full = bars;               // [2]
-    uint64_t* empty = bars + 2;          // [2]
-    uint64_t* s_full = bars + 4;         // [2]
-    uint64_t* s_empty = bars + 6;        // [2]
-    uint64_t* ds_full = bars + 8;
-    uint64_t* ds_empty = bars + 9;
-    uint64_t* acc_full = bars + 10;
-    uint64_t* in_full = bars + 11;       // Q and dO tiles
-    uint64_t* mma_done = bars + 12;
+    uint64_t* full = bars;                     // [kNst]
+    uint64_t* empty = full + kNst;             // [kNst]
+    uint64_t* s_full = empty + kNst;           // [kSbufDq]
+    uint64_t* s_empty = s_full + kSbufDq;      // [kSbufDq]
+    uint64_t* ds_full = s_empty + kSbufDq;
+    uint64_t* ds_empty = ds_full + 1;
+    uint64_t* acc_full = ds_empty + 1;
+    uint64_t* in_full = acc_full + 1;          // Q and dO tiles
+    uint64_t* mma_done = in_full + 1;
     Misc* misc = reinterpret_cast<Misc*>(smem + L::kMisc);
     int* jobs = reinterpret_cast<int*>(smem + L::kList);   // key offsets of the 64-key sub-blocks
 
@@ -147,10 +150,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const Abort ab{&misc->abort, a.hdr};
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&full[s], 1); mbar_init(&empty[s], 1);
-            mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps);
-        }
+        for (int s = 0; s < kNst; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < kSbufDq; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps); }
         mbar_init(ds_full, kEwWarps);
         mbar_init(ds_empty, 1);
         mbar_init(acc_full, 1);
@@ -194,8 +195,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             bool ok = true;
             for (; job < total && ok; ++job) {
                 const int j0 = jobs[job % njobs];
-                const int st = job & 1;
-                if (!(ok = mbar_wait(&empty[st], ((job >> 1) & 1) ^ 1, ab, 21))) break;
+                const int st = job % kNst;
+                if (!(ok = mbar_wait(&empty[st], ((job / kNst) & 1) ^ 1, ab, 21))) break;
                 uint8_t* sb = smem + L::kStage0 + st * L::kStageBytes;
                 mbar_arrive_expect_tx(&full[st], 2 * L::kSubT);
                 for (int at = 0; at < D / 64; ++at) {
@@ -204,7 +205,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             }
             drain_wait(in_full, 0);
-            for (int j = job - 1; j >= 0 && j >= job - kNst; --j) drain_wait(&full[j & 1], (j >> 1) & 1);
+            for (int j = job - 1; j >= 0 && j >= job - kNst; --j) drain_wait(&full[j % kNst], (j / kNst) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -218,15 +219,15 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const uint64_t dst_mn = sdesc_sw128(smem_u32(smem + L::kStage0), kAtom64, 1024);
             bool ok = mbar_wait(in_full, 0, ab, 22);
             tc_fence_after();
-            // issue S and dP of job j into TMEM buffer j & 1
+            // issue S and dP of job j into TMEM pair j % kSbufDq
             auto issue_sdp = [&](int j) -> bool {
-                const int st = j & 1, sbuf = j & 1;
-                if (!mbar_wait(&full[st], (j >> 1) & 1, ab, 23)) return false;
-                if (!mbar_wait(&s_empty[sbuf], ((j >> 1) & 1) ^ 1, ab, 24)) return false;
+                const int st = j % kNst, sbuf = j % kSbufDq;
+                if (!mbar_wait(&full[st], (j / kNst) & 1, ab, 23)) return false;
+                if (!mbar_wait(&s_empty[sbuf], ((j / kSbufDq) & 1) ^ 1, ab, 24)) return false;
                 tc_fence_after();
                 const uint64_t dk = dst + ((st * L::kStageBytes) >> 4);
                 const uint64_t dv = dk + (L::kSubT >> 4);
-                const uint32_t dS = tmem + sbuf * 128, dPc = tmem + sbuf * 128 + 64;
+                const uint32_t dS = tmem + dq_sbuf_col(sbuf), dPc = dS + 64;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t oa = ((kk >> 2) * kAtom128 + (kk & 3) * 32) >> 4;
@@ -240,7 +241,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (ok && total > 0) ok = issue_sdp(0);
             for (int j = 0; j < total && ok; ++j) {
                 if (j + 1 < total && !(ok = issue_sdp(j + 1))) break;
-                const int st = j & 1;
+                const int st = j % kNst;
                 if (j < njobs) {                 // phase A: K/V stage only fed S and dP
                     umma_commit(&empty[st]);
                     continue;
@@ -282,12 +283,12 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float sg = 0.f, sgdp = 0.f, delta = 0.f;
         bool ok = true;
         for (int j = 0; j < total && ok; ++j) {
-            const int sbuf = j & 1;
-            if (!(ok = mbar_wait(&s_full[sbuf], (j >> 1) & 1, ab, 26))) break;
+            const int sbuf = j % kSbufDq;
+            if (!(ok = mbar_wait(&s_full[sbuf], (j / kSbufDq) & 1, ab, 26))) break;
             tc_fence_after();
             float s[32], dp[32];
-            tmem_ld32(lane_base + sbuf * 128, &s[0]);
-            tmem_ld32(lane_base + sbuf * 128 + 64, &dp[0]);
+            tmem_ld32(lane_base + dq_sbuf_col(sbuf), &s[0]);
+            tmem_ld32(lane_base + dq_sbuf_col(sbuf) + 64, &dp[0]);
             tmem_wait_ld();
             reg_fence<32>(s);
             reg_fence<32>(dp);
@@ -295,12 +296,16 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[sbuf]);
             const int nv = key_end - jobs[j < njobs ? j : j - njobs] - half * 32;
+            if (!__all_sync(0xffffffffu, nv >= 32)) {   // diagonal or ragged sub-block
+#pragma unroll
+                for (int c = 0; c < 32; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
+            }
             if (j < njobs) {
                 float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const float g0 = (c < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c], -tau), gamma) : 0.f;
-                    const float g1 = (c + 1 < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c + 1], -tau), gamma) : 0.f;
+                    const float g0 = entmax_g_bf<GM>(__fmaf_rn(cx, s[c], -tau), gamma);
+                    const float g1 = entmax_g_bf<GM>(__fmaf_rn(cx, s[c + 1], -tau), gamma);
                     a0 += g0; a1 += g1;
                     b0 = fmaf(g0, dp[c], b0); b1 = fmaf(g1, dp[c + 1], b1);
                 }
@@ -319,8 +324,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 uint32_t whi[16], wlo[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const float g0 = (c < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c], -tau), gamma) : 0.f;
-                    const float g1 = (c + 1 < nv) ? entmax_g<GM>(__fmaf_rn(cx, s[c + 1], -tau), gamma) : 0.f;
+                    const float g0 = entmax_g_bf<GM>(__fmaf_rn(cx, s[c], -tau), gamma);
+                    const float g1 = entmax_g_bf<GM>(__fmaf_rn(cx, s[c + 1], -tau), gamma);
                     const float d0 = g0 * (dp[c] - delta), d1 = g1 * (dp[c + 1] - delta);
                     const __nv_bfloat162 h = __floats2bfloat162_rn(d0, d1);
                     const float2 hf = __bfloat1622float2(h);
@@ -394,15 +399,15 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + 2;
-    uint64_t* s_full = bars + 4;
-    uint64_t* s_empty = bars + 6;
-    uint64_t* p_full = bars + 8;
-    uint64_t* p_empty = bars + 9;
-    uint64_t* acc_full = bars + 10;
-    uint64_t* in_full = bars + 11;
-    uint64_t* mma_done = bars + 12;
+    uint64_t* full = bars;                     // [kNst]
+    uint64_t* empty = full + kNst;             // [kNst]
+    uint64_t* s_full = empty + kNst;           // [2]
+    uint64_t* s_empty = s_full + 2;            // [2]
+    uint64_t* p_full = s_empty + 2;
+    uint64_t* p_empty = p_full + 1;
+    uint64_t* acc_full = p_empty + 1;
+    uint64_t* in_full = acc_full + 1;
+    uint64_t* mma_done = in_full + 1;
     Misc* misc = reinterpret_cast<Misc*>(smem + L::kMisc);
     int* jobs = reinterpret_cast<int*>(smem + L::kList);   // row offsets of the 64-row sub-tiles
     float* td = reinterpret_cast<float*>(smem + L::kTauDelta);   // [buf][tau|delta][64]
@@ -414,10 +419,8 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const Abort ab{&misc->abort, a.hdr};
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&full[s], 1); mbar_init(&empty[s], 1);
-            mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps);
-        }
+        for (int s = 0; s < kNst; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps); }
         mbar_init(p_full, kEwWarps);
         mbar_init(p_empty, 1);
         mbar_init(acc_full, 1);
@@ -459,8 +462,8 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             bool ok = true;
             for (; job < njobs && ok; ++job) {
                 const int i0 = jobs[job];
-                const int st = job & 1;
-                if (!(ok = mbar_wait(&empty[st], ((job >> 1) & 1) ^ 1, ab, 31))) break;
+                const int st = job % kNst;
+                if (!(ok = mbar_wait(&empty[st], ((job / kNst) & 1) ^ 1, ab, 31))) break;
                 uint8_t* sb = smem + L::kStage0 + st * L::kStageBytes;
                 mbar_arrive_expect_tx(&full[st], 2 * L::kSubT);
                 for (int at = 0; at < D / 64; ++at) {
@@ -469,7 +472,7 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 }
             }
             drain_wait(in_full, 0);
-            for (int j = job - 1; j >= 0 && j >= job - kNst; --j) drain_wait(&full[j & 1], (j >> 1) & 1);
+            for (int j = job - 1; j >= 0 && j >= job - kNst; --j) drain_wait(&full[j % kNst], (j / kNst) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -484,8 +487,8 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             bool ok = mbar_wait(in_full, 0, ab, 32);
             tc_fence_after();
             auto issue_sdp = [&](int j) -> bool {
-                const int st = j & 1, sbuf = j & 1;
-                if (!mbar_wait(&full[st], (j >> 1) & 1, ab, 33)) return false;
+                const int st = j % kNst, sbuf = j & 1;
+                if (!mbar_wait(&full[st], (j / kNst) & 1, ab, 33)) return false;
                 if (!mbar_wait(&s_empty[sbuf], ((j >> 1) & 1) ^ 1, ab, 34)) return false;
                 tc_fence_after();
                 const uint64_t dqs = dst + ((st * L::kStageBytes) >> 4);
@@ -505,7 +508,7 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 if (j + 1 < njobs && !(ok = issue_sdp(j + 1))) break;
                 if (!(ok = mbar_wait(p_full, j & 1, ab, 35))) break;
                 tc_fence_after();
-                const int st = j & 1;
+                const int st = j % kNst;
                 const uint64_t qmn = dst_mn + ((st * L::kStageBytes) >> 4);
                 const uint64_t domn = qmn + (L::kSubT >> 4);
 #pragma unroll
@@ -559,22 +562,25 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             const int cmin = a.causal ? jkey - ib : 0;       // c >= cmin
             const int cmax = min(32, N - ib);                // c < cmax
             const float* tcol = tdb + half * 32;
+            if (!__all_sync(0xffffffffu, key_valid && cmin <= 0 && cmax >= 32)) {
+                // diagonal or ragged sub-tile: inadmissible columns get s = -inf (u < 0)
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    s[c] = (key_valid && c >= cmin && c < cmax) ? s[c] : -INFINITY;
+            }
             uint32_t wp[16], wd[16];
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-                float p0 = 0.f, p1 = 0.f, d0 = 0.f, d1 = 0.f;
-                if (key_valid && c >= cmin && c < cmax) {
-                    const float u = __fmaf_rn(cx, s[c], -tcol[c]);
-                    p0 = entmax_p<GM>(u, gamma);
-                    d0 = entmax_g<GM>(u, gamma) * (dp[c] - tcol[64 + c]);
-                }
-                if (key_valid && c + 1 >= cmin && c + 1 < cmax) {
-                    const float u = __fmaf_rn(cx, s[c + 1], -tcol[c + 1]);
-                    p1 = entmax_p<GM>(u, gamma);
-                    d1 = entmax_g<GM>(u, gamma) * (dp[c + 1] - tcol[64 + c + 1]);
-                }
-                wp[c >> 1] = pack_bf16(p0, p1);
-                wd[c >> 1] = pack_bf16(d0, d1);
+            for (int c = 0; c < 32; c += 4) {
+                const float4 tq = *reinterpret_cast<const float4*>(tcol + c);
+                const float4 dl = *reinterpret_cast<const float4*>(tcol + 64 + c);
+                const float u0 = __fmaf_rn(cx, s[c], -tq.x), u1 = __fmaf_rn(cx, s[c + 1], -tq.y);
+                const float u2 = __fmaf_rn(cx, s[c + 2], -tq.z), u3 = __fmaf_rn(cx, s[c + 3], -tq.w);
+                wp[c >> 1] = pack_bf16(entmax_p_bf<GM>(u0, gamma), entmax_p_bf<GM>(u1, gamma));
+                wp[(c >> 1) + 1] = pack_bf16(entmax_p_bf<GM>(u2, gamma), entmax_p_bf<GM>(u3, gamma));
+                wd[c >> 1] = pack_bf16(entmax_g_bf<GM>(u0, gamma) * (dp[c] - dl.x),
+                                       entmax_g_bf<GM>(u1, gamma) * (dp[c + 1] - dl.y));
+                wd[(c >> 1) + 1] = pack_bf16(entmax_g_bf<GM>(u2, gamma) * (dp[c + 2] - dl.z),
+                                             entmax_g_bf<GM>(u3, gamma) * (dp[c + 3] - dl.w));
             }
             if (!(ok = mbar_wait(p_empty, (j & 1) ^ 1, ab, 37))) break;
             store_half_row_sw128(smem + L::kPT, krow, half, wp);

@@ -138,12 +138,20 @@ __device__ __forceinline__ void hist_slide(C* hist, int stride, int A_old, int A
     }
 }
 
-// Bracket and start for tau from a row histogram (slots as above, top bin A,
-// max m, n admissible keys), using ptab[k] = (k/63)^gamma, k = 0..64.
-// For an edge E = e/63 the counts c_a give rigorous bounds of f:
-//   F_low(e) = sum_{a > e} c_a ptab[a-e] - 1  <=  f(E)  <=  F_up(e) = sum_{a >= e} c_a ptab[a+1-e] - 1.
-// Scanning edges down from the top bin: hi = the lowest edge with F_up <= 0,
-// lo = the first (highest) edge with F_low >= 0 (both functions are monotone).
+// Bracket and start for tau from a row histogram (top bin A, max m, n admissible
+// keys), using ptab[k] = (k/63)^gamma, k = 0..64.
+// With k = A - a (k = 0 the top bin) and the edge index j = A + 1 - e of the edge
+// E = e/63 (j = 0 the top edge), let
+//     G(j) = sum_{k < j} c_k (j - k)^gamma.
+// The bins give rigorous bounds of f at the edges:
+//     F_up(E)  = G(j)     / 63^gamma - 1  >=  f(E),
+//     F_low(E) = G(j - 1) / 63^gamma - 1  <=  f(E)
+// (every element of bin a lies in [a/63, (a+1)/63)).  G grows with j, so
+// hi = the lowest edge with F_up <= 0 (the largest j with G(j) <= 63^gamma) and
+// lo = the highest edge with F_low >= 0 (j = j* + 1 for the smallest j* with
+// G(j*) >= 63^gamma).  For an integer gamma (1..4) G comes from running moments
+// M_r = sum_{k<j} c_k k^r in one sweep over the bins (exact: double holds these
+// integers); otherwise G is evaluated directly inside two binary searches.
 // Both ends are widened by a few ulps of m against rounding in the bin
 // assignment and intersected with the plain bracket [m-1, m - n^(1-alpha)].
 // tau_0 is the root of the straight line through the bin-centre model
@@ -155,23 +163,51 @@ template <int GM, typename CountFn>
 __device__ __forceinline__ void hist_start_fn(CountFn count, int A, int ebot, float m, int n,
                                               float alpha, float gamma, const float* ptab,
                                               float& lo, float& hi, float& tau0) {
-    int h_ok = A + 1;
-    int l_ok = kNoBin;
-    for (int e = A; e >= ebot; --e) {
-        float fu = -1.f, fl = -1.f;
-        for (int a = e; a <= A; ++a) {
-            const float c = (float)count(a);
-            fu = fmaf(c, ptab[a + 1 - e], fu);
-            fl = fmaf(c, ptab[a - e], fl);
+    const int jmax = A + 1 - ebot;        // usable edges j = 0 .. jmax
+    int h_j = 0;                          // largest j with G(j) <= 63^gamma
+    int l_j = -1;                         // smallest j with G(j) >= 63^gamma
+    if (GM >= 1 && GM <= 4) {
+        double M0 = 0.0, M1 = 0.0, M2 = 0.0, M3 = 0.0, M4 = 0.0;
+        const double thr = (GM == 1) ? 63.0 : (GM == 2) ? 3969.0 : (GM == 3) ? 250047.0 : 15752961.0;
+        for (int j = 0; j <= jmax; ++j) {
+            const double x = (double)j;
+            double G;
+            if (GM == 1) G = x * M0 - M1;
+            else if (GM == 2) G = (x * M0 - 2.0 * M1) * x + M2;
+            else if (GM == 3) G = ((x * M0 - 3.0 * M1) * x + 3.0 * M2) * x - M3;
+            else G = (((x * M0 - 4.0 * M1) * x + 6.0 * M2) * x - 4.0 * M3) * x + M4;
+            if (G <= thr) h_j = j;
+            if (l_j < 0 && G >= thr) l_j = j;
+            if (j < jmax) {
+                const double c = (double)count(A - j);
+                if (c != 0.0) {
+                    M0 += c; M1 += c * x;
+                    if (GM >= 2) M2 += c * x * x;
+                    if (GM >= 3) M3 += c * x * x * x;
+                    if (GM >= 4) M4 += c * x * x * x * x;
+                }
+            }
         }
-        if (fu <= 0.f) h_ok = e;
-        if (fl >= 0.f) { l_ok = e; break; }
+    } else {
+        auto Gn = [&](int j) {   // G(j) / 63^gamma
+            float acc = 0.f;
+            for (int k = 0; k < j; ++k) acc = fmaf((float)count(A - k), ptab[j - k], acc);
+            return acc;
+        };
+        int ok_ = 0, bad = jmax + 1;               // Gn(0) = 0 <= 1; Gn(jmax+1) treated as > 1
+        while (bad - ok_ > 1) { const int mid = (ok_ + bad) >> 1; if (Gn(mid) <= 1.f) ok_ = mid; else bad = mid; }
+        h_j = ok_;
+        if (Gn(jmax) >= 1.f) {
+            int lo_ = 0, hi_ = jmax;               // Gn(0) = 0 < 1, Gn(jmax) >= 1
+            while (hi_ - lo_ > 1) { const int mid = (lo_ + hi_) >> 1; if (Gn(mid) >= 1.f) hi_ = mid; else lo_ = mid; }
+            l_j = hi_;
+        }
     }
     const float slack = 4.f * 1.1920929e-7f * fmaxf(1.f, fabsf(m));
     const float plain_lo = m - 1.f;
     const float plain_hi = m - exp2f((1.f - alpha) * __log2f((float)n));
-    lo = (l_ok != kNoBin) ? fmaxf((float)l_ok / kBinsPerUnit - slack, plain_lo) : plain_lo;
-    hi = fminf((float)h_ok / kBinsPerUnit + slack, plain_hi);
+    lo = (l_j >= 0 && l_j + 1 <= jmax) ? fmaxf((float)(A - l_j) / kBinsPerUnit - slack, plain_lo) : plain_lo;
+    hi = fminf((float)(A + 1 - h_j) / kBinsPerUnit + slack, plain_hi);
     if (hi < lo) hi = lo;
     float fcl = -1.f, fch = -1.f;
     for (int a = A; a >= ebot; --a) {

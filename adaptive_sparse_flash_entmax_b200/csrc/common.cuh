@@ -167,25 +167,29 @@ __device__ __forceinline__ void hist_start_fn(CountFn count, int A, int ebot, fl
     int h_j = 0;                          // largest j with G(j) <= 63^gamma
     int l_j = -1;                         // smallest j with G(j) >= 63^gamma
     if (GM >= 1 && GM <= 4) {
-        double M0 = 0.0, M1 = 0.0, M2 = 0.0, M3 = 0.0, M4 = 0.0;
-        const double thr = (GM == 1) ? 63.0 : (GM == 2) ? 3969.0 : (GM == 3) ? 250047.0 : 15752961.0;
-        for (int j = 0; j <= jmax; ++j) {
-            const double x = (double)j;
-            double G;
-            if (GM == 1) G = x * M0 - M1;
-            else if (GM == 2) G = (x * M0 - 2.0 * M1) * x + M2;
-            else if (GM == 3) G = ((x * M0 - 3.0 * M1) * x + 3.0 * M2) * x - M3;
-            else G = (((x * M0 - 4.0 * M1) * x + 6.0 * M2) * x - 4.0 * M3) * x + M4;
-            if (G <= thr) h_j = j;
-            if (l_j < 0 && G >= thr) l_j = j;
-            if (j < jmax) {
-                const double c = (double)count(A - j);
-                if (c != 0.0) {
-                    M0 += c; M1 += c * x;
-                    if (GM >= 2) M2 += c * x * x;
-                    if (GM >= 3) M3 += c * x * x * x;
-                    if (GM >= 4) M4 += c * x * x * x * x;
-                }
+        // counts into registers first (independent loads), then an exact sweep:
+        // finite differences of G in j are integer recurrences (64-bit: G <= 65535 * 64^4).
+        unsigned int cr[kBins];
+#pragma unroll
+        for (int k = 0; k < kBins; ++k) cr[k] = (k < jmax) ? count(A - k) : 0u;
+        const long long thr = (GM == 1) ? 63ll : (GM == 2) ? 3969ll : (GM == 3) ? 250047ll : 15752961ll;
+        // D_r(j) = sum_{k<j} c_k (j-k)^r ; D_r(j+1) = sum_{k<j} c_k (j+1-k)^r + c_j
+        //        = sum_{i<=r} C(r,i) D_i(j) + c_j     (binomial expansion of (j-k+1)^r)
+        long long D0 = 0, D1 = 0, D2 = 0, D3 = 0, D4 = 0;
+#pragma unroll
+        for (int j = 0; j <= kBins; ++j) {
+            if (j <= jmax) {
+                const long long G = (GM == 1) ? D1 : (GM == 2) ? D2 : (GM == 3) ? D3 : D4;
+                if (G <= thr) h_j = j;
+                if (l_j < 0 && G >= thr) l_j = j;
+            }
+            if (j < kBins) {
+                const long long c = (long long)cr[j];
+                if (GM >= 4) D4 = D4 + 4 * D3 + 6 * D2 + 4 * D1 + D0 + c;
+                if (GM >= 3) D3 = D3 + 3 * D2 + 3 * D1 + D0 + c;
+                if (GM >= 2) D2 = D2 + 2 * D1 + D0 + c;
+                D1 = D1 + D0 + c;
+                D0 = D0 + c;
             }
         }
     } else {

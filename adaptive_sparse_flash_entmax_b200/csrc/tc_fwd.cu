@@ -59,7 +59,7 @@ struct Layout {
     static constexpr int kBars = kXch + 4 * 2 * 128 * 4;
     static constexpr int kNumBars = 24;
     static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, decision, njobs, abort
-    static constexpr int kPtab = kMisc + 16;              // 68 floats
+    static constexpr int kPtab = kMisc + 32;              // 68 floats
     static constexpr int kLive = kPtab + 68 * 4;          // live[T], cand[T] (bytes), list[T] (int),
                                                           // per-warp block maxima [T][8] (bf16)
     __host__ __device__ static size_t r16(int T) { return (size_t)((T + 15) / 16) * 16; }
@@ -71,6 +71,8 @@ struct Misc {
     int decision;
     int njobs;      // blocks in job_list for the next pass
     int abort;
+    int inserts;    // histogram inserts of the whole tile so far (pass 0)
+    int pad[3];
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -134,6 +136,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         misc->decision = 0;
         misc->njobs = 0;
         misc->abort = 0;
+        misc->inserts = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -292,14 +295,16 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const uint32_t hinc = half ? 65536u : 1u;
         const uint32_t hkeep = half ? 0x0000FFFFu : 0xFFFF0000u;   // red.and mask clearing my half
         const float c63 = cx * kBinsPerUnit;
-        // Insert budget per half-row: a row whose window keeps filling with scores
-        // (a dense row) stops building its histogram after kInsertBudget inserts and
-        // starts from the plain bracket [m-1, m - n^(1-alpha)]: on such rows the
-        // inserts cost more than the solver pass the histogram saves (measured;
-        // narrowing the window instead of stopping was slower still).  The window
-        // width `wbins` is kept general: counts are complete for every bin inside
-        // it, so any bracket taken from it is rigorous.
-        constexpr int kInsertBudget = 48;
+        // Insert budget per tile: a tile whose windows keep filling with scores
+        // (dense rows) stops building histograms once the tile has made
+        // kTileBudget inserts, and all its rows start from the plain bracket
+        // [m-1, m - n^(1-alpha)].  The decision is tile-wide because the tile runs
+        // as many solver passes as its slowest row needs: a histogram kept for some
+        // rows only would cost the inserts without saving a pass.  On dense rows
+        // the inserts (shared-memory reductions) cost more than the pass they save
+        // (measured).  The window width `wbins` is general: counts are complete for
+        // every bin inside it, so any bracket taken from it is rigorous.
+        constexpr int kTileBudget = 128 * 2 * 24;
         int n_ins = 0;
         int wbins = kBins;                        // window width in bins (0: stopped)
         auto clear_bin = [&](int ab2) { red_shared_and_b32(hist_saddr + (ab2 & (kBins - 1)) * 512, hkeep); };
@@ -377,6 +382,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                     // Elements below the window's lowest bin (A-63)/63 <= m-1 are never in the
                     // support; blocks whose maximum is below the window are skipped as a whole.
+                    if (wbins > 0 && *reinterpret_cast<volatile int*>(&misc->inserts) > kTileBudget) {
+                        for (int sl = 0; sl < kBins; ++sl) clear_bin(sl);   // tile over budget: stop
+                        wbins = 0;
+                    }
                     const float thr_x = (float)(A - (wbins - 1)) / kBinsPerUnit - 1e-3f;
                     if (__any_sync(0xffffffffu, xm >= thr_x && wbins > 0)) {
                         // bin = floor(x*63) via the 1.5*2^23 rounding trick: rint(x*63 - 1/2)
@@ -391,12 +400,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             if (q) red_shared_add_u32(hist_saddr + (ab2 & (kBins - 1)) * 512, hinc);
                             n_ins += q;
                         }
-                        const int want = n_ins > kInsertBudget ? 0 : kBins;
-                        if (want < wbins) {
-                            // narrow the window: bins [A-w+1, A-want] leave (all of it when stopping)
-                            for (int ab2 = A - wbins + 1; ab2 <= A - want; ++ab2) clear_bin(ab2);
-                            wbins = want;
-                        }
+                        const int wsum = __reduce_add_sync(0xffffffffu, n_ins);
+                        if (lane == 0 && wsum) atomicAdd(&misc->inserts, wsum);
+                        n_ins = 0;
                     }
                 } else {
                     float f0a = 0.f, f0b = 0.f, f1a = 0.f, f1b = 0.f, f2a = 0.f, f2b = 0.f;
@@ -418,6 +424,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (!ok) break;
             if (pass == 0) {
                 // merge the two half-row histograms; the half-0 thread computes the start
+                named_bar(1, kEw);   // the tile's insert count is final
+                if (wbins > 0 && *reinterpret_cast<volatile int*>(&misc->inserts) > kTileBudget) wbins = 0;
                 X(3, half) = m;
                 X(2, half) = (float)wbins;
                 named_bar(1, kEw);

@@ -167,30 +167,28 @@ __device__ __forceinline__ void hist_start_fn(CountFn count, int A, int ebot, fl
     int h_j = 0;                          // largest j with G(j) <= 63^gamma
     int l_j = -1;                         // smallest j with G(j) >= 63^gamma
     if (GM >= 1 && GM <= 4) {
-        // counts into registers first (independent loads), then an exact sweep:
-        // finite differences of G in j are integer recurrences (64-bit: G <= 65535 * 64^4).
-        unsigned int cr[kBins];
-#pragma unroll
-        for (int k = 0; k < kBins; ++k) cr[k] = (k < jmax) ? count(A - k) : 0u;
+        // Exact sweep from the top edge down: finite differences of G in j are
+        // integer recurrences (64-bit: G <= 65535 * 64^4),
+        //   D_r(j) = sum_{k<j} c_k (j-k)^r,
+        //   D_r(j+1) = sum_{i<=r} C(r,i) D_i(j) + c_j   (binomial expansion of (j-k+1)^r).
+        // G = D_gamma grows with j, so the sweep stops at the first edge with
+        // G >= 63^gamma.  A compact loop: this code runs once per row, and an
+        // unrolled version costs more in instruction fetch than in arithmetic.
         const long long thr = (GM == 1) ? 63ll : (GM == 2) ? 3969ll : (GM == 3) ? 250047ll : 15752961ll;
-        // D_r(j) = sum_{k<j} c_k (j-k)^r ; D_r(j+1) = sum_{k<j} c_k (j+1-k)^r + c_j
-        //        = sum_{i<=r} C(r,i) D_i(j) + c_j     (binomial expansion of (j-k+1)^r)
         long long D0 = 0, D1 = 0, D2 = 0, D3 = 0, D4 = 0;
-#pragma unroll
-        for (int j = 0; j <= kBins; ++j) {
-            if (j <= jmax) {
-                const long long G = (GM == 1) ? D1 : (GM == 2) ? D2 : (GM == 3) ? D3 : D4;
-                if (G <= thr) h_j = j;
-                if (l_j < 0 && G >= thr) l_j = j;
-            }
-            if (j < kBins) {
-                const long long c = (long long)cr[j];
-                if (GM >= 4) D4 = D4 + 4 * D3 + 6 * D2 + 4 * D1 + D0 + c;
-                if (GM >= 3) D3 = D3 + 3 * D2 + 3 * D1 + D0 + c;
-                if (GM >= 2) D2 = D2 + 2 * D1 + D0 + c;
-                D1 = D1 + D0 + c;
-                D0 = D0 + c;
-            }
+        unsigned int c_next = (jmax > 0) ? count(A) : 0u;
+#pragma unroll 1
+        for (int j = 0; j <= jmax; ++j) {
+            const long long G = (GM == 1) ? D1 : (GM == 2) ? D2 : (GM == 3) ? D3 : D4;
+            if (G >= thr) { l_j = j; h_j = (G == thr) ? j : j - 1; break; }
+            h_j = j;
+            const long long c = (long long)c_next;
+            c_next = (j + 1 < jmax) ? count(A - j - 1) : 0u;
+            if (GM >= 4) D4 = D4 + 4 * D3 + 6 * D2 + 4 * D1 + D0 + c;
+            if (GM >= 3) D3 = D3 + 3 * D2 + 3 * D1 + D0 + c;
+            if (GM >= 2) D2 = D2 + 2 * D1 + D0 + c;
+            D1 = D1 + D0 + c;
+            D0 = D0 + c;
         }
     } else {
         auto Gn = [&](int j) {   // G(j) / 63^gamma
@@ -213,14 +211,16 @@ __device__ __forceinline__ void hist_start_fn(CountFn count, int A, int ebot, fl
     lo = (l_j >= 0 && l_j + 1 <= jmax) ? fmaxf((float)(A - l_j) / kBinsPerUnit - slack, plain_lo) : plain_lo;
     hi = fminf((float)(A + 1 - h_j) / kBinsPerUnit + slack, plain_hi);
     if (hi < lo) hi = lo;
+    // Bins whose centre lies below lo add nothing to either model value; with lo
+    // from the histogram those are the bins k > l_j (k = A - a).
+    const int kend = (l_j >= 0 && l_j + 1 <= jmax) ? min(jmax, l_j + 2) : jmax;
     float fcl = -1.f, fch = -1.f;
-    for (int a = A; a >= ebot; --a) {
-        const unsigned int c = count(a);
-        if (c) {
-            const float centre = ((float)a + 0.5f) / kBinsPerUnit;
-            fcl = fmaf((float)c, entmax_p<GM>(centre - lo, gamma), fcl);
-            fch = fmaf((float)c, entmax_p<GM>(centre - hi, gamma), fch);
-        }
+#pragma unroll 1
+    for (int k = 0; k < kend; ++k) {
+        const unsigned int c = count(A - k);
+        const float centre = ((float)(A - k) + 0.5f) / kBinsPerUnit;
+        fcl = fmaf((float)c, entmax_p<GM>(centre - lo, gamma), fcl);
+        fch = fmaf((float)c, entmax_p<GM>(centre - hi, gamma), fch);
     }
     float t0 = 0.5f * (lo + hi);
     if (fcl > 0.f && fch < 0.f) t0 = lo + (hi - lo) * (fcl / (fcl - fch));
@@ -264,6 +264,83 @@ __device__ __forceinline__ float entmax_g_bf(float u, float gamma) {
     if (GM == 4) return up * up * up;
     const float v = exp2f((gamma - 1.f) * __log2f(up));   // inf at up = 0 when gamma < 1 (not used)
     return (u > 0.f) ? v : 0.f;
+}
+
+// Packed (two-lane f32x2) accumulation of the power terms for the streaming
+// passes: a0 += u^gamma, a1 += u^(gamma-1), a2 += u^(gamma-2) for both lanes of
+// u, zeros where u <= 0.  The sm_100 packed FMA/ADD/MUL issue two fp32 lanes per
+// instruction.
+__device__ __forceinline__ float step_pos(float u) { return (u > 0.f) ? 1.f : 0.f; }
+
+template <int GM>
+__device__ __forceinline__ void entmax_acc_x2(float2 u, float gamma, float2& a0, float2& a1,
+                                              float2& a2) {
+    const float2 up = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
+    if (GM == 1) {
+        a0 = __fadd2_rn(a0, up);
+        a1 = __fadd2_rn(a1, make_float2(step_pos(u.x), step_pos(u.y)));
+    } else if (GM == 2) {
+        a0 = __ffma2_rn(up, up, a0);
+        a1 = __fadd2_rn(a1, up);
+        a2 = __fadd2_rn(a2, make_float2(step_pos(u.x), step_pos(u.y)));
+    } else if (GM == 3) {
+        const float2 t1 = __fmul2_rn(up, up);
+        a0 = __ffma2_rn(t1, up, a0);
+        a1 = __fadd2_rn(a1, t1);
+        a2 = __fadd2_rn(a2, up);
+    } else if (GM == 4) {
+        const float2 t2 = __fmul2_rn(up, up);
+        a0 = __ffma2_rn(t2, t2, a0);
+        a1 = __ffma2_rn(t2, up, a1);
+        a2 = __fadd2_rn(a2, t2);
+    } else {
+        const float vx = exp2f((gamma - 2.f) * __log2f(up.x));   // inf at 0 when gamma < 2
+        const float vy = exp2f((gamma - 2.f) * __log2f(up.y));
+        const float2 t2 = make_float2((u.x > 0.f) ? vx : 0.f, (u.y > 0.f) ? vy : 0.f);
+        const float2 t1 = __fmul2_rn(t2, up);
+        a0 = __ffma2_rn(t1, up, a0);
+        a1 = __fadd2_rn(a1, t1);
+        a2 = __fadd2_rn(a2, t2);
+    }
+}
+
+// Packed p = u_+^gamma for both lanes.
+template <int GM>
+__device__ __forceinline__ float2 entmax_p_x2(float2 u, float gamma) {
+    const float2 up = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
+    if (GM == 1) return up;
+    if (GM == 2) return __fmul2_rn(up, up);
+    if (GM == 3) return __fmul2_rn(__fmul2_rn(up, up), up);
+    if (GM == 4) { const float2 u2 = __fmul2_rn(up, up); return __fmul2_rn(u2, u2); }
+    return make_float2(exp2f(gamma * __log2f(up.x)), exp2f(gamma * __log2f(up.y)));
+}
+
+// Packed g = u_+^(gamma-1) for both lanes (the backward's weights).
+template <int GM>
+__device__ __forceinline__ float2 entmax_g_x2(float2 u, float gamma) {
+    const float2 up = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
+    if (GM == 1) return make_float2(step_pos(u.x), step_pos(u.y));
+    if (GM == 2) return up;
+    if (GM == 3) return __fmul2_rn(up, up);
+    if (GM == 4) return __fmul2_rn(__fmul2_rn(up, up), up);
+    const float vx = exp2f((gamma - 1.f) * __log2f(up.x)), vy = exp2f((gamma - 1.f) * __log2f(up.y));
+    return make_float2((u.x > 0.f) ? vx : 0.f, (u.y > 0.f) ? vy : 0.f);
+}
+
+// Packed p = u_+^gamma and g = u_+^(gamma-1) together.
+template <int GM>
+__device__ __forceinline__ void entmax_pg_x2(float2 u, float gamma, float2& p, float2& g) {
+    const float2 up = make_float2(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f));
+    if (GM == 1) { p = up; g = make_float2(step_pos(u.x), step_pos(u.y)); }
+    else if (GM == 2) { g = up; p = __fmul2_rn(up, up); }
+    else if (GM == 3) { g = __fmul2_rn(up, up); p = __fmul2_rn(g, up); }
+    else if (GM == 4) { const float2 t = __fmul2_rn(up, up); g = __fmul2_rn(t, up); p = __fmul2_rn(t, t); }
+    else {
+        const float lx = __log2f(up.x), ly = __log2f(up.y);
+        p = make_float2(exp2f(gamma * lx), exp2f(gamma * ly));
+        g = make_float2((u.x > 0.f) ? exp2f((gamma - 1.f) * lx) : 0.f,
+                        (u.y > 0.f) ? exp2f((gamma - 1.f) * ly) : 0.f);
+    }
 }
 
 template <int GM>

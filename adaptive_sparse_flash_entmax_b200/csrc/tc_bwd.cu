@@ -281,6 +281,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float tau = row_valid ? a.tau[(size_t)bh * N + i] : 0.f;
         float* xch = reinterpret_cast<float*>(smem + L::kXch);   // [2][2][128]
         float sg = 0.f, sgdp = 0.f, delta = 0.f;
+        const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-tau, -tau);
         bool ok = true;
         for (int j = 0; j < total && ok; ++j) {
             const int sbuf = j % kSbufDq;
@@ -301,16 +302,17 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int c = 0; c < 32; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
             }
             if (j < njobs) {
-                float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+                float2 a0 = make_float2(0.f, 0.f), b0 = a0, a1 = a0, b1 = a0;
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float g0 = entmax_g_bf<GM>(__fmaf_rn(cx, s[c], -tau), gamma);
-                    const float g1 = entmax_g_bf<GM>(__fmaf_rn(cx, s[c + 1], -tau), gamma);
-                    a0 += g0; a1 += g1;
-                    b0 = fmaf(g0, dp[c], b0); b1 = fmaf(g1, dp[c + 1], b1);
+                for (int c = 0; c < 32; c += 4) {
+                    const float2 g0 = entmax_g_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma);
+                    const float2 g1 = entmax_g_x2<GM>(__ffma2_rn(make_float2(s[c + 2], s[c + 3]), cx2, nt2), gamma);
+                    a0 = __fadd2_rn(a0, g0); b0 = __ffma2_rn(g0, make_float2(dp[c], dp[c + 1]), b0);
+                    a1 = __fadd2_rn(a1, g1); b1 = __ffma2_rn(g1, make_float2(dp[c + 2], dp[c + 3]), b1);
                 }
-                sg += a0 + a1;
-                sgdp += b0 + b1;
+                a0 = __fadd2_rn(a0, a1); b0 = __fadd2_rn(b0, b1);
+                sg += a0.x + a0.y;
+                sgdp += b0.x + b0.y;
                 if (j == njobs - 1) {
                     xch[(0 * 2 + half) * 128 + row] = sg;
                     xch[(1 * 2 + half) * 128 + row] = sgdp;
@@ -322,15 +324,15 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             } else {
                 uint32_t whi[16], wlo[16];
+                const float2 nd2 = make_float2(-delta, -delta), m1 = make_float2(-1.f, -1.f);
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const float g0 = entmax_g_bf<GM>(__fmaf_rn(cx, s[c], -tau), gamma);
-                    const float g1 = entmax_g_bf<GM>(__fmaf_rn(cx, s[c + 1], -tau), gamma);
-                    const float d0 = g0 * (dp[c] - delta), d1 = g1 * (dp[c + 1] - delta);
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(d0, d1);
-                    const float2 hf = __bfloat1622float2(h);
+                    const float2 g = entmax_g_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma);
+                    const float2 d = __fmul2_rn(g, __fadd2_rn(make_float2(dp[c], dp[c + 1]), nd2));
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(d.x, d.y);
+                    const float2 lo = __ffma2_rn(__bfloat1622float2(h), m1, d);   // d - bf16(d), exact
                     whi[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-                    wlo[c >> 1] = pack_bf16(d0 - hf.x, d1 - hf.y);
+                    wlo[c >> 1] = pack_bf16(lo.x, lo.y);
                 }
                 const int bj = j - njobs;
                 if (!(ok = mbar_wait(ds_empty, (bj & 1) ^ 1, ab, 27))) break;
@@ -541,8 +543,8 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             float* tdb = td + (j & 1) * 128;
             if (ew < 64) {
                 const int ii = i0 + ew;
-                tdb[ew] = ii < N ? a.tau[(size_t)bh * N + ii] : 0.f;
-                tdb[64 + ew] = ii < N ? a.delta[(size_t)bh * N + ii] : 0.f;
+                tdb[ew] = ii < N ? -a.tau[(size_t)bh * N + ii] : 0.f;         // -tau
+                tdb[64 + ew] = ii < N ? -a.delta[(size_t)bh * N + ii] : 0.f;  // -delta
             }
             named_bar(1, kEw);
             const int sbuf = j & 1;
@@ -569,18 +571,22 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     s[c] = (key_valid && c >= cmin && c < cmax) ? s[c] : -INFINITY;
             }
             uint32_t wp[16], wd[16];
+            const float2 cx2 = make_float2(cx, cx);
 #pragma unroll
             for (int c = 0; c < 32; c += 4) {
-                const float4 tq = *reinterpret_cast<const float4*>(tcol + c);
-                const float4 dl = *reinterpret_cast<const float4*>(tcol + 64 + c);
-                const float u0 = __fmaf_rn(cx, s[c], -tq.x), u1 = __fmaf_rn(cx, s[c + 1], -tq.y);
-                const float u2 = __fmaf_rn(cx, s[c + 2], -tq.z), u3 = __fmaf_rn(cx, s[c + 3], -tq.w);
-                wp[c >> 1] = pack_bf16(entmax_p_bf<GM>(u0, gamma), entmax_p_bf<GM>(u1, gamma));
-                wp[(c >> 1) + 1] = pack_bf16(entmax_p_bf<GM>(u2, gamma), entmax_p_bf<GM>(u3, gamma));
-                wd[c >> 1] = pack_bf16(entmax_g_bf<GM>(u0, gamma) * (dp[c] - dl.x),
-                                       entmax_g_bf<GM>(u1, gamma) * (dp[c + 1] - dl.y));
-                wd[(c >> 1) + 1] = pack_bf16(entmax_g_bf<GM>(u2, gamma) * (dp[c + 2] - dl.z),
-                                             entmax_g_bf<GM>(u3, gamma) * (dp[c + 3] - dl.w));
+                const float4 ntq = *reinterpret_cast<const float4*>(tcol + c);        // -tau
+                const float4 ndl = *reinterpret_cast<const float4*>(tcol + 64 + c);   // -delta
+                float2 p0, g0, p1, g1;
+                entmax_pg_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, make_float2(ntq.x, ntq.y)),
+                                 gamma, p0, g0);
+                entmax_pg_x2<GM>(__ffma2_rn(make_float2(s[c + 2], s[c + 3]), cx2, make_float2(ntq.z, ntq.w)),
+                                 gamma, p1, g1);
+                const float2 d0 = __fmul2_rn(g0, __fadd2_rn(make_float2(dp[c], dp[c + 1]), make_float2(ndl.x, ndl.y)));
+                const float2 d1 = __fmul2_rn(g1, __fadd2_rn(make_float2(dp[c + 2], dp[c + 3]), make_float2(ndl.z, ndl.w)));
+                wp[c >> 1] = pack_bf16(p0.x, p0.y);
+                wp[(c >> 1) + 1] = pack_bf16(p1.x, p1.y);
+                wd[c >> 1] = pack_bf16(d0.x, d0.y);
+                wd[(c >> 1) + 1] = pack_bf16(d1.x, d1.y);
             }
             if (!(ok = mbar_wait(p_empty, (j & 1) ^ 1, ab, 37))) break;
             store_half_row_sw128(smem + L::kPT, krow, half, wp);

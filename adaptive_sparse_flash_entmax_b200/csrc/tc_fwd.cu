@@ -297,7 +297,9 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const float c63 = cx * kBinsPerUnit;
         // Insert budget per tile: a tile whose windows keep filling with scores
         // (dense rows) stops building histograms once the tile has made
-        // kTileBudget inserts, and all its rows start from the plain bracket
+        // kTileBudget inserts after its first block (the first block's window
+        // hangs from that block's own maximum and takes in most of it whatever
+        // the rows look like), and all its rows start from the plain bracket
         // [m-1, m - n^(1-alpha)].  The decision is tile-wide because the tile runs
         // as many solver passes as its slowest row needs: a histogram kept for some
         // rows only would cost the inserts without saving a pass.  On dense rows
@@ -401,21 +403,21 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             n_ins += q;
                         }
                         const int wsum = __reduce_add_sync(0xffffffffu, n_ins);
-                        if (lane == 0 && wsum) atomicAdd(&misc->inserts, wsum);
+                        if (lane == 0 && wsum && jj > 0) atomicAdd(&misc->inserts, wsum);
                         n_ins = 0;
                     }
                 } else {
-                    float f0a = 0.f, f0b = 0.f, f1a = 0.f, f1b = 0.f, f2a = 0.f, f2b = 0.f;
+                    // two packed accumulator sets (columns c mod 4 < 2 and >= 2)
+                    float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, b0 = a0, b1 = a0, b2 = a0;
+                    const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-sv.tau, -sv.tau);
 #pragma unroll
-                    for (int c = 0; c < 64; c += 2) {
-                        float t0, t1, t2, q0, q1, q2;
-                        entmax_terms_bf<GM>(__fmaf_rn(cx, s[c], -sv.tau), gamma, t0, t1, t2);
-                        entmax_terms_bf<GM>(__fmaf_rn(cx, s[c + 1], -sv.tau), gamma, q0, q1, q2);
-                        f0a += t0; f1a += t1; f2a += t2;
-                        f0b += q0; f1b += q1; f2b += q2;
+                    for (int c = 0; c < 64; c += 4) {
+                        entmax_acc_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma, a0, a1, a2);
+                        entmax_acc_x2<GM>(__ffma2_rn(make_float2(s[c + 2], s[c + 3]), cx2, nt2), gamma, b0, b1, b2);
                     }
-                    const float f1 = f1a + f1b;
-                    F0 += f0a + f0b; F1 += f1; F2 += f2a + f2b;
+                    a0 = __fadd2_rn(a0, b0); a1 = __fadd2_rn(a1, b1); a2 = __fadd2_rn(a2, b2);
+                    const float f1 = a1.x + a1.y;
+                    F0 += a0.x + a0.y; F1 += f1; F2 += a2.x + a2.y;
                     // liveness: t1 = u^(gamma-1) > 0 exactly where u > 0 (up to underflow,
                     // where p = u^gamma is 0 as well)
                     if (__any_sync(0xffffffffu, f1 > 0.f) && lane == 0) live[b] = 1;
@@ -518,13 +520,16 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_empty[sb]);
                 const int nv = key_end - b * kBlk - c0;
+                if (!__all_sync(0xffffffffu, nv >= 64)) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
+                }
                 uint32_t pk[32];
+                const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-sv.tau, -sv.tau);
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
-                    const float u0 = (c < nv) ? __fmaf_rn(cx, s[c], -sv.tau) : -1.f;
-                    const float u1 = (c + 1 < nv) ? __fmaf_rn(cx, s[c + 1], -sv.tau) : -1.f;
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(entmax_p_bf<GM>(u0, gamma),
-                                                                    entmax_p_bf<GM>(u1, gamma));
+                    const float2 p2 = entmax_p_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma);
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(p2.x, p2.y);
                     pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
                 }
                 if (!(ok = mbar_wait(p_empty, (li & 1) ^ 1, ab, 10))) break;

@@ -4,18 +4,19 @@
 // Technical Deep Dive / AdaSplash: Fused GPU Kernel for Attention: the Q tile is
 // loaded once and stays on chip; K tiles stream for the tau passes; a final pass
 // streams K and V and accumulates O = P V).  Warp roles:
-//   warp 0   TMA producer: Q once, then K blocks into a four-slot ring during
-//            the score passes, or (K, V) pairs into two stages (the same memory)
-//            in the P.V pass;
+//   warp 0   TMA producer: Q once, then tiles into a four-slot ring: K blocks
+//            in the score passes, K and V of each live block in the P.V pass;
 //   warp 1   MMA issuer: S = Q K^T into three TMEM accumulators (128 x 128
-//            fp32), and O += P V (P from shared memory, V MN-major);
+//            fp32), and O += P V with P read from TMEM (it replaces S in its
+//            buffer) and V from shared memory (MN-major);
 //   warps 2-9 elementwise: two threads per query row (= TMEM lane), 64 columns
 //            each.  Pass 0 builds the
 //            row max and the sliding 64-bin histogram ("AdaSplash-2: ...",
 //            Sparse Attention Makes Waves); solver passes accumulate
 //            F0, F1, F2 and take a Halley-bisection step (Accelerated Alpha-Entmax
 //            Transformation); the last solver pass marks live key blocks
-//            (Exploiting Sparsity); the P.V pass writes P (bf16) for live blocks.
+//            (Exploiting Sparsity); the P.V pass writes P (bf16) for live blocks
+//            into TMEM.
 // Solver passes visit only candidate blocks: pass 0 records each warp's block
 // maximum of x, and a block is streamed again only if some warp's maximum
 // exceeds that warp's smallest current tau (otherwise no row of the tile has
@@ -35,8 +36,7 @@ using namespace tc;
 
 namespace {
 
-constexpr int kSlots = 4;          // K slots of the score-pass ring
-constexpr int kPvStages = 2;       // (K, V) stages of the P.V pass (same memory as the slots)
+constexpr int kSlots = 4;          // tile slots of the K / V ring
 constexpr int kSbuf = 3;           // S accumulators in TMEM
 constexpr int kThreads = 320;      // 10 warps
 constexpr int kEw = 256;           // elementwise threads (warps 2-9): two per query row
@@ -51,10 +51,9 @@ template <int D>
 struct Layout {
     static constexpr int kTile = D / 64 * kAtom;          // [128 x D] bf16
     static constexpr int kQ = 0;
-    static constexpr int kRing = kQ + kTile;              // kSlots tiles: score-pass K slots,
-                                                          // or two (K, V) stages in the P.V pass
-    static constexpr int kP = kRing + kSlots * kTile;     // P [128 x 128] bf16; in pass 0 the two
-    static constexpr int kPBytes = 2 * kAtom;             // half-row histograms [64][128] u16
+    static constexpr int kRing = kQ + kTile;              // kSlots tiles (K or V blocks)
+    static constexpr int kP = kRing + kSlots * kTile;     // pass 0: the two half-row
+    static constexpr int kPBytes = 2 * kAtom;             // histograms [64][128] u16
     static constexpr int kXch = kP + kPBytes;             // [4][2][128] f32 exchange
     static constexpr int kBars = kXch + 4 * 2 * 128 * 4;
     static constexpr int kNumBars = 24;
@@ -97,15 +96,13 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-    uint64_t* kfull = bars;                    // [kSlots]     TMA -> MMA (score passes)
+    uint64_t* kfull = bars;                    // [kSlots]     TMA -> MMA
     uint64_t* kempty = kfull + kSlots;         // [kSlots]     MMA -> TMA
-    uint64_t* pvfull = kempty + kSlots;        // [kPvStages]  TMA -> MMA (P.V pass)
-    uint64_t* pvempty = pvfull + kPvStages;    // [kPvStages]  MMA -> TMA
-    uint64_t* s_full = pvempty + kPvStages;    // [kSbuf]      MMA -> elementwise
-    uint64_t* s_empty = s_full + kSbuf;        // [kSbuf]      elementwise -> MMA
-    uint64_t* p_full = s_empty + kSbuf;        //              elementwise -> MMA
-    uint64_t* p_empty = p_full + 1;            //              MMA -> elementwise
-    uint64_t* o_full = p_empty + 1;            //              MMA -> elementwise
+    uint64_t* s_full = kempty + kSlots;        // [kSbuf]      MMA -> elementwise
+    uint64_t* s_empty = s_full + kSbuf;        // [kSbuf]      elementwise -> MMA (score passes)
+    uint64_t* pv_sfree = s_empty + kSbuf;      // [kSbuf]      MMA -> MMA (P.V pass: P(i) consumed)
+    uint64_t* p_full = pv_sfree + kSbuf;       // [kSbuf]      elementwise -> MMA (P(i) in TMEM)
+    uint64_t* o_full = p_full + kSbuf;         //              MMA -> elementwise
     uint64_t* q_full = o_full + 1;             //              TMA -> MMA
     uint64_t* dec_bar = q_full + 1;            //              elementwise -> TMA, MMA
     uint64_t* mma_done = dec_bar + 1;          //              MMA -> MMA (all MMAs retired)
@@ -125,10 +122,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSlots; ++s) { mbar_init(&kfull[s], 1); mbar_init(&kempty[s], 1); }
-        for (int s = 0; s < kPvStages; ++s) { mbar_init(&pvfull[s], 1); mbar_init(&pvempty[s], 1); }
-        for (int s = 0; s < kSbuf; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps); }
-        mbar_init(p_full, kEwWarps);
-        mbar_init(p_empty, 1);
+        for (int s = 0; s < kSbuf; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], kEwWarps);
+            mbar_init(&pv_sfree[s], 1);
+            mbar_init(&p_full[s], kEwWarps);
+        }
         mbar_init(o_full, 1);
         mbar_init(q_full, 1);
         mbar_init(dec_bar, 1);
@@ -158,34 +157,26 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_arrive_expect_tx(q_full, L::kTile);
             for (int at = 0; at < D / 64; ++at)
                 tma_load_3d(smem + L::kQ + at * kAtom, &tm_q, at * 64, t * kBlk, bh, q_full);
-            int sj = 0, pj = 0, kind = kDecSolve;   // score-pass and P.V-pass load counters
+            int sj = 0, kind = kDecSolve;   // tiles loaded into the ring so far
             uint32_t dec_phase = 0;
             bool ok = true, first = true;
+            auto load_tile = [&](const CUtensorMap* map, int b) -> bool {
+                const int sl = sj % kSlots;
+                if (!mbar_wait(&kempty[sl], ((sj / kSlots) & 1) ^ 1, ab, 1)) return false;
+                mbar_arrive_expect_tx(&kfull[sl], L::kTile);
+                uint8_t* kb = smem + L::kRing + sl * L::kTile;
+                for (int at = 0; at < D / 64; ++at)
+                    tma_load_3d(kb + at * kAtom, map, at * 64, b * kBlk, bh, &kfull[sl]);
+                ++sj;
+                return true;
+            };
             while (ok) {
                 const bool pv = kind == kDecPv;
                 const int njobs = first ? nblk : misc->njobs;
                 for (int i = 0; i < njobs && ok; ++i) {
                     const int b = first ? i : job_list[i];
-                    if (!pv) {
-                        const int sl = sj % kSlots;
-                        if (!(ok = mbar_wait(&kempty[sl], ((sj / kSlots) & 1) ^ 1, ab, 1))) break;
-                        mbar_arrive_expect_tx(&kfull[sl], L::kTile);
-                        uint8_t* kb = smem + L::kRing + sl * L::kTile;
-                        for (int at = 0; at < D / 64; ++at)
-                            tma_load_3d(kb + at * kAtom, &tm_k, at * 64, b * kBlk, bh, &kfull[sl]);
-                        ++sj;
-                    } else {
-                        const int st = pj % kPvStages;
-                        if (!(ok = mbar_wait(&pvempty[st], ((pj / kPvStages) & 1) ^ 1, ab, 1))) break;
-                        mbar_arrive_expect_tx(&pvfull[st], 2 * L::kTile);
-                        uint8_t* kb = smem + L::kRing + st * 2 * L::kTile;
-                        for (int at = 0; at < D / 64; ++at) {
-                            tma_load_3d(kb + at * kAtom, &tm_k, at * 64, b * kBlk, bh, &pvfull[st]);
-                            tma_load_3d(kb + L::kTile + at * kAtom, &tm_v, at * 64, b * kBlk, bh,
-                                        &pvfull[st]);
-                        }
-                        ++pj;
-                    }
+                    ok = load_tile(&tm_k, b);
+                    if (ok && pv) ok = load_tile(&tm_v, b);
                 }
                 first = false;
                 if (!ok || pv) break;
@@ -196,8 +187,6 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // Copies issued but possibly not consumed land before the CTA ends.
             drain_wait(q_full, 0);
             for (int j = sj - 1; j >= 0 && j >= sj - kSlots; --j) drain_wait(&kfull[j % kSlots], (j / kSlots) & 1);
-            for (int j = pj - 1; j >= 0 && j >= pj - kPvStages; --j)
-                drain_wait(&pvfull[j % kPvStages], (j / kPvStages) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -207,66 +196,82 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // Descriptors differ only in the start-address field (bits 0-13, address >> 4),
             // so each operand's base descriptor is built once and offsets are added.
             const uint64_t dq = sdesc_sw128(smem_u32(smem + L::kQ), 16, 1024);
-            const uint64_t dp = sdesc_sw128(smem_u32(smem + L::kP), 16, 1024);
             const uint64_t dring = sdesc_sw128(smem_u32(smem + L::kRing), 16, 1024);
             const uint64_t dring_mn = sdesc_sw128(smem_u32(smem + L::kRing), kAtom, 1024);
             bool ok = mbar_wait(q_full, 0, ab, 3);
             tc_fence_after();
-            int job = 0, sj = 0, pj = 0, kind = kDecSolve;
+            int job = 0, sj = 0, kind = kDecSolve;   // S jobs issued; ring tiles consumed
             uint32_t dec_phase = 0;
             bool first = true;
+            auto wait_tile = [&](int tt) { return mbar_wait(&kfull[tt % kSlots], (tt / kSlots) & 1, ab, 4); };
+            auto issue_s = [&](int sb, int tt) {
+                const uint64_t dk = dring + ((uint32_t)((tt % kSlots) * L::kTile) >> 4);
+                const uint32_t dS = tmem + sbuf_col(sb);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
+                    umma_bf16(dS, dq + off, dk + off, idesc_qk, kk > 0);
+                }
+                umma_commit(&s_full[sb]);
+                umma_commit(&kempty[tt % kSlots]);
+            };
             while (ok) {
                 const bool pv = kind == kDecPv;
                 const int njobs = first ? nblk : misc->njobs;
                 first = false;
-                for (int i = 0; i < njobs && ok; ++i, ++job) {
-                    const int sb = job % kSbuf;
-                    uint32_t kofs;   // byte offset of the K tile from the ring start
-                    if (!pv) {
-                        const int sl = sj % kSlots;
-                        if (!(ok = mbar_wait(&kfull[sl], (sj / kSlots) & 1, ab, 4))) break;
-                        kofs = sl * L::kTile;
-                    } else {
-                        const int st = pj % kPvStages;
-                        if (!(ok = mbar_wait(&pvfull[st], (pj / kPvStages) & 1, ab, 4))) break;
-                        kofs = st * 2 * L::kTile;
+                if (!pv) {
+                    for (int i = 0; i < njobs && ok; ++i, ++job, ++sj) {
+                        const int sb = job % kSbuf;
+                        if (!(ok = wait_tile(sj))) break;
+                        if (!(ok = mbar_wait(&s_empty[sb], ((job / kSbuf) & 1) ^ 1, ab, 5))) break;
+                        tc_fence_after();
+                        issue_s(sb, sj);
                     }
-                    if (!(ok = mbar_wait(&s_empty[sb], ((job / kSbuf) & 1) ^ 1, ab, 5))) break;
-                    tc_fence_after();
-                    const uint64_t dk = dring + (kofs >> 4);
-                    const uint32_t dS = tmem + sbuf_col(sb);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
-                        umma_bf16(dS, dq + off, dk + off, idesc_qk, kk > 0);
-                    }
-                    umma_commit(&s_full[sb]);
-                    if (!pv) {
-                        umma_commit(&kempty[sj % kSlots]);
-                        ++sj;
-                        continue;
-                    }
-                    if (!(ok = mbar_wait(p_full, pj & 1, ab, 6))) break;
-                    tc_fence_after();
-                    const uint64_t dv = dring_mn + ((kofs + L::kTile) >> 4);
-#pragma unroll
-                    for (int kk = 0; kk < kBlk / 16; ++kk) {
-                        const uint32_t aoff = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
-                        umma_bf16(tmem + 256, dp + aoff, dv + ((kk * 16 * 128) >> 4), idesc_pv,
-                                  (pj > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    umma_commit(p_empty);
-                    umma_commit(&pvempty[pj % kPvStages]);
-                    ++pj;
+                    if (!ok) break;
+                    if (!(ok = mbar_wait(dec_bar, dec_phase, ab, 7))) break;
+                    dec_phase ^= 1;
+                    kind = misc->decision;
+                    continue;
                 }
-                if (!ok) break;
-                if (pv) {
-                    umma_commit(o_full);
-                    break;
+                // P.V pass over the live blocks; ring tiles K_i = sj + 2i, V_i = sj + 2i + 1.
+                // S(i) is issued ahead of P.V(i-1), so the score MMA of the next block
+                // runs while the elementwise warps turn S(i-1) into P(i-1).  P(i)
+                // replaces S(i) in its TMEM buffer, which is free again once P.V(i)
+                // is done (pv_sfree); a buffer's first use in this pass waits for the
+                // elementwise release of its last score-pass job instead.
+                for (int i = 0; i <= njobs && ok; ++i) {
+                    if (i < njobs) {
+                        const int jb = job + i, sb = jb % kSbuf;
+                        if (!(ok = wait_tile(sj + 2 * i))) break;
+                        ok = (i < kSbuf) ? mbar_wait(&s_empty[sb], ((jb / kSbuf) & 1) ^ 1, ab, 5)
+                                         : mbar_wait(&pv_sfree[sb], ((i / kSbuf) - 1) & 1, ab, 5);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(sb, sj + 2 * i);
+                    }
+                    if (i > 0) {
+                        const int ip = i - 1, sb = (job + ip) % kSbuf, tv = sj + 2 * ip + 1;
+                        if (!(ok = wait_tile(tv))) break;
+                        // one p_full per buffer: P(i+3) cannot complete before P.V(i) frees
+                        // the buffer, so the elementwise warps never lap this wait
+                        if (!(ok = mbar_wait(&p_full[sb], (ip / kSbuf) & 1, ab, 6))) break;
+                        tc_fence_after();
+                        const uint64_t dv = dring_mn + ((uint32_t)((tv % kSlots) * L::kTile) >> 4);
+                        const uint32_t ap = tmem + sbuf_col(sb);
+#pragma unroll
+                        for (int kk = 0; kk < kBlk / 16; ++kk) {
+                            // keys 16kk .. 16kk+15: the half (kk >> 2) that owns them wrote
+                            // their P, two per column, into its own first 32 columns
+                            const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
+                            umma_bf16_ts(tmem + 256, ap + acol, dv + ((kk * 16 * 128) >> 4), idesc_pv,
+                                         (ip > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&pv_sfree[sb]);
+                        umma_commit(&kempty[tv % kSlots]);
+                    }
                 }
-                if (!(ok = mbar_wait(dec_bar, dec_phase, ab, 7))) break;
-                dec_phase ^= 1;
-                kind = misc->decision;
+                if (ok) umma_commit(o_full);
+                break;
             }
             // every issued MMA retires before TMEM is freed
             umma_commit(mma_done);
@@ -516,9 +521,6 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tmem_ld32(lane_base + sbuf_col(sb) + c0 + 32, &s[32]);
                 tmem_wait_ld();
                 reg_fence<64>(s);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[sb]);
                 const int nv = key_end - b * kBlk - c0;
                 if (!__all_sync(0xffffffffu, nv >= 64)) {
 #pragma unroll
@@ -532,15 +534,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(p2.x, p2.y);
                     pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
                 }
-                if (!(ok = mbar_wait(p_empty, (li & 1) ^ 1, ab, 10))) break;
-                uint8_t* prow = smem + L::kP + half * kAtom + row * 128;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)   // 16-byte chunk = 8 keys
-                    *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
-                        make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-                fence_proxy_async_smem();
+                // P over this thread's own S columns: keys c0 .. c0+63 -> columns c0 .. c0+31
+                tmem_st32(lane_base + sbuf_col(sb) + c0, pk);
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(p_full);
+                if (lane == 0) mbar_arrive(&p_full[sb]);
             }
         }
         // epilogue: this thread's half of the O row, tau, iters, mask row, counters

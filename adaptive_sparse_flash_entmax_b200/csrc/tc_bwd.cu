@@ -9,18 +9,19 @@
 // Only the 128 x 128 blocks marked live by the forward's block mask are visited.
 //
 // Two kernels, both with warp roles (warp 0 TMA, warp 1 MMA issuer, warps 2-9
-// elementwise, two threads per TMEM lane) and 64-wide sub-tiles so that two stages,
-// double-buffered TMEM accumulators and the bf16 operand written by the
-// elementwise warps fit on chip:
+// elementwise, two threads per TMEM lane) and 64-wide sub-tiles so that three
+// stages and several TMEM accumulator pairs fit on chip.  The bf16 operand the
+// elementwise warps produce (dS, P^T, dS^T) is written into TMEM over the S
+// columns it came from, and the MMA reads it from there as its A operand:
 //   dq kernel   one CTA per 128-row query tile, K/V in 64-key sub-blocks of
 //               the live blocks.  Phase A: S = Q K^T, dP = dO V^T -> delta per
 //               row (also written to the workspace).  Phase B: again S and dP,
-//               dS as a pair of bf16 parts (hi + lo, shared memory) and
-//               dQ += dS K (K read MN-major).
+//               dS as a pair of bf16 parts (hi + lo) and dQ += dS K (K read
+//               MN-major).
 //   dkv kernel  one CTA per 128-key block, Q/dO in 64-row sub-tiles of the
 //               live query tiles.  S^T = K Q^T, dP^T = V dO^T, then P^T and
-//               dS^T (bf16, shared memory) and dV += P^T dO, dK += dS^T Q (dO
-//               and Q read MN-major from the same tiles that fed S^T and dP^T).
+//               dS^T (bf16) and dV += P^T dO, dK += dS^T Q (dO and Q read
+//               MN-major from the same tiles that fed S^T and dP^T).
 // All waits are bounded as in the forward.
 #include <cudaTypedefs.h>
 
@@ -69,27 +70,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Write 64 bf16 values (32 packed words) as one 128-byte row `row` of a
-// K-major 128-byte-swizzled atom starting at `atom`.
-__device__ __forceinline__ void store_row_sw128(uint8_t* atom, int row, const uint32_t* w) {
-    uint8_t* base = atom + row * 128;
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(base + ((ch ^ (row & 7)) << 4)) =
-            make_uint4(w[ch * 4], w[ch * 4 + 1], w[ch * 4 + 2], w[ch * 4 + 3]);
-}
-
-// Write 32 bf16 values (16 packed words): chunks 4*half .. 4*half+3 of row `row`.
-__device__ __forceinline__ void store_half_row_sw128(uint8_t* atom, int row, int half, const uint32_t* w) {
-    uint8_t* base = atom + row * 128;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int ch = half * 4 + q;
-        *reinterpret_cast<uint4*>(base + ((ch ^ (row & 7)) << 4)) =
-            make_uint4(w[q * 4], w[q * 4 + 1], w[q * 4 + 2], w[q * 4 + 3]);
-    }
-}
-
 __device__ __forceinline__ void store_out_row(void* out, size_t off, const float* v, int D, float sc) {
     __nv_bfloat16* p = static_cast<__nv_bfloat16*>(out) + off;
     for (int c = 0; c < D; c += 8) {
@@ -112,10 +92,9 @@ struct DqLayout {
     static constexpr int kDO = kQ + kTile;
     static constexpr int kStage0 = kDO + kTile;
     static constexpr int kStageBytes = 2 * kSubT;       // K_sub, V_sub
-    static constexpr int kDS = kStage0 + kNst * kStageBytes;   // dS hi, dS lo: [128 x 64] bf16 atoms
-    static constexpr int kXch = kDS + 2 * kAtom128;            // [2][2][128] f32
+    static constexpr int kXch = kStage0 + kNst * kStageBytes;  // [2][2][128] f32
     static constexpr int kBars = kXch + 2 * 2 * 128 * 4;
-    static constexpr int kMisc = kBars + 8 * 16;
+    static constexpr int kMisc = kBars + 8 * 24;   // up to 24 mbarriers
     static constexpr int kList = kMisc + 16;            // int job list [2*T]
     static size_t bytes(int T) { return (size_t)kList + 8 * (size_t)T + 1024; }
 };
@@ -131,11 +110,11 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
     uint64_t* full = bars;                     // [kNst]
     uint64_t* empty = full + kNst;             // [kNst]
-    uint64_t* s_full = empty + kNst;           // [kSbufDq]
-    uint64_t* s_empty = s_full + kSbufDq;      // [kSbufDq]
-    uint64_t* ds_full = s_empty + kSbufDq;
-    uint64_t* ds_empty = ds_full + 1;
-    uint64_t* acc_full = ds_empty + 1;
+    uint64_t* s_full = empty + kNst;           // [kSbufDq]  MMA -> elementwise
+    uint64_t* s_empty = s_full + kSbufDq;      // [kSbufDq]  elementwise -> MMA (phase A jobs)
+    uint64_t* ds_full = s_empty + kSbufDq;     // [kSbufDq]  elementwise -> MMA (dS in TMEM)
+    uint64_t* ds_free = ds_full + kSbufDq;     // [kSbufDq]  MMA -> MMA (dQ of a phase B job done)
+    uint64_t* acc_full = ds_free + kSbufDq;
     uint64_t* in_full = acc_full + 1;          // Q and dO tiles
     uint64_t* mma_done = in_full + 1;
     Misc* misc = reinterpret_cast<Misc*>(smem + L::kMisc);
@@ -151,9 +130,12 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kNst; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int s = 0; s < kSbufDq; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps); }
-        mbar_init(ds_full, kEwWarps);
-        mbar_init(ds_empty, 1);
+        for (int s = 0; s < kSbufDq; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], kEwWarps);
+            mbar_init(&ds_full[s], kEwWarps);
+            mbar_init(&ds_free[s], 1);
+        }
         mbar_init(acc_full, 1);
         mbar_init(in_full, 1);
         mbar_init(mma_done, 1);
@@ -214,16 +196,21 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // base descriptors; operands differ only by start-address offsets
             const uint64_t dq_ = sdesc_sw128(smem_u32(smem + L::kQ), 16, 1024);
             const uint64_t ddo = sdesc_sw128(smem_u32(smem + L::kDO), 16, 1024);
-            const uint64_t dds = sdesc_sw128(smem_u32(smem + L::kDS), 16, 1024);
             const uint64_t dst = sdesc_sw128(smem_u32(smem + L::kStage0), 16, 1024);
             const uint64_t dst_mn = sdesc_sw128(smem_u32(smem + L::kStage0), kAtom64, 1024);
             bool ok = mbar_wait(in_full, 0, ab, 22);
             tc_fence_after();
-            // issue S and dP of job j into TMEM pair j % kSbufDq
+            // issue S and dP of job j into TMEM pair j % kSbufDq.  The pair is free once
+            // the previous job on it is done with it: a phase A job when the elementwise
+            // warps have read S and dP, a phase B job when the dQ MMA has read its dS.
             auto issue_sdp = [&](int j) -> bool {
                 const int st = j % kNst, sbuf = j % kSbufDq;
                 if (!mbar_wait(&full[st], (j / kNst) & 1, ab, 23)) return false;
-                if (!mbar_wait(&s_empty[sbuf], ((j / kSbufDq) & 1) ^ 1, ab, 24)) return false;
+                const int jp = j - kSbufDq;
+                const bool fr = (jp < njobs)
+                                    ? mbar_wait(&s_empty[sbuf], ((j / kSbufDq) & 1) ^ 1, ab, 24)
+                                    : mbar_wait(&ds_free[sbuf], ((jp - njobs) / kSbufDq) & 1, ab, 24);
+                if (!fr) return false;
                 tc_fence_after();
                 const uint64_t dk = dst + ((st * L::kStageBytes) >> 4);
                 const uint64_t dv = dk + (L::kSubT >> 4);
@@ -247,19 +234,23 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     continue;
                 }
                 const int bj = j - njobs;        // phase B job: dQ += dS K
-                if (!(ok = mbar_wait(ds_full, bj & 1, ab, 25))) break;
+                const int sbuf = j % kSbufDq;
+                // one ds_full per pair: dS(j+3) cannot complete before dQ(j) frees the pair
+                if (!(ok = mbar_wait(&ds_full[sbuf], (bj / kSbufDq) & 1, ab, 25))) break;
                 tc_fence_after();
                 const uint64_t dkmn = dst_mn + ((st * L::kStageBytes) >> 4);
                 // dQ += (dS_hi + dS_lo) K: the two bf16 parts carry dS to ~16 bits, which
-                // the cancellation in sum_j dS_ij k_j (rows of dS sum to 0) needs.
+                // the cancellation in sum_j dS_ij k_j (rows of dS sum to 0) needs.  The
+                // half (kk >> 1) that owns keys 16kk .. 16kk+15 wrote their dS_hi into its
+                // first 16 S columns and dS_lo into the next 16, two keys per column.
 #pragma unroll
                 for (int kk = 0; kk < kSub / 16; ++kk) {
                     const uint64_t bdesc = dkmn + ((kk * 16 * 128) >> 4);
-                    umma_bf16(tmem + 256, dds + ((kk * 32) >> 4), bdesc, idesc_dq,
-                              (bj > 0 || kk > 0) ? 1u : 0u);
-                    umma_bf16(tmem + 256, dds + ((kAtom128 + kk * 32) >> 4), bdesc, idesc_dq, 1u);
+                    const uint32_t hcol = tmem + dq_sbuf_col(sbuf) + 32 * (kk >> 1) + 8 * (kk & 1);
+                    umma_bf16_ts(tmem + 256, hcol, bdesc, idesc_dq, (bj > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16_ts(tmem + 256, hcol + 16, bdesc, idesc_dq, 1u);
                 }
-                umma_commit(ds_empty);
+                umma_commit(&ds_free[sbuf]);
                 umma_commit(&empty[st]);
             }
             if (ok) umma_commit(acc_full);
@@ -293,9 +284,11 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tmem_wait_ld();
             reg_fence<32>(s);
             reg_fence<32>(dp);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[sbuf]);
+            if (j < njobs) {   // phase A: the pair is free again (phase B overwrites S with dS)
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[sbuf]);
+            }
             const int nv = key_end - jobs[j < njobs ? j : j - njobs] - half * 32;
             if (!__all_sync(0xffffffffu, nv >= 32)) {   // diagonal or ragged sub-block
 #pragma unroll
@@ -334,13 +327,13 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     whi[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
                     wlo[c >> 1] = pack_bf16(lo.x, lo.y);
                 }
-                const int bj = j - njobs;
-                if (!(ok = mbar_wait(ds_empty, (bj & 1) ^ 1, ab, 27))) break;
-                store_half_row_sw128(smem + L::kDS, row, half, whi);
-                store_half_row_sw128(smem + L::kDS + kAtom128, row, half, wlo);
-                fence_proxy_async_smem();
+                // dS over this thread's own S columns: hi in the first 16, lo in the next 16
+                tmem_st16(lane_base + dq_sbuf_col(sbuf), whi);
+                tmem_st16(lane_base + dq_sbuf_col(sbuf) + 16, wlo);
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(ds_full);
+                if (lane == 0) mbar_arrive(&ds_full[sbuf]);
             }
         }
         if (njobs == 0 && row_valid && half == 0) a.delta[(size_t)bh * N + i] = 0.f;
@@ -383,11 +376,9 @@ struct DkvLayout {
     static constexpr int kV = kK + kTile;
     static constexpr int kStage0 = kV + kTile;
     static constexpr int kStageBytes = 2 * kSubT;       // Q_sub, dO_sub
-    static constexpr int kPT = kStage0 + kNst * kStageBytes;   // P^T [128 keys x 64] bf16: one atom
-    static constexpr int kDST = kPT + kAtom128;                 // dS^T
-    static constexpr int kTauDelta = kDST + kAtom128;           // [2][2][64] floats
+    static constexpr int kTauDelta = kStage0 + kNst * kStageBytes;   // [2][2][64] floats
     static constexpr int kBars = kTauDelta + 4 * 64 * 4;
-    static constexpr int kMisc = kBars + 8 * 16;
+    static constexpr int kMisc = kBars + 8 * 24;   // up to 24 mbarriers
     static constexpr int kList = kMisc + 16;
     static size_t bytes(int T) { return (size_t)kList + 8 * (size_t)T + 1024; }
 };
@@ -403,11 +394,10 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
     uint64_t* full = bars;                     // [kNst]
     uint64_t* empty = full + kNst;             // [kNst]
-    uint64_t* s_full = empty + kNst;           // [2]
-    uint64_t* s_empty = s_full + 2;            // [2]
-    uint64_t* p_full = s_empty + 2;
-    uint64_t* p_empty = p_full + 1;
-    uint64_t* acc_full = p_empty + 1;
+    uint64_t* s_full = empty + kNst;           // [2]  MMA -> elementwise
+    uint64_t* s_free = s_full + 2;             // [2]  MMA -> MMA (dV, dK of the pair's job done)
+    uint64_t* p_full = s_free + 2;             // [2]  elementwise -> MMA (P^T, dS^T in TMEM)
+    uint64_t* acc_full = p_full + 2;
     uint64_t* in_full = acc_full + 1;
     uint64_t* mma_done = in_full + 1;
     Misc* misc = reinterpret_cast<Misc*>(smem + L::kMisc);
@@ -422,9 +412,11 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kNst; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], kEwWarps); }
-        mbar_init(p_full, kEwWarps);
-        mbar_init(p_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_free[s], 1);
+            mbar_init(&p_full[s], kEwWarps);
+        }
         mbar_init(acc_full, 1);
         mbar_init(in_full, 1);
         mbar_init(mma_done, 1);
@@ -482,8 +474,6 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             constexpr uint32_t idesc_acc = idesc_bf16(128, D, 0, 1);    // dV, dK: B (dO, Q) MN-major
             const uint64_t dkk = sdesc_sw128(smem_u32(smem + L::kK), 16, 1024);
             const uint64_t dvv = sdesc_sw128(smem_u32(smem + L::kV), 16, 1024);
-            const uint64_t dpt = sdesc_sw128(smem_u32(smem + L::kPT), 16, 1024);
-            const uint64_t ddst = sdesc_sw128(smem_u32(smem + L::kDST), 16, 1024);
             const uint64_t dst = sdesc_sw128(smem_u32(smem + L::kStage0), 16, 1024);
             const uint64_t dst_mn = sdesc_sw128(smem_u32(smem + L::kStage0), kAtom64, 1024);
             bool ok = mbar_wait(in_full, 0, ab, 32);
@@ -491,7 +481,8 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             auto issue_sdp = [&](int j) -> bool {
                 const int st = j % kNst, sbuf = j & 1;
                 if (!mbar_wait(&full[st], (j / kNst) & 1, ab, 33)) return false;
-                if (!mbar_wait(&s_empty[sbuf], ((j >> 1) & 1) ^ 1, ab, 34)) return false;
+                // the pair holds P^T, dS^T of job j-2 until its dV, dK MMAs are done
+                if (!mbar_wait(&s_free[sbuf], ((j >> 1) & 1) ^ 1, ab, 34)) return false;
                 tc_fence_after();
                 const uint64_t dqs = dst + ((st * L::kStageBytes) >> 4);
                 const uint64_t dos = dqs + (L::kSubT >> 4);
@@ -508,7 +499,8 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             if (ok && njobs > 0) ok = issue_sdp(0);
             for (int j = 0; j < njobs && ok; ++j) {
                 if (j + 1 < njobs && !(ok = issue_sdp(j + 1))) break;
-                if (!(ok = mbar_wait(p_full, j & 1, ab, 35))) break;
+                const int sbuf = j & 1;
+                if (!(ok = mbar_wait(&p_full[sbuf], (j >> 1) & 1, ab, 35))) break;
                 tc_fence_after();
                 const int st = j % kNst;
                 const uint64_t qmn = dst_mn + ((st * L::kStageBytes) >> 4);
@@ -517,10 +509,13 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 for (int kk = 0; kk < kSub / 16; ++kk) {
                     const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
                     const uint32_t ok_ = (kk * 16 * 128) >> 4;
-                    umma_bf16(tm_dv, dpt + ((kk * 32) >> 4), domn + ok_, idesc_acc, acc);
-                    umma_bf16(tm_dk, ddst + ((kk * 32) >> 4), qmn + ok_, idesc_acc, acc);
+                    // queries 16kk .. 16kk+15 belong to half (kk >> 1), which wrote their P^T
+                    // (dS^T) into its first 16 S^T (dP^T) columns, two queries per column
+                    const uint32_t pcol = tmem + sbuf * 128 + 32 * (kk >> 1) + 8 * (kk & 1);
+                    umma_bf16_ts(tm_dv, pcol, domn + ok_, idesc_acc, acc);
+                    umma_bf16_ts(tm_dk, pcol + 64, qmn + ok_, idesc_acc, acc);
                 }
-                umma_commit(p_empty);
+                umma_commit(&s_free[sbuf]);
                 umma_commit(&empty[st]);
             }
             if (ok) umma_commit(acc_full);
@@ -538,13 +533,21 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + half * 32;
         const float gamma = a.gamma, cx = a.cx;
         bool ok = true;
+        // -tau, -delta of the sub-tile's 64 query rows, loaded one job ahead
+        float ntau_n = 0.f, ndel_n = 0.f;
+        auto load_td = [&](int jj) {
+            const int ii = jobs[jj] + ew;
+            ntau_n = ii < N ? -a.tau[(size_t)bh * N + ii] : 0.f;
+            ndel_n = ii < N ? -a.delta[(size_t)bh * N + ii] : 0.f;
+        };
+        if (ew < 64 && njobs > 0) load_td(0);
         for (int j = 0; j < njobs && ok; ++j) {
             const int i0 = jobs[j];
             float* tdb = td + (j & 1) * 128;
             if (ew < 64) {
-                const int ii = i0 + ew;
-                tdb[ew] = ii < N ? -a.tau[(size_t)bh * N + ii] : 0.f;         // -tau
-                tdb[64 + ew] = ii < N ? -a.delta[(size_t)bh * N + ii] : 0.f;  // -delta
+                tdb[ew] = ntau_n;
+                tdb[64 + ew] = ndel_n;
+                if (j + 1 < njobs) load_td(j + 1);
             }
             named_bar(1, kEw);
             const int sbuf = j & 1;
@@ -556,9 +559,6 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             tmem_wait_ld();
             reg_fence<32>(s);
             reg_fence<32>(dp);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[sbuf]);
             // column c is query i0 + 32*half + c: admissible iff i < N, key valid, key <= i if causal
             const int ib = i0 + half * 32;
             const int cmin = a.causal ? jkey - ib : 0;       // c >= cmin
@@ -588,12 +588,13 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 wd[c >> 1] = pack_bf16(d0.x, d0.y);
                 wd[(c >> 1) + 1] = pack_bf16(d1.x, d1.y);
             }
-            if (!(ok = mbar_wait(p_empty, (j & 1) ^ 1, ab, 37))) break;
-            store_half_row_sw128(smem + L::kPT, krow, half, wp);
-            store_half_row_sw128(smem + L::kDST, krow, half, wd);
-            fence_proxy_async_smem();
+            // P^T over this thread's own S^T columns, dS^T over its own dP^T columns
+            tmem_st16(lane_base + sbuf * 128, wp);
+            tmem_st16(lane_base + sbuf * 128 + 64, wd);
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(&p_full[sbuf]);
         }
         constexpr int DH = D / 2;
         float acc[DH];

@@ -9,17 +9,17 @@
 // Only the 128 x 128 blocks marked live by the forward's block mask are visited.
 //
 // Two kernels, both with warp roles (warp 0 TMA, warp 1 MMA issuer, warps 2-9
-// elementwise, two threads per TMEM lane) and 64-wide sub-tiles so that three
-// stages and several TMEM accumulator pairs fit on chip.  The bf16 operand the
-// elementwise warps produce (dS, P^T, dS^T) is written into TMEM over the S
-// columns it came from, and the MMA reads it from there as its A operand:
-//   dq kernel   one CTA per 128-row query tile, K/V in 64-key sub-blocks of
-//               the live blocks.  Phase A: S = Q K^T, dP = dO V^T -> delta per
-//               row (also written to the workspace).  Phase B: again S and dP,
-//               dS as a pair of bf16 parts (hi + lo) and dQ += dS K (K read
-//               MN-major).
+// elementwise, two threads per TMEM lane).  The bf16 operand the elementwise
+// warps produce (dS, P^T, dS^T) is written into TMEM and the MMA reads it from
+// there as its A operand:
+//   dq kernel   one CTA per 128-row query tile, one live 128-key block per job.
+//               Phase A: S = Q K^T, dP = dO V^T -> delta per row (also written
+//               to the workspace).  Phase B: again S and dP, dS as a pair of
+//               bf16 parts (hi + lo) and dQ += dS K (K read MN-major).
 //   dkv kernel  one CTA per 128-key block, Q/dO in 64-row sub-tiles of the
-//               live query tiles.  S^T = K Q^T, dP^T = V dO^T, then P^T and
+//               live query tiles (so that two S^T/dP^T pairs fit in TMEM
+//               beside dV and dK), P^T and dS^T over their own S^T and dP^T
+//               columns.  S^T = K Q^T, dP^T = V dO^T, then P^T and
 //               dS^T (bf16) and dV += P^T dO, dK += dS^T Q (dO and Q read
 //               MN-major from the same tiles that fed S^T and dP^T).
 // All waits are bounded as in the forward.
@@ -43,9 +43,6 @@ constexpr int kTmemCols = 512;
 constexpr int kSub = 64;                       // sub-tile width (keys or query rows)
 constexpr int kAtom128 = 128 * 128;            // [128 rows x 64 bf16] atom
 constexpr int kAtom64 = 64 * 128;              // [64 rows x 64 bf16] atom
-constexpr int kSbufDq = 3;                     // S/dP accumulator pairs of the dq kernel
-// TMEM column of S/dP pair `sb` in the dq kernel (dQ lives at columns 256..383)
-__host__ __device__ constexpr uint32_t dq_sbuf_col(int sb) { return sb < 2 ? sb * 128 : 384; }
 
 struct Misc {
     uint32_t tmem_base;
@@ -82,75 +79,74 @@ __device__ __forceinline__ void store_out_row(void* out, size_t off, const float
 }  // namespace
 
 // =========================================================================
-// dq kernel: delta and dQ for one 128-row query tile.
+// dq kernel: delta and dQ for one 128-row query tile, one 128-key live block
+// per job (128-wide MMAs run at the tensor rate; 64-wide ones do not).
+// TMEM: phase A keeps two S/dP pairs (S at 256p, dP at 256p + 128); phase B
+// one pair at 0, dQ at 256 and dS (bf16 hi at 384, lo at 448, two keys per
+// column).  K blocks stay three jobs in shared memory (S, then dQ reads them
+// MN-major one job later); V blocks feed dP only.
 // =========================================================================
 template <int D>
 struct DqLayout {
-    static constexpr int kTile = D / 64 * kAtom128;     // Q or dO [128 x D]
-    static constexpr int kSubT = D / 64 * kAtom64;      // K or V sub-block [64 x D]
+    static constexpr int kTile = D / 64 * kAtom128;     // [128 x D] bf16: Q, dO, a K or a V block
+    static constexpr int kKSlots = 3;
+    static constexpr int kVSlots = (D == 64) ? 2 : 1;
     static constexpr int kQ = 0;
     static constexpr int kDO = kQ + kTile;
-    static constexpr int kStage0 = kDO + kTile;
-    static constexpr int kStageBytes = 2 * kSubT;       // K_sub, V_sub
-    static constexpr int kXch = kStage0 + kNst * kStageBytes;  // [2][2][128] f32
+    static constexpr int kK0 = kDO + kTile;
+    static constexpr int kV0 = kK0 + kKSlots * kTile;
+    static constexpr int kXch = kV0 + kVSlots * kTile;  // [2][2][128] f32
     static constexpr int kBars = kXch + 2 * 2 * 128 * 4;
-    static constexpr int kMisc = kBars + 8 * 24;   // up to 24 mbarriers
-    static constexpr int kList = kMisc + 16;            // int job list [2*T]
-    static size_t bytes(int T) { return (size_t)kList + 8 * (size_t)T + 1024; }
+    static constexpr int kMisc = kBars + 8 * 24;        // up to 24 mbarriers
+    static constexpr int kList = kMisc + 16;            // live key blocks, uint16 [T]
+    static size_t bytes(int T) { return (size_t)kList + 2 * (size_t)T + 16 + 1024; }
 };
 
 template <int D, int GM>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                 const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v64,
+                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const BwdArgs a) {
     using L = DqLayout<D>;
+    constexpr int KS = L::kKSlots, VS = L::kVSlots;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-    uint64_t* full = bars;                     // [kNst]
-    uint64_t* empty = full + kNst;             // [kNst]
-    uint64_t* s_full = empty + kNst;           // [kSbufDq]  MMA -> elementwise
-    uint64_t* s_empty = s_full + kSbufDq;      // [kSbufDq]  elementwise -> MMA (phase A jobs)
-    uint64_t* ds_full = s_empty + kSbufDq;     // [kSbufDq]  elementwise -> MMA (dS in TMEM)
-    uint64_t* ds_free = ds_full + kSbufDq;     // [kSbufDq]  MMA -> MMA (dQ of a phase B job done)
-    uint64_t* acc_full = ds_free + kSbufDq;
+    uint64_t* kfull = bars;                    // [KS]  TMA -> MMA
+    uint64_t* kempty = kfull + KS;             // [KS]  MMA -> TMA (after S in phase A, after dQ in B)
+    uint64_t* vfull = kempty + KS;             // [VS]
+    uint64_t* vempty = vfull + VS;             // [VS]  MMA -> TMA (after dP)
+    uint64_t* s_full = vempty + VS;            // [2]   MMA -> elementwise (S and dP of a pair)
+    uint64_t* s_empty = s_full + 2;            // [2]   elementwise -> MMA (pair read)
+    uint64_t* ds_full = s_empty + 2;           //       elementwise -> MMA (dS in TMEM)
+    uint64_t* ds_free = ds_full + 1;           //       MMA -> elementwise (dQ read dS)
+    uint64_t* acc_full = ds_free + 1;
     uint64_t* in_full = acc_full + 1;          // Q and dO tiles
     uint64_t* mma_done = in_full + 1;
     Misc* misc = reinterpret_cast<Misc*>(smem + L::kMisc);
-    int* jobs = reinterpret_cast<int*>(smem + L::kList);   // key offsets of the 64-key sub-blocks
+    uint16_t* list = reinterpret_cast<uint16_t*>(smem + L::kList);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, N = a.N;
     const int t = a.causal ? (T - 1 - (int)blockIdx.x) : (int)blockIdx.x;
     const int bh = blockIdx.y;
     const int nblk = a.causal ? t + 1 : T;
-    const int last_row = min(t * kBlk + kBlk - 1, N - 1);
     const Abort ab{&misc->abort, a.hdr};
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kNst; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int s = 0; s < kSbufDq; ++s) {
-            mbar_init(&s_full[s], 1);
-            mbar_init(&s_empty[s], kEwWarps);
-            mbar_init(&ds_full[s], kEwWarps);
-            mbar_init(&ds_free[s], 1);
-        }
+        for (int i = 0; i < KS; ++i) { mbar_init(&kfull[i], 1); mbar_init(&kempty[i], 1); }
+        for (int i = 0; i < VS; ++i) { mbar_init(&vfull[i], 1); mbar_init(&vempty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], kEwWarps); }
+        mbar_init(ds_full, kEwWarps);
+        mbar_init(ds_free, 1);
         mbar_init(acc_full, 1);
         mbar_init(in_full, 1);
         mbar_init(mma_done, 1);
         misc->abort = 0;
-        // sub-block list of the live key blocks of this tile
         const uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
         int n = 0;
-        for (int b = 0; b < nblk; ++b) {
-            if (!mrow[b]) continue;
-            for (int h = 0; h < 2; ++h) {
-                const int j0 = b * kBlk + h * kSub;
-                if (j0 >= N || (a.causal && j0 > last_row)) continue;
-                jobs[n++] = j0;
-            }
-        }
+        for (int b = 0; b < nblk; ++b)
+            if (mrow[b]) list[n++] = (uint16_t)b;
         misc->njobs = n;
         fence_barrier_init();
     }
@@ -162,104 +158,108 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
-    const int njobs = misc->njobs;
-    const int total = 2 * njobs;     // phase A then phase B
+    const int nA = misc->njobs;      // phase A jobs 0..nA-1, phase B jobs nA..2nA-1, same blocks
+    const int total = 2 * nA;
+    // pair of job j and the number of earlier jobs on that pair
+    auto pair_of = [&](int j) { return j < nA ? (j & 1) : 0; };
+    auto use_of = [&](int j) { return j < nA ? (j >> 1) : ((nA + 1) >> 1) + (j - nA); };
 
     if (warp == 0) {
         if (lane == 0) {
-            prefetch_tmap(&tm_q); prefetch_tmap(&tm_do); prefetch_tmap(&tm_k64); prefetch_tmap(&tm_v64);
+            prefetch_tmap(&tm_q); prefetch_tmap(&tm_do); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
             mbar_arrive_expect_tx(in_full, 2 * L::kTile);
             for (int at = 0; at < D / 64; ++at) {
                 tma_load_3d(smem + L::kQ + at * kAtom128, &tm_q, at * 64, t * kBlk, bh, in_full);
                 tma_load_3d(smem + L::kDO + at * kAtom128, &tm_do, at * 64, t * kBlk, bh, in_full);
             }
-            int job = 0;
+            int nk = 0, nv = 0;   // K and V blocks issued
             bool ok = true;
-            for (; job < total && ok; ++job) {
-                const int j0 = jobs[job % njobs];
-                const int st = job % kNst;
-                if (!(ok = mbar_wait(&empty[st], ((job / kNst) & 1) ^ 1, ab, 21))) break;
-                uint8_t* sb = smem + L::kStage0 + st * L::kStageBytes;
-                mbar_arrive_expect_tx(&full[st], 2 * L::kSubT);
-                for (int at = 0; at < D / 64; ++at) {
-                    tma_load_3d(sb + at * kAtom64, &tm_k64, at * 64, j0, bh, &full[st]);
-                    tma_load_3d(sb + L::kSubT + at * kAtom64, &tm_v64, at * 64, j0, bh, &full[st]);
-                }
+            for (int j = 0; j < total && ok; ++j) {
+                const int b = list[j < nA ? j : j - nA];
+                const int ks = j % KS, vs = j % VS;
+                if (!(ok = mbar_wait(&kempty[ks], ((j / KS) & 1) ^ 1, ab, 21))) break;
+                mbar_arrive_expect_tx(&kfull[ks], L::kTile);
+                for (int at = 0; at < D / 64; ++at)
+                    tma_load_3d(smem + L::kK0 + ks * L::kTile + at * kAtom128, &tm_k, at * 64, b * kBlk, bh,
+                                &kfull[ks]);
+                ++nk;
+                if (!(ok = mbar_wait(&vempty[vs], ((j / VS) & 1) ^ 1, ab, 21))) break;
+                mbar_arrive_expect_tx(&vfull[vs], L::kTile);
+                for (int at = 0; at < D / 64; ++at)
+                    tma_load_3d(smem + L::kV0 + vs * L::kTile + at * kAtom128, &tm_v, at * 64, b * kBlk, bh,
+                                &vfull[vs]);
+                ++nv;
             }
             drain_wait(in_full, 0);
-            for (int j = job - 1; j >= 0 && j >= job - kNst; --j) drain_wait(&full[j % kNst], (j / kNst) & 1);
+            for (int j = nk - 1; j >= 0 && j >= nk - KS; --j) drain_wait(&kfull[j % KS], (j / KS) & 1);
+            for (int j = nv - 1; j >= 0 && j >= nv - VS; --j) drain_wait(&vfull[j % VS], (j / VS) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16(128, kSub, 0, 0);   // [128 x 64], K = d
-            constexpr uint32_t idesc_dq = idesc_bf16(128, D, 0, 1);     // dQ += dS K, K MN-major
-            // base descriptors; operands differ only by start-address offsets
+            constexpr uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);   // [128 x 128], K = d
+            constexpr uint32_t idesc_dq = idesc_bf16(128, D, 0, 1);    // dQ += dS K, K MN-major
             const uint64_t dq_ = sdesc_sw128(smem_u32(smem + L::kQ), 16, 1024);
             const uint64_t ddo = sdesc_sw128(smem_u32(smem + L::kDO), 16, 1024);
-            const uint64_t dst = sdesc_sw128(smem_u32(smem + L::kStage0), 16, 1024);
-            const uint64_t dst_mn = sdesc_sw128(smem_u32(smem + L::kStage0), kAtom64, 1024);
+            const uint64_t dk = sdesc_sw128(smem_u32(smem + L::kK0), 16, 1024);
+            const uint64_t dkmn = sdesc_sw128(smem_u32(smem + L::kK0), kAtom128, 1024);
+            const uint64_t dv = sdesc_sw128(smem_u32(smem + L::kV0), 16, 1024);
             bool ok = mbar_wait(in_full, 0, ab, 22);
             tc_fence_after();
-            // issue S and dP of job j into TMEM pair j % kSbufDq.  The pair is free once
-            // the previous job on it is done with it: a phase A job when the elementwise
-            // warps have read S and dP, a phase B job when the dQ MMA has read its dS.
-            auto issue_sdp = [&](int j) -> bool {
-                const int st = j % kNst, sbuf = j % kSbufDq;
-                if (!mbar_wait(&full[st], (j / kNst) & 1, ab, 23)) return false;
-                const int jp = j - kSbufDq;
-                const bool fr = (jp < njobs)
-                                    ? mbar_wait(&s_empty[sbuf], ((j / kSbufDq) & 1) ^ 1, ab, 24)
-                                    : mbar_wait(&ds_free[sbuf], ((jp - njobs) / kSbufDq) & 1, ab, 24);
-                if (!fr) return false;
-                tc_fence_after();
-                const uint64_t dk = dst + ((st * L::kStageBytes) >> 4);
-                const uint64_t dv = dk + (L::kSubT >> 4);
-                const uint32_t dS = tmem + dq_sbuf_col(sbuf), dPc = dS + 64;
+            auto issue_128 = [&](uint32_t dcol, uint64_t da, uint64_t db) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t oa = ((kk >> 2) * kAtom128 + (kk & 3) * 32) >> 4;
-                    const uint32_t ob = ((kk >> 2) * kAtom64 + (kk & 3) * 32) >> 4;
-                    umma_bf16(dS, dq_ + oa, dk + ob, idesc_s, kk > 0);
-                    umma_bf16(dPc, ddo + oa, dv + ob, idesc_s, kk > 0);
+                    const uint32_t off = ((kk >> 2) * kAtom128 + (kk & 3) * 32) >> 4;
+                    umma_bf16(tmem + dcol, da + off, db + off, idesc_s, kk > 0);
                 }
-                umma_commit(&s_full[sbuf]);
+            };
+            // S and dP of job j into its pair; phase A releases the K block after S,
+            // phase B keeps it for dQ
+            auto issue_sdp = [&](int j) -> bool {
+                const int p = pair_of(j), ks = j % KS, vs = j % VS;
+                if (!mbar_wait(&s_empty[p], (use_of(j) & 1) ^ 1, ab, 24)) return false;
+                if (!mbar_wait(&kfull[ks], (j / KS) & 1, ab, 23)) return false;
+                tc_fence_after();
+                issue_128(p * 256, dq_, dk + ((uint32_t)(ks * L::kTile) >> 4));
+                if (j < nA) umma_commit(&kempty[ks]);
+                if (!mbar_wait(&vfull[vs], (j / VS) & 1, ab, 23)) return false;
+                tc_fence_after();
+                issue_128(p * 256 + 128, ddo, dv + ((uint32_t)(vs * L::kTile) >> 4));
+                umma_commit(&vempty[vs]);
+                umma_commit(&s_full[p]);
                 return true;
             };
-            if (ok && total > 0) ok = issue_sdp(0);
-            for (int j = 0; j < total && ok; ++j) {
-                if (j + 1 < total && !(ok = issue_sdp(j + 1))) break;
-                const int st = j % kNst;
-                if (j < njobs) {                 // phase A: K/V stage only fed S and dP
-                    umma_commit(&empty[st]);
-                    continue;
-                }
-                const int bj = j - njobs;        // phase B job: dQ += dS K
-                const int sbuf = j % kSbufDq;
-                // one ds_full per pair: dS(j+3) cannot complete before dQ(j) frees the pair
-                if (!(ok = mbar_wait(&ds_full[sbuf], (bj / kSbufDq) & 1, ab, 25))) break;
+            // dQ += (dS_hi + dS_lo) K for phase B job i: the two bf16 parts carry dS to
+            // ~16 bits, which the cancellation in sum_j dS_ij k_j (rows of dS sum to 0) needs
+            auto issue_dq = [&](int i) -> bool {
+                const int ks = (nA + i) % KS;
+                if (!mbar_wait(ds_full, i & 1, ab, 25)) return false;
                 tc_fence_after();
-                const uint64_t dkmn = dst_mn + ((st * L::kStageBytes) >> 4);
-                // dQ += (dS_hi + dS_lo) K: the two bf16 parts carry dS to ~16 bits, which
-                // the cancellation in sum_j dS_ij k_j (rows of dS sum to 0) needs.  The
-                // half (kk >> 1) that owns keys 16kk .. 16kk+15 wrote their dS_hi into its
-                // first 16 S columns and dS_lo into the next 16, two keys per column.
+                const uint64_t bk = dkmn + ((uint32_t)(ks * L::kTile) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kSub / 16; ++kk) {
-                    const uint64_t bdesc = dkmn + ((kk * 16 * 128) >> 4);
-                    const uint32_t hcol = tmem + dq_sbuf_col(sbuf) + 32 * (kk >> 1) + 8 * (kk & 1);
-                    umma_bf16_ts(tmem + 256, hcol, bdesc, idesc_dq, (bj > 0 || kk > 0) ? 1u : 0u);
-                    umma_bf16_ts(tmem + 256, hcol + 16, bdesc, idesc_dq, 1u);
+                for (int kk = 0; kk < kBlk / 16; ++kk) {
+                    const uint64_t bdesc = bk + ((kk * 16 * 128) >> 4);
+                    umma_bf16_ts(tmem + 256, tmem + 384 + kk * 8, bdesc, idesc_dq, (i > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16_ts(tmem + 256, tmem + 448 + kk * 8, bdesc, idesc_dq, 1u);
                 }
-                umma_commit(&ds_free[sbuf]);
-                umma_commit(&empty[st]);
+                umma_commit(ds_free);
+                umma_commit(&kempty[ks]);
+                return true;
+            };
+            for (int j = 0; j < nA && ok; ++j) ok = issue_sdp(j);
+            // phase B: S and dP of job i go in ahead of dQ of job i-1, so the tensor
+            // pipe has work while the elementwise warps turn job i-1 into dS
+            for (int i = 0; i < nA && ok; ++i) {
+                ok = issue_sdp(nA + i);
+                if (ok && i > 0) ok = issue_dq(i - 1);
             }
+            if (ok && nA > 0) ok = issue_dq(nA - 1);
             if (ok) umma_commit(acc_full);
             umma_commit(mma_done);
             drain_wait(mma_done, 0);
         }
     } else {
-        // two threads per query row: `half` takes columns [32*half, 32*half + 32)
-        // of each 64-key sub-block; delta's partial sums meet in shared memory
+        // two threads per query row: `half` takes keys [64*half, 64*half + 64) of each
+        // block, in two rounds of 32; delta's partial sums meet in shared memory
         const int ew = threadIdx.x - 64;
         const int half = ew >> 7;
         const int quarter = warp & 3;
@@ -267,35 +267,43 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int i = t * kBlk + row;
         const bool row_valid = i < N;
         const int key_end = !row_valid ? 0 : (a.causal ? i + 1 : N);
-        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + half * 32;
+        const uint32_t lane0 = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t lane_base = lane0 + half * 64;
         const float gamma = a.gamma, cx = a.cx;
         const float tau = row_valid ? a.tau[(size_t)bh * N + i] : 0.f;
         float* xch = reinterpret_cast<float*>(smem + L::kXch);   // [2][2][128]
-        float sg = 0.f, sgdp = 0.f, delta = 0.f;
         const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-tau, -tau);
         bool ok = true;
-        for (int j = 0; j < total && ok; ++j) {
-            const int sbuf = j % kSbufDq;
-            if (!(ok = mbar_wait(&s_full[sbuf], (j / kSbufDq) & 1, ab, 26))) break;
-            tc_fence_after();
-            float s[32], dp[32];
-            tmem_ld32(lane_base + dq_sbuf_col(sbuf), &s[0]);
-            tmem_ld32(lane_base + dq_sbuf_col(sbuf) + 64, &dp[0]);
+        // S and dP of job j, columns [32r, 32r + 32) of this thread's 64 keys; the pair is
+        // released after the second round
+        auto load_round = [&](int j, int r, float* s, float* dp) -> void {
+            const int p = pair_of(j);
+            tmem_ld32(lane_base + p * 256 + r * 32, s);
+            tmem_ld32(lane_base + p * 256 + 128 + r * 32, dp);
             tmem_wait_ld();
             reg_fence<32>(s);
             reg_fence<32>(dp);
-            if (j < njobs) {   // phase A: the pair is free again (phase B overwrites S with dS)
+            if (r == 1) {
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[sbuf]);
+                if (lane == 0) mbar_arrive(&s_empty[p]);
             }
-            const int nv = key_end - jobs[j < njobs ? j : j - njobs] - half * 32;
-            if (!__all_sync(0xffffffffu, nv >= 32)) {   // diagonal or ragged sub-block
+            const int nv = key_end - list[j < nA ? j : j - nA] * kBlk - half * 64 - r * 32;
+            if (!__all_sync(0xffffffffu, nv >= 32)) {   // diagonal or ragged block
 #pragma unroll
                 for (int c = 0; c < 32; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
             }
-            if (j < njobs) {
-                float2 a0 = make_float2(0.f, 0.f), b0 = a0, a1 = a0, b1 = a0;
+        };
+        // phase A: sum_j g and sum_j g dP
+        float sg = 0.f, sgdp = 0.f;
+        for (int j = 0; j < nA && ok; ++j) {
+            if (!(ok = mbar_wait(&s_full[pair_of(j)], use_of(j) & 1, ab, 26))) break;
+            tc_fence_after();
+            float2 a0 = make_float2(0.f, 0.f), b0 = a0, a1 = a0, b1 = a0;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                float s[32], dp[32];
+                load_round(j, r, s, dp);
 #pragma unroll
                 for (int c = 0; c < 32; c += 4) {
                     const float2 g0 = entmax_g_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma);
@@ -303,46 +311,55 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     a0 = __fadd2_rn(a0, g0); b0 = __ffma2_rn(g0, make_float2(dp[c], dp[c + 1]), b0);
                     a1 = __fadd2_rn(a1, g1); b1 = __ffma2_rn(g1, make_float2(dp[c + 2], dp[c + 3]), b1);
                 }
-                a0 = __fadd2_rn(a0, a1); b0 = __fadd2_rn(b0, b1);
-                sg += a0.x + a0.y;
-                sgdp += b0.x + b0.y;
-                if (j == njobs - 1) {
-                    xch[(0 * 2 + half) * 128 + row] = sg;
-                    xch[(1 * 2 + half) * 128 + row] = sgdp;
-                    named_bar(1, kEw);
-                    const float SG = sg + xch[(0 * 2 + (half ^ 1)) * 128 + row];
-                    const float SGDP = sgdp + xch[(1 * 2 + (half ^ 1)) * 128 + row];
-                    delta = (SG > 0.f) ? SGDP / SG : 0.f;
-                    if (row_valid && half == 0) a.delta[(size_t)bh * N + i] = delta;
-                }
-            } else {
-                uint32_t whi[16], wlo[16];
-                const float2 nd2 = make_float2(-delta, -delta), m1 = make_float2(-1.f, -1.f);
+            }
+            a0 = __fadd2_rn(a0, a1); b0 = __fadd2_rn(b0, b1);
+            sg += a0.x + a0.y;
+            sgdp += b0.x + b0.y;
+        }
+        // every elementwise thread reaches this barrier once, also after an abort
+        xch[(0 * 2 + half) * 128 + row] = sg;
+        xch[(1 * 2 + half) * 128 + row] = sgdp;
+        named_bar(1, kEw);
+        const float SG = sg + xch[(0 * 2 + (half ^ 1)) * 128 + row];
+        const float SGDP = sgdp + xch[(1 * 2 + (half ^ 1)) * 128 + row];
+        const float delta = (SG > 0.f) ? SGDP / SG : 0.f;
+        if (row_valid && half == 0) a.delta[(size_t)bh * N + i] = delta;
+        // phase B: dS = g (dP - delta) as bf16 hi + lo into TMEM
+        const float2 nd2 = make_float2(-delta, -delta), m1 = make_float2(-1.f, -1.f);
+        for (int ib = 0; ib < nA && ok; ++ib) {
+            const int j = nA + ib;
+            if (!(ok = mbar_wait(&s_full[0], use_of(j) & 1, ab, 26))) break;
+            tc_fence_after();
+            uint32_t whi[32], wlo[32];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                float s[32], dp[32];
+                load_round(j, r, s, dp);
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const float2 g = entmax_g_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma);
                     const float2 d = __fmul2_rn(g, __fadd2_rn(make_float2(dp[c], dp[c + 1]), nd2));
                     const __nv_bfloat162 h = __floats2bfloat162_rn(d.x, d.y);
                     const float2 lo = __ffma2_rn(__bfloat1622float2(h), m1, d);   // d - bf16(d), exact
-                    whi[c >> 1] = *reinterpret_cast<const uint32_t*>(&h);
-                    wlo[c >> 1] = pack_bf16(lo.x, lo.y);
+                    whi[r * 16 + (c >> 1)] = *reinterpret_cast<const uint32_t*>(&h);
+                    wlo[r * 16 + (c >> 1)] = pack_bf16(lo.x, lo.y);
                 }
-                // dS over this thread's own S columns: hi in the first 16, lo in the next 16
-                tmem_st16(lane_base + dq_sbuf_col(sbuf), whi);
-                tmem_st16(lane_base + dq_sbuf_col(sbuf) + 16, wlo);
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ds_full[sbuf]);
             }
+            // the dS region is free once dQ of the previous job has read it
+            if (!(ok = mbar_wait(ds_free, (ib & 1) ^ 1, ab, 27))) break;
+            tmem_st32(lane0 + 384 + half * 32, whi);
+            tmem_st32(lane0 + 448 + half * 32, wlo);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ds_full);
         }
-        if (njobs == 0 && row_valid && half == 0) a.delta[(size_t)bh * N + i] = 0.f;
         constexpr int DH = D / 2;
         float acc[DH];
-        if (ok && njobs > 0) {
+        if (ok && nA > 0) {
             ok = mbar_wait(acc_full, 0, ab, 28);
             tc_fence_after();
-            const uint32_t ob = tmem + ((uint32_t)(quarter * 32) << 16) + 256 + half * DH;
+            const uint32_t ob = lane0 + 256 + half * DH;
 #pragma unroll
             for (int c = 0; c < DH / 32; ++c) tmem_ld32(ob + c * 32, &acc[c * 32]);
             tmem_wait_ld();
@@ -352,8 +369,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int c = 0; c < DH; ++c) acc[c] = 0.f;
         }
         if (row_valid) store_out_row(a.dq, ((size_t)bh * N + i) * D + half * DH, acc, DH, a.scale);
-        if (threadIdx.x == 64)   // block products: phase A S,dP (2) + phase B S,dP,dQ hi,lo (4), per 64-key half
-            atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(3 * njobs));
+        if (threadIdx.x == 64)   // block products: phase A S, dP (2) + phase B S, dP, dQ hi, lo (4)
+            atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(6 * nA));
     }
 
     tc_fence_before();
@@ -634,7 +651,7 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 // ------------------------------------------------------------------ host side
 template <int D, int GM>
 static cudaError_t launch_tc_bwd(const BwdArgs& a, cudaStream_t s, const CUtensorMap* m) {
-    // m: q128, do128, k64, v64, k128, v128, q64, do64
+    // m: q128, do128, k128, v128, q64, do64
     {
         const size_t sm = DqLayout<D>::bytes(a.T);
         auto kern = tc_bwd_dq_kernel<D, GM>;
@@ -647,7 +664,7 @@ static cudaError_t launch_tc_bwd(const BwdArgs& a, cudaStream_t s, const CUtenso
     auto kern = tc_bwd_dkv_kernel<D, GM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(m[4], m[5], m[6], m[7], a);
+    kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(m[2], m[3], m[4], m[5], a);
     return cudaGetLastError();
 }
 
@@ -662,15 +679,13 @@ static cudaError_t tc_bwd_d(const BwdArgs& a, int gm, cudaStream_t s, const CUte
 }
 
 cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char** why) {
-    CUtensorMap m[8];
+    CUtensorMap m[6];
     const bool ok = make_tmap_bf16_rows(&m[0], a.q, a.BH, a.N, d, 128) &&
                     make_tmap_bf16_rows(&m[1], a.dout, a.BH, a.N, d, 128) &&
-                    make_tmap_bf16_rows(&m[2], a.k, a.BH, a.N, d, 64) &&
-                    make_tmap_bf16_rows(&m[3], a.v, a.BH, a.N, d, 64) &&
-                    make_tmap_bf16_rows(&m[4], a.k, a.BH, a.N, d, 128) &&
-                    make_tmap_bf16_rows(&m[5], a.v, a.BH, a.N, d, 128) &&
-                    make_tmap_bf16_rows(&m[6], a.q, a.BH, a.N, d, 64) &&
-                    make_tmap_bf16_rows(&m[7], a.dout, a.BH, a.N, d, 64);
+                    make_tmap_bf16_rows(&m[2], a.k, a.BH, a.N, d, 128) &&
+                    make_tmap_bf16_rows(&m[3], a.v, a.BH, a.N, d, 128) &&
+                    make_tmap_bf16_rows(&m[4], a.q, a.BH, a.N, d, 64) &&
+                    make_tmap_bf16_rows(&m[5], a.dout, a.BH, a.N, d, 64);
     if (!ok) {
         *why = "cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;

@@ -558,7 +558,7 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             ndel_n = ii < N ? -a.delta[(size_t)bh * N + ii] : 0.f;
         };
         if (ew < 64 && njobs > 0) load_td(0);
-        for (int j = 0; j < njobs && ok; ++j) {
+        for (int j = 0; j < njobs; ++j) {
             const int i0 = jobs[j];
             float* tdb = td + (j & 1) * 128;
             if (ew < 64) {
@@ -566,9 +566,12 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 tdb[64 + ew] = ndel_n;
                 if (j + 1 < njobs) load_td(j + 1);
             }
-            named_bar(1, kEw);
+            // the group agrees on `ok` at its barrier: a wait that gave up in the previous
+            // job makes every thread leave here together
+            ok = named_bar_and(1, kEw, ok);
+            if (!ok) break;
             const int sbuf = j & 1;
-            if (!(ok = mbar_wait(&s_full[sbuf], (j >> 1) & 1, ab, 36))) break;
+            if (!(ok = mbar_wait(&s_full[sbuf], (j >> 1) & 1, ab, 36))) continue;
             tc_fence_after();
             float s[32], dp[32];
             tmem_ld32(lane_base + sbuf * 128, &s[0]);

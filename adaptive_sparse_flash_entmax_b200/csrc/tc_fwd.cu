@@ -4,11 +4,16 @@
 // Technical Deep Dive / AdaSplash: Fused GPU Kernel for Attention: the Q tile is
 // loaded once and stays on chip; K tiles stream for the tau passes; a final pass
 // streams K and V and accumulates O = P V).  Warp roles:
-//   warp 0   TMA producer: Q once, then tiles into a four-slot ring: K blocks
-//            in the score passes, K and V of each live block in the P.V pass;
-//   warp 1   MMA issuer: S = Q K^T into three TMEM accumulators (128 x 128
-//            fp32), and O += P V with P read from TMEM (it replaces S in its
-//            buffer) and V from shared memory (MN-major);
+//   warp 0   TMA producer: Q once, then K blocks two at a time into two double
+//            slots of the ring in the score passes (stacked as [256 rows x 64]
+//            atoms), or K and V of each live block into four single slots (the
+//            same memory) in the P.V pass;
+//   warp 1   MMA issuer: in the score passes S = Q [K_a; K_b]^T as one 128 x 256
+//            MMA into two 256-column TMEM buffers (a 256-wide instruction does
+//            twice the work of a 128-wide one in ~1.5x the time, and the
+//            elementwise warps' arithmetic slows every instruction); in the P.V
+//            pass S = Q K^T into three 128-column buffers and O += P V with P
+//            read from TMEM (it replaces S in its buffer), V MN-major;
 //   warps 2-9 elementwise: two threads per query row (= TMEM lane), 64 columns
 //            each.  Pass 0 builds the
 //            row max and the sliding 64-bin histogram ("AdaSplash-2: ...",
@@ -36,13 +41,15 @@ using namespace tc;
 
 namespace {
 
-constexpr int kSlots = 4;          // tile slots of the K / V ring
-constexpr int kSbuf = 3;           // S accumulators in TMEM
+constexpr int kSlots = 4;          // single tile slots of the P.V pass (K or V blocks)
+constexpr int kDSlots = 2;         // double slots of the score passes (two K blocks), same memory
+constexpr int kSbuf = 3;           // 128-column S accumulators in TMEM (P.V pass)
 constexpr int kThreads = 320;      // 10 warps
 constexpr int kEw = 256;           // elementwise threads (warps 2-9): two per query row
 constexpr int kEwWarps = 8;
 constexpr int kAtom = 128 * 128;   // bytes of a [128 rows x 64 bf16] swizzled atom
-constexpr int kTmemCols = 512;     // S0 [0,128), S1 [128,256), O [256, 256+D), S2 [384, 512)
+constexpr int kTmemCols = 512;     // score passes: S [0,256), [256,512); P.V pass: S0 [0,128),
+                                   // S1 [128,256), O [256, 256+D), S2 [384, 512)
 constexpr int kDecSolve = 1, kDecPv = 2;
 
 __host__ __device__ constexpr uint32_t sbuf_col(int sb) { return sb < 2 ? sb * 128 : 384; }
@@ -56,7 +63,7 @@ struct Layout {
     static constexpr int kPBytes = 2 * kAtom;             // histograms [64][128] u16
     static constexpr int kXch = kP + kPBytes;             // [4][2][128] f32 exchange
     static constexpr int kBars = kXch + 4 * 2 * 128 * 4;
-    static constexpr int kNumBars = 24;
+    static constexpr int kNumBars = 40;
     static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, decision, njobs, abort
     static constexpr int kPtab = kMisc + 32;              // 68 floats
     static constexpr int kLive = kPtab + 68 * 4;          // live[T], cand[T] (bytes), list[T] (int),
@@ -96,10 +103,14 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-    uint64_t* kfull = bars;                    // [kSlots]     TMA -> MMA
+    uint64_t* kfull = bars;                    // [kSlots]     TMA -> MMA (P.V pass)
     uint64_t* kempty = kfull + kSlots;         // [kSlots]     MMA -> TMA
-    uint64_t* s_full = kempty + kSlots;        // [kSbuf]      MMA -> elementwise
-    uint64_t* s_empty = s_full + kSbuf;        // [kSbuf]      elementwise -> MMA (score passes)
+    uint64_t* kfull2 = kempty + kSlots;        // [kDSlots]    TMA -> MMA (score passes)
+    uint64_t* kempty2 = kfull2 + kDSlots;      // [kDSlots]    MMA -> TMA
+    uint64_t* s_full2 = kempty2 + kDSlots;     // [2]          MMA -> elementwise (score passes)
+    uint64_t* s_empty2 = s_full2 + 2;          // [2]          elementwise -> MMA
+    uint64_t* s_full = s_empty2 + 2;           // [kSbuf]      MMA -> elementwise (P.V pass)
+    uint64_t* s_empty = s_full + kSbuf;        // [kSbuf]      (first use of a P.V buffer: fresh)
     uint64_t* pv_sfree = s_empty + kSbuf;      // [kSbuf]      MMA -> MMA (P.V pass: P(i) consumed)
     uint64_t* p_full = pv_sfree + kSbuf;       // [kSbuf]      elementwise -> MMA (P(i) in TMEM)
     uint64_t* o_full = p_full + kSbuf;         //              MMA -> elementwise
@@ -122,6 +133,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSlots; ++s) { mbar_init(&kfull[s], 1); mbar_init(&kempty[s], 1); }
+        for (int s = 0; s < kDSlots; ++s) { mbar_init(&kfull2[s], 1); mbar_init(&kempty2[s], 1); }
+        for (int s = 0; s < 2; ++s) { mbar_init(&s_full2[s], 1); mbar_init(&s_empty2[s], kEwWarps); }
         for (int s = 0; s < kSbuf; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&s_empty[s], kEwWarps);
@@ -157,9 +170,24 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_arrive_expect_tx(q_full, L::kTile);
             for (int at = 0; at < D / 64; ++at)
                 tma_load_3d(smem + L::kQ + at * kAtom, &tm_q, at * 64, t * kBlk, bh, q_full);
-            int sj = 0, kind = kDecSolve;   // tiles loaded into the ring so far
+            int sj = 0, dj = 0, kind = kDecSolve;   // P.V-pass tiles, score-pass double slots loaded
             uint32_t dec_phase = 0;
             bool ok = true, first = true;
+            // a score-pass job: K blocks b0 and b1 (b1 < 0: none) stacked in one double slot,
+            // block h at rows 128h of each [256 rows x 64] atom
+            auto load_pair = [&](int b0, int b1) -> bool {
+                const int ds = dj % kDSlots;
+                if (!mbar_wait(&kempty2[ds], ((dj / kDSlots) & 1) ^ 1, ab, 1)) return false;
+                mbar_arrive_expect_tx(&kfull2[ds], (b1 >= 0 ? 2 : 1) * L::kTile);
+                uint8_t* base = smem + L::kRing + ds * 2 * L::kTile;
+                for (int at = 0; at < D / 64; ++at) {
+                    tma_load_3d(base + at * 2 * kAtom, &tm_k, at * 64, b0 * kBlk, bh, &kfull2[ds]);
+                    if (b1 >= 0)
+                        tma_load_3d(base + at * 2 * kAtom + kAtom, &tm_k, at * 64, b1 * kBlk, bh, &kfull2[ds]);
+                }
+                ++dj;
+                return true;
+            };
             auto load_tile = [&](const CUtensorMap* map, int b) -> bool {
                 const int sl = sj % kSlots;
                 if (!mbar_wait(&kempty[sl], ((sj / kSlots) & 1) ^ 1, ab, 1)) return false;
@@ -173,10 +201,18 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             while (ok) {
                 const bool pv = kind == kDecPv;
                 const int njobs = first ? nblk : misc->njobs;
-                for (int i = 0; i < njobs && ok; ++i) {
-                    const int b = first ? i : job_list[i];
-                    ok = load_tile(&tm_k, b);
-                    if (ok && pv) ok = load_tile(&tm_v, b);
+                if (!pv) {
+                    for (int i = 0; i < njobs && ok; i += 2) {
+                        const int b0 = first ? i : job_list[i];
+                        const int b1 = (i + 1 < njobs) ? (first ? i + 1 : job_list[i + 1]) : -1;
+                        ok = load_pair(b0, b1);
+                    }
+                } else {
+                    for (int i = 0; i < njobs && ok; ++i) {
+                        const int b = job_list[i];
+                        ok = load_tile(&tm_k, b);
+                        if (ok) ok = load_tile(&tm_v, b);
+                    }
                 }
                 first = false;
                 if (!ok || pv) break;
@@ -187,11 +223,13 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // Copies issued but possibly not consumed land before the CTA ends.
             drain_wait(q_full, 0);
             for (int j = sj - 1; j >= 0 && j >= sj - kSlots; --j) drain_wait(&kfull[j % kSlots], (j / kSlots) & 1);
+            for (int j = dj - 1; j >= 0 && j >= dj - kDSlots; --j) drain_wait(&kfull2[j % kDSlots], (j / kDSlots) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t idesc_qk2 = idesc_bf16(128, 256, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16(128, D, 0, 1);
             // Descriptors differ only in the start-address field (bits 0-13, address >> 4),
             // so each operand's base descriptor is built once and offsets are added.
@@ -200,7 +238,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const uint64_t dring_mn = sdesc_sw128(smem_u32(smem + L::kRing), kAtom, 1024);
             bool ok = mbar_wait(q_full, 0, ab, 3);
             tc_fence_after();
-            int job = 0, sj = 0, kind = kDecSolve;   // S jobs issued; ring tiles consumed
+            int sjob = 0, kind = kDecSolve;   // score-pass jobs issued (= double slots consumed)
             uint32_t dec_phase = 0;
             bool first = true;
             auto wait_tile = [&](int tt) { return mbar_wait(&kfull[tt % kSlots], (tt / kSlots) & 1, ab, 4); };
@@ -220,12 +258,21 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const int njobs = first ? nblk : misc->njobs;
                 first = false;
                 if (!pv) {
-                    for (int i = 0; i < njobs && ok; ++i, ++job, ++sj) {
-                        const int sb = job % kSbuf;
-                        if (!(ok = wait_tile(sj))) break;
-                        if (!(ok = mbar_wait(&s_empty[sb], ((job / kSbuf) & 1) ^ 1, ab, 5))) break;
+                    for (int i = 0; i < njobs && ok; i += 2, ++sjob) {
+                        const int sb = sjob & 1, ds = sjob % kDSlots;
+                        if (!(ok = mbar_wait(&kfull2[ds], (sjob / kDSlots) & 1, ab, 4))) break;
+                        if (!(ok = mbar_wait(&s_empty2[sb], ((sjob >> 1) & 1) ^ 1, ab, 5))) break;
                         tc_fence_after();
-                        issue_s(sb, sj);
+                        const uint32_t idesc = (i + 1 < njobs) ? idesc_qk2 : idesc_qk;
+                        const uint64_t dk = dring + ((uint32_t)(ds * 2 * L::kTile) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oa = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
+                            const uint32_t ob = ((kk >> 2) * 2 * kAtom + (kk & 3) * 32) >> 4;
+                            umma_bf16(tmem + sb * 256, dq + oa, dk + ob, idesc, kk > 0);
+                        }
+                        umma_commit(&s_full2[sb]);
+                        umma_commit(&kempty2[ds]);
                     }
                     if (!ok) break;
                     if (!(ok = mbar_wait(dec_bar, dec_phase, ab, 7))) break;
@@ -233,12 +280,14 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     kind = misc->decision;
                     continue;
                 }
-                // P.V pass over the live blocks; ring tiles K_i = sj + 2i, V_i = sj + 2i + 1.
+                // P.V pass over the live blocks, with its own barriers and ring counters:
+                // ring tiles K_i = 2i, V_i = 2i + 1.
                 // S(i) is issued ahead of P.V(i-1), so the score MMA of the next block
                 // runs while the elementwise warps turn S(i-1) into P(i-1).  P(i)
                 // replaces S(i) in its TMEM buffer, which is free again once P.V(i)
-                // is done (pv_sfree); a buffer's first use in this pass waits for the
-                // elementwise release of its last score-pass job instead.
+                // is done (pv_sfree).  Every score-pass S buffer was read before the
+                // decision that started this pass, so TMEM is free.
+                const int job = 0, sj = 0;
                 for (int i = 0; i <= njobs && ok; ++i) {
                     if (i < njobs) {
                         const int jb = job + i, sb = jb % kSbuf;
@@ -329,7 +378,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         sv.done = row_valid ? 0 : 1;
         sv.iters = 0;
         const int wi = warp - 2;                  // elementwise warp index 0..7
-        int job = 0, pass = 0, nlive = 0;
+        int sjob = 0, pass = 0, nlive = 0;
         long long qk_blocks = nblk;
         bool ok = true;
         for (;; ++pass) {
@@ -341,93 +390,105 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 npj = misc->njobs;
                 qk_blocks += npj;
             }
-            for (int jj = 0; jj < npj; ++jj, ++job) {
-                const int b = (pass == 0) ? jj : job_list[jj];
-                const int sb = job % kSbuf;
-                if (!(ok = mbar_wait(&s_full[sb], (job / kSbuf) & 1, ab, 8))) break;
+            // jobs of two blocks (one 256-column S buffer); the buffer is released after
+            // the second block's load
+            for (int jj = 0; jj < npj; jj += 2, ++sjob) {
+                const int sb = sjob & 1;
+                if (!(ok = mbar_wait(&s_full2[sb], (sjob >> 1) & 1, ab, 8))) break;
                 tc_fence_after();
-                float s[64];
-                tmem_ld32(lane_base + sbuf_col(sb) + c0, &s[0]);
-                tmem_ld32(lane_base + sbuf_col(sb) + c0 + 32, &s[32]);
-                tmem_wait_ld();
-                reg_fence<64>(s);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[sb]);
-                const int nv = key_end - b * kBlk - c0;   // valid columns of this thread: c < nv
-                const bool full_blk = __all_sync(0xffffffffu, nv >= 64);
-                if (!full_blk) {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
-                }
-                if (pass == 0) {
-                    float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
-#pragma unroll
-                    for (int c = 4; c < 64; c += 4) {
-                        m0 = fmaxf(m0, s[c]); m1 = fmaxf(m1, s[c + 1]);
-                        m2 = fmaxf(m2, s[c + 2]); m3 = fmaxf(m3, s[c + 3]);
+                const int nb2 = (jj + 1 < npj) ? 2 : 1;
+#pragma unroll 1
+                for (int h = 0; h < nb2; ++h) {
+                    const int bi = jj + h;      // block index within this pass
+                    const int b = (pass == 0) ? bi : job_list[bi];
+                    float s[64];
+                    tmem_ld32(lane_base + sb * 256 + h * 128 + c0, &s[0]);
+                    tmem_ld32(lane_base + sb * 256 + h * 128 + c0 + 32, &s[32]);
+                    tmem_wait_ld();
+                    reg_fence<64>(s);
+                    if (h == nb2 - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&s_empty2[sb]);
                     }
-                    const float xm = __fmul_rn(cx, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
-                    // per-warp block maximum (rounded up) for skipping in the solver passes
-                    float xw = xm;
+                    const int nv = key_end - b * kBlk - c0;   // valid columns of this thread: c < nv
+                    const bool full_blk = __all_sync(0xffffffffu, nv >= 64);
+                    if (!full_blk) {
 #pragma unroll
-                    for (int o2 = 16; o2 > 0; o2 >>= 1) xw = fmaxf(xw, __shfl_xor_sync(0xffffffffu, xw, o2));
-                    if (lane == 0) bmw[b * 8 + wi] = __float2bfloat16_ru(xw);
-                    if (xm > m) {
-                        m = xm;
-                        const int An = abs_bin(m);
-                        // bins leaving the window [A-w+1, A]: clear this half's 16 bits
-                        if (An > A && wbins > 0) {
-                            const int moved = An - A;
-                            if (moved >= wbins) {
-                                for (int sl = 0; sl < kBins; ++sl) clear_bin(sl);
-                            } else {
-                                for (int k2 = 0; k2 < moved; ++k2) clear_bin(A - wbins + 1 + k2);
+                        for (int c = 0; c < 64; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
+                    }
+                    if (pass == 0) {
+                        float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+#pragma unroll
+                        for (int c = 4; c < 64; c += 4) {
+                            m0 = fmaxf(m0, s[c]); m1 = fmaxf(m1, s[c + 1]);
+                            m2 = fmaxf(m2, s[c + 2]); m3 = fmaxf(m3, s[c + 3]);
+                        }
+                        const float xm = __fmul_rn(cx, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
+                        // per-warp block maximum (rounded up) for skipping in the solver passes
+                        float xw = xm;
+#pragma unroll
+                        for (int o2 = 16; o2 > 0; o2 >>= 1) xw = fmaxf(xw, __shfl_xor_sync(0xffffffffu, xw, o2));
+                        if (lane == 0) bmw[b * 8 + wi] = __float2bfloat16_ru(xw);
+                        if (xm > m) {
+                            m = xm;
+                            const int An = abs_bin(m);
+                            // bins leaving the window [A-w+1, A]: clear this half's 16 bits
+                            if (An > A && wbins > 0) {
+                                const int moved = An - A;
+                                if (moved >= wbins) {
+                                    for (int sl = 0; sl < kBins; ++sl) clear_bin(sl);
+                                } else {
+                                    for (int k2 = 0; k2 < moved; ++k2) clear_bin(A - wbins + 1 + k2);
+                                }
                             }
+                            A = An;
                         }
-                        A = An;
-                    }
-                    // Elements below the window's lowest bin (A-63)/63 <= m-1 are never in the
-                    // support; blocks whose maximum is below the window are skipped as a whole.
-                    if (wbins > 0 && *reinterpret_cast<volatile int*>(&misc->inserts) > kTileBudget) {
-                        for (int sl = 0; sl < kBins; ++sl) clear_bin(sl);   // tile over budget: stop
-                        wbins = 0;
-                    }
-                    const float thr_x = (float)(A - (wbins - 1)) / kBinsPerUnit - 1e-3f;
-                    if (__any_sync(0xffffffffu, xm >= thr_x && wbins > 0)) {
-                        // bin = floor(x*63) via the 1.5*2^23 rounding trick: rint(x*63 - 1/2)
-                        // (an element exactly on an edge may land one bin low, which keeps
-                        // the edge bounds valid)
-                        const int lo_bin = (wbins > 0) ? A - (wbins - 1) : 0x7FFFFFFF;
-#pragma unroll
-                        for (int c = 0; c < 64; ++c) {
-                            const float y = __fmaf_rn(s[c], c63, -0.5f) + 12582912.0f;
-                            const int ab2 = __float_as_int(y) - 0x4B400000;
-                            const bool q = ab2 >= lo_bin;
-                            if (q) red_shared_add_u32(hist_saddr + (ab2 & (kBins - 1)) * 512, hinc);
-                            n_ins += q;
+                        // Elements below the window's lowest bin (A-63)/63 <= m-1 are never in the
+                        // support; blocks whose maximum is below the window are skipped as a whole.
+                        if (wbins > 0 && *reinterpret_cast<volatile int*>(&misc->inserts) > kTileBudget) {
+                            for (int sl = 0; sl < kBins; ++sl) clear_bin(sl);   // tile over budget: stop
+                            wbins = 0;
                         }
-                        const int wsum = __reduce_add_sync(0xffffffffu, n_ins);
-                        if (lane == 0 && wsum && jj > 0) atomicAdd(&misc->inserts, wsum);
-                        n_ins = 0;
-                    }
-                } else {
-                    // two packed accumulator sets (columns c mod 4 < 2 and >= 2)
-                    float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, b0 = a0, b1 = a0, b2 = a0;
-                    const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-sv.tau, -sv.tau);
+                        const float thr_x = (float)(A - (wbins - 1)) / kBinsPerUnit - 1e-3f;
+                        if (__any_sync(0xffffffffu, xm >= thr_x && wbins > 0)) {
+                            // bin = floor(x*63) via the 1.5*2^23 rounding trick: rint(x*63 - 1/2)
+                            // (an element exactly on an edge may land one bin low, which keeps
+                            // the edge bounds valid)
+                            const int lo_bin = (wbins > 0) ? A - (wbins - 1) : 0x7FFFFFFF;
 #pragma unroll
-                    for (int c = 0; c < 64; c += 4) {
-                        entmax_acc_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma, a0, a1, a2);
-                        entmax_acc_x2<GM>(__ffma2_rn(make_float2(s[c + 2], s[c + 3]), cx2, nt2), gamma, b0, b1, b2);
+                            for (int c = 0; c < 64; ++c) {
+                                const float y = __fmaf_rn(s[c], c63, -0.5f) + 12582912.0f;
+                                const int ab2 = __float_as_int(y) - 0x4B400000;
+                                const bool q = ab2 >= lo_bin;
+                                if (q) red_shared_add_u32(hist_saddr + (ab2 & (kBins - 1)) * 512, hinc);
+                                n_ins += q;
+                            }
+                            const int wsum = __reduce_add_sync(0xffffffffu, n_ins);
+                            if (lane == 0 && wsum && bi > 0) atomicAdd(&misc->inserts, wsum);
+                            n_ins = 0;
+                        }
+                    } else {
+                        // two packed accumulator sets (columns c mod 4 < 2 and >= 2)
+                        float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, b0 = a0, b1 = a0, b2 = a0;
+                        const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-sv.tau, -sv.tau);
+#pragma unroll
+                        for (int c = 0; c < 64; c += 4) {
+                            entmax_acc_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma, a0, a1, a2);
+                            entmax_acc_x2<GM>(__ffma2_rn(make_float2(s[c + 2], s[c + 3]), cx2, nt2), gamma, b0, b1, b2);
+                        }
+                        a0 = __fadd2_rn(a0, b0); a1 = __fadd2_rn(a1, b1); a2 = __fadd2_rn(a2, b2);
+                        const float f1 = a1.x + a1.y;
+                        F0 += a0.x + a0.y; F1 += f1; F2 += a2.x + a2.y;
+                        // liveness: t1 = u^(gamma-1) > 0 exactly where u > 0 (up to underflow,
+                        // where p = u^gamma is 0 as well)
+                        if (__any_sync(0xffffffffu, f1 > 0.f) && lane == 0) live[b] = 1;
                     }
-                    a0 = __fadd2_rn(a0, b0); a1 = __fadd2_rn(a1, b1); a2 = __fadd2_rn(a2, b2);
-                    const float f1 = a1.x + a1.y;
-                    F0 += a0.x + a0.y; F1 += f1; F2 += a2.x + a2.y;
-                    // liveness: t1 = u^(gamma-1) > 0 exactly where u > 0 (up to underflow,
-                    // where p = u^gamma is 0 as well)
-                    if (__any_sync(0xffffffffu, f1 > 0.f) && lane == 0) live[b] = 1;
                 }
             }
+            // A wait that gave up ends the pass for this thread only; the group agrees
+            // here, so every thread leaves together and none is left at a barrier.
+            ok = named_bar_and(1, kEw, ok);
             if (!ok) break;
             if (pass == 0) {
                 // merge the two half-row histograms; the half-0 thread computes the start
@@ -511,10 +572,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (ok) {
             named_bar(1, kEw);   // job_list / njobs of the P.V pass visible to the group
             nlive = misc->njobs;
-            for (int li = 0; li < nlive; ++li, ++job) {
+            for (int li = 0; li < nlive; ++li) {
                 const int b = job_list[li];
-                const int sb = job % kSbuf;
-                if (!(ok = mbar_wait(&s_full[sb], (job / kSbuf) & 1, ab, 9))) break;
+                const int sb = li % kSbuf;   // the P.V pass counts its own jobs
+                if (!(ok = mbar_wait(&s_full[sb], (li / kSbuf) & 1, ab, 9))) break;
                 tc_fence_after();
                 float s[64];
                 tmem_ld32(lane_base + sbuf_col(sb) + c0, &s[0]);

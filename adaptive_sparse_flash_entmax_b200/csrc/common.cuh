@@ -99,9 +99,15 @@ struct RowSolver {
 // within the closed bracket [lo, hi] (a point that rounding put a few ulps
 // outside is clamped onto it: a root on a bracket end, such as tau = m - 1 for
 // a one-element support, must stay reachable); otherwise the bracket is bisected.
+// `accept` > 0 also stops on an upward Halley step of at most accept*max(1,|tau|),
+// taking the new point without evaluating it: the root is then within the step of
+// it (Halley's error is cubic in the step between support changes), and since tau
+// only grew the support only shrank, so the live blocks marked in this pass still
+// cover every block with p > 0 (a block marked live whose elements all lie in
+// (tau_old, tau_new] has max(x - tau) > -accept*max(1,|tau|)).
 __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1, float F2,
                                               float gamma, bool gamma_is_one, int pass,
-                                              float ftol, float stol) {
+                                              float ftol, float stol, float accept = 0.f) {
     if (st.done) return;
     const float f = F0 - 1.f;
     if (fabsf(f) <= ftol || pass >= kMaxPass) { st.done = 1; st.iters = pass; return; }
@@ -109,11 +115,14 @@ __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1,
     const float fp = -gamma * F1;
     const float fpp = gamma_is_one ? 0.f : gamma * (gamma - 1.f) * F2;
     const float h = st.tau - 2.f * f * fp / (2.f * fp * fp - f * fpp);
-    const float tol = stol * fmaxf(1.f, fabsf(st.tau));
-    const float next = (isfinite(h) && h >= st.lo - tol && h <= st.hi + tol)
-                           ? fminf(fmaxf(h, st.lo), st.hi)
-                           : 0.5f * (st.lo + st.hi);
+    const float scale = fmaxf(1.f, fabsf(st.tau));
+    const float tol = stol * scale;
+    const bool halley = isfinite(h) && h >= st.lo - tol && h <= st.hi + tol;
+    const float next = halley ? fminf(fmaxf(h, st.lo), st.hi) : 0.5f * (st.lo + st.hi);
     if (fabsf(next - st.tau) <= tol) { st.done = 1; st.iters = pass; return; }
+    if (halley && next > st.tau && next - st.tau <= accept * scale) {
+        st.tau = next; st.done = 1; st.iters = pass; return;
+    }
     st.tau = next;
 }
 

@@ -51,6 +51,8 @@ constexpr int kAtom = 128 * 128;   // bytes of a [128 rows x 64 bf16] swizzled a
 constexpr int kTmemCols = 512;     // score passes: S [0,256), [256,512); P.V pass: S0 [0,128),
                                    // S1 [128,256), O [256, 256+D), S2 [384, 512)
 constexpr int kDecSolve = 1, kDecPv = 2;
+// Largest upward Halley step taken without a verifying pass, relative to max(1,|tau|).
+constexpr float kAcceptStep = 5e-4f;
 
 __host__ __device__ constexpr uint32_t sbuf_col(int sb) { return sb < 2 ? sb * 128 : 384; }
 
@@ -535,7 +537,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 X(0, half) = F0; X(1, half) = F1; X(2, half) = F2;
                 named_bar(1, kEw);
                 const float G0 = F0 + X(0, half ^ 1), G1 = F1 + X(1, half ^ 1), G2 = F2 + X(2, half ^ 1);
-                solver_update(sv, G0, G1, G2, gamma, gamma == 1.f, pass, a.ftol, a.stol);
+                solver_update(sv, G0, G1, G2, gamma, gamma == 1.f, pass, a.ftol, a.stol, kAcceptStep);
             }
             const int all = named_bar_and(1, kEw, sv.done) && pass > 0;
             const uint8_t tag = (uint8_t)(pass + 2);

@@ -143,12 +143,20 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_init(in_full, 1);
         mbar_init(mma_done, 1);
         misc->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 2) {
+        // live key blocks of this tile, in order: 32 mask bytes per step, compacted by ballot
         const uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
         int n = 0;
-        for (int b = 0; b < nblk; ++b)
-            if (mrow[b]) list[n++] = (uint16_t)b;
-        misc->njobs = n;
-        fence_barrier_init();
+        for (int base = 0; base < nblk; base += 32) {
+            const int b = base + lane;
+            const bool f = b < nblk && mrow[b] != 0;
+            const unsigned int msk = __ballot_sync(0xffffffffu, f);
+            if (f) list[n + __popc(msk & ((1u << lane) - 1u))] = (uint16_t)b;
+            n += __popc(msk);
+        }
+        if (lane == 0) misc->njobs = n;
     }
     if (warp == 1) {
         tmem_alloc(&misc->tmem_base, kTmemCols);
@@ -438,17 +446,36 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         mbar_init(in_full, 1);
         mbar_init(mma_done, 1);
         misc->abort = 0;
-        int n = 0;
-        for (int t = a.causal ? b : 0; t < T; ++t) {
-            if (!a.mask[((size_t)bh * T + t) * T + b]) continue;
-            for (int h = 0; h < 2; ++h) {
-                const int i0 = t * kBlk + h * kSub;
-                if (i0 >= N || (a.causal && i0 + kSub - 1 < b * kBlk)) continue;
-                jobs[n++] = i0;
-            }
-        }
-        misc->njobs = n;
         fence_barrier_init();
+    }
+    if (warp == 2) {
+        // 64-row sub-tiles of the live query tiles of this key block, in order: one query
+        // tile per lane and step (the mask column is strided, so the loads go out in
+        // parallel), up to two jobs each, placed by a warp prefix sum
+        int n = 0;
+        for (int base = a.causal ? b : 0; base < T; base += 32) {
+            const int t = base + lane;
+            int c = 0, i0a = 0, i0b = 0;
+            if (t < T && a.mask[((size_t)bh * T + t) * T + b]) {
+                for (int h = 0; h < 2; ++h) {
+                    const int i0 = t * kBlk + h * kSub;
+                    if (i0 >= N || (a.causal && i0 + kSub - 1 < b * kBlk)) continue;
+                    if (c == 0) i0a = i0; else i0b = i0;
+                    ++c;
+                }
+            }
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int pos = n + incl - c;
+            if (c > 0) jobs[pos] = i0a;
+            if (c > 1) jobs[pos + 1] = i0b;
+            n += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) misc->njobs = n;
     }
     if (warp == 1) {
         tmem_alloc(&misc->tmem_base, kTmemCols);

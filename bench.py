@@ -226,6 +226,23 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------- ours
+def combine_ranks(ms: float, units: float, world: int, device) -> tuple:
+    """(max over ranks of the device time `ms`, sum over ranks of the work `units`).
+
+    Every rank calls it at the same point of the run (two all-reduces: MAX, then
+    SUM), so ``value = units / ms`` counts the work of all ranks against the slowest
+    rank's clock."""
+    if world == 1:
+        return ms, units
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return t.item(), u.item()
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -304,10 +321,8 @@ def run_ours(args):
     elapsed = t_start.elapsed_time(t_end)
     ms_fwd = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     ms_bwd = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step = t.item() / args.steps
+    ms_total, flops_all = combine_ranks(elapsed, exec_flops, world, dev)
+    ms_step = ms_total / args.steps
 
     # end to end through the public API from pinned host memory: every step copies its
     # inputs (Q, K, V, dO) in, runs forward + backward and copies O, dQ, dK, dV out.
@@ -362,10 +377,7 @@ def run_ours(args):
     e0.record(s_in)
     e1 = e2e_run(args.e2e_steps)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    ms_e2e = te.item()
+    ms_e2e, _ = combine_ranks(e0.elapsed_time(e1) / args.e2e_steps, exec_flops, world, dev)
 
     peaks, peak_kind = measured_peaks()
     sm_max = peaks.get("sm_max_mhz", 1965.0)
@@ -387,7 +399,7 @@ def run_ours(args):
         launches = 4    # forward + three backward kernels
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = profiled_traffic(w, roof["kernel"].split(":")[0])
-    value = world * exec_flops / (ms_step * 1e-3) / 1e12
+    value = flops_all / (ms_step * 1e-3) / 1e12
     line = None
     if rank == 0:
         clocks = clk.summary()
@@ -409,7 +421,7 @@ def run_ours(args):
             "data": "synthetic",
             "config": config_of(w, world),
             "ms_fwd": ms_fwd, "ms_bwd": ms_bwd,
-            "executed_tflop_per_step": exec_flops / 1e12,
+            "executed_tflop_per_step": flops_all / 1e12,
             "effective_dense_tflops": world * dense_flops(w) / (ms_step * 1e-3) / 1e12,
             "pct_bf16_peak_executed": 100 * value / world / peaks["bf16_tflops"],
             "block_sparsity": 1.0 - live / admissible,
@@ -417,7 +429,7 @@ def run_ours(args):
                            "tile_mean": cf[2] / max(1, cf[3])},
             "roofline": roof,
             "cpu_baseline": cpu,
-            "e2e": {"value": world * exec_flops / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+            "e2e": {"value": flops_all / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
             "gpu_launches": launches * args.steps,
             "clocks": clocks,

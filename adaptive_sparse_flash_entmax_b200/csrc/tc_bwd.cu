@@ -144,6 +144,13 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_init(mma_done, 1);
         misc->abort = 0;
         fence_barrier_init();
+        // Q and dO of the tile do not depend on the job list: start them first
+        prefetch_tmap(&tm_q); prefetch_tmap(&tm_do); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
+        mbar_arrive_expect_tx(in_full, 2 * L::kTile);
+        for (int at = 0; at < D / 64; ++at) {
+            tma_load_3d(smem + L::kQ + at * kAtom128, &tm_q, at * 64, t * kBlk, bh, in_full);
+            tma_load_3d(smem + L::kDO + at * kAtom128, &tm_do, at * 64, t * kBlk, bh, in_full);
+        }
     }
     if (warp == 2) {
         // live key blocks of this tile, in order: 32 mask bytes per step, compacted by ballot
@@ -174,12 +181,6 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     if (warp == 0) {
         if (lane == 0) {
-            prefetch_tmap(&tm_q); prefetch_tmap(&tm_do); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
-            mbar_arrive_expect_tx(in_full, 2 * L::kTile);
-            for (int at = 0; at < D / 64; ++at) {
-                tma_load_3d(smem + L::kQ + at * kAtom128, &tm_q, at * 64, t * kBlk, bh, in_full);
-                tma_load_3d(smem + L::kDO + at * kAtom128, &tm_do, at * 64, t * kBlk, bh, in_full);
-            }
             int nk = 0, nv = 0;   // K and V blocks issued
             bool ok = true;
             for (int j = 0; j < total && ok; ++j) {
@@ -447,6 +448,13 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         mbar_init(mma_done, 1);
         misc->abort = 0;
         fence_barrier_init();
+        // K and V of the block do not depend on the job list: start them first
+        prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_q64); prefetch_tmap(&tm_do64);
+        mbar_arrive_expect_tx(in_full, 2 * L::kTile);
+        for (int at = 0; at < D / 64; ++at) {
+            tma_load_3d(smem + L::kK + at * kAtom128, &tm_k, at * 64, b * kBlk, bh, in_full);
+            tma_load_3d(smem + L::kV + at * kAtom128, &tm_v, at * 64, b * kBlk, bh, in_full);
+        }
     }
     if (warp == 2) {
         // 64-row sub-tiles of the live query tiles of this key block, in order: one query
@@ -490,12 +498,6 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 
     if (warp == 0) {
         if (lane == 0) {
-            prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_q64); prefetch_tmap(&tm_do64);
-            mbar_arrive_expect_tx(in_full, 2 * L::kTile);
-            for (int at = 0; at < D / 64; ++at) {
-                tma_load_3d(smem + L::kK + at * kAtom128, &tm_k, at * 64, b * kBlk, bh, in_full);
-                tma_load_3d(smem + L::kV + at * kAtom128, &tm_v, at * 64, b * kBlk, bh, in_full);
-            }
             int job = 0;
             bool ok = true;
             for (; job < njobs && ok; ++job) {

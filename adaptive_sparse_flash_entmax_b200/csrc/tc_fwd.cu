@@ -152,6 +152,11 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         misc->abort = 0;
         misc->inserts = 0;
         fence_barrier_init();
+        // the Q tile goes first, before the block-wide setup
+        prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
+        mbar_arrive_expect_tx(q_full, L::kTile);
+        for (int at = 0; at < D / 64; ++at)
+            tma_load_3d(smem + L::kQ + at * kAtom, &tm_q, at * 64, t * kBlk, bh, q_full);
     }
     if (warp == 1) {
         tmem_alloc(&misc->tmem_base, kTmemCols);
@@ -166,12 +171,6 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
-            mbar_arrive_expect_tx(q_full, L::kTile);
-            for (int at = 0; at < D / 64; ++at)
-                tma_load_3d(smem + L::kQ + at * kAtom, &tm_q, at * 64, t * kBlk, bh, q_full);
             int sj = 0, dj = 0, kind = kDecSolve;   // P.V-pass tiles, score-pass double slots loaded
             uint32_t dec_phase = 0;
             bool ok = true, first = true;

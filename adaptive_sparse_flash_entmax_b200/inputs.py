@@ -19,6 +19,9 @@ stand-ins; the pages measure only on trained models and public datasets):
   distinct centres and every row of the tile is their mean + 0.1 N(0, I).
 * ``lm``    -- B8 H12 N2048 d64 bf16, causal, alpha 1.5; Q, K, V are heads of
   X W with X ~ N(0,1) [B, N, 768] and W Xavier-uniform [768, 2304].
+* ``clustered4k`` (supplementary) -- the ``long`` generator at the iid shape
+  (B4 H16 N4096 d128, beta 4); the cluster span (keys per centre, default 512)
+  sets the block sparsity, for a sweep between the dense iid case and ~95 %.
 """
 from __future__ import annotations
 
@@ -39,6 +42,7 @@ class Workload:
     alpha: float
     beta: float
     kind: str           # "iid", "clustered", "lm"
+    span: int = 512     # clustered: contiguous keys per cluster
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -54,6 +58,9 @@ WORKLOADS = {
     "alpha": Workload("alpha", 2, 16, 8192, 64, "bf16", True, 1.5, 4.0, "iid"),
     "long": Workload("long", 1, 16, 32768, 128, "bf16", True, 1.5, 4.0, "clustered"),
     "lm": Workload("lm", 8, 12, 2048, 64, "bf16", True, 1.5, 1.0, "lm"),
+    # supplementary (not one of the five configurations): the long workload's clustered
+    # generator at the iid shape, for a block-sparsity sweep over the cluster span
+    "clustered4k": Workload("clustered4k", 4, 16, 4096, 128, "bf16", True, 1.5, 4.0, "clustered"),
 }
 
 
@@ -97,7 +104,7 @@ def make_inputs(w: Workload, seed: int = 0):
     elif w.kind == "clustered":
         g = rng(seed * 16 + 0)
         centres = _normal(g, (B, H, 64, d))
-        span = np.arange(N) // 512 % 64
+        span = np.arange(N) // w.span % 64
         k = centres[:, :, span, :] + 0.1 * _normal(rng(seed * 16 + 1), (B, H, N, d))
         T = -(-N // 128)
         q = np.empty((B, H, T * 128, d), np.float32)

@@ -41,6 +41,10 @@ def parse():
     p.add_argument("--workload", default="iid", choices=sorted(inputs.WORKLOADS))
     p.add_argument("--beta", type=float, default=None)
     p.add_argument("--alpha", type=float, default=None)
+    p.add_argument("--span", type=int, default=None,
+                   help="cluster span in keys (clustered workloads; block-sparsity sweep)")
+    p.add_argument("--no-comparator", action="store_true",
+                   help="skip timing the dense softmax comparator (torch SDPA)")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--B", type=int, default=None, help="override the batch (profiling cases)")
     p.add_argument("--H", type=int, default=None, help="override the head count")
@@ -64,6 +68,8 @@ def workload(args) -> inputs.Workload:
         kw["B"] = args.B
     if args.H is not None:
         kw["H"] = args.H
+    if args.span is not None:
+        kw["span"] = args.span
     return w.replace(**kw) if kw else w
 
 
@@ -76,6 +82,8 @@ def config_of(w, n_gpus, extra=None):
          "parallelism": f"replicas x{n_gpus} (independent batches per GPU)",
          "l2": "inputs larger than L2: q, k, v, dO = %d MiB per GPU" % (
              4 * w.B * w.H * w.N * w.d * (2 if w.dtype == 'bf16' else 4) >> 20)}
+    if w.kind == "clustered":
+        c["cluster_span"] = w.span
     if extra:
         c.update(extra)
     return c
@@ -226,6 +234,47 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------- ours
+NOMINAL_BF16_TFLOPS = 2250.0   # dense bf16 tensor peak, nominal
+
+
+def time_dense_comparator(q, k, v, do, causal, steps):
+    """Softmax attention forward + backward with torch SDPA on the same tensors
+    (flash and cuDNN backends, the faster counts): measurement context only, not
+    part of the method.  Returns {"flash_ms", "cudnn_ms", "ms_per_step", "backend"}."""
+    import torch
+    import torch.nn.functional as F
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    out = {}
+    for name, backend in (("flash", SDPBackend.FLASH_ATTENTION), ("cudnn", SDPBackend.CUDNN_ATTENTION)):
+        try:
+            qq, kk, vv = (x.detach().requires_grad_() for x in (q, k, v))
+
+            def step():
+                qq.grad = kk.grad = vv.grad = None
+                with sdpa_kernel(backend):
+                    o = F.scaled_dot_product_attention(qq, kk, vv, is_causal=causal)
+                o.backward(do)
+
+            for _ in range(3):
+                step()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                step()
+            e1.record()
+            torch.cuda.synchronize()
+            out[name + "_ms"] = e0.elapsed_time(e1) / steps
+        except Exception:   # backend unavailable for this shape or build
+            out[name + "_ms"] = None
+    done = {k: v for k, v in out.items() if v is not None}
+    if done:
+        best = min(done, key=done.get)
+        out["ms_per_step"] = done[best]
+        out["backend"] = best[:-3]
+    return out
+
+
 def combine_ranks(ms: float, units: float, world: int, device) -> tuple:
     """(max over ranks of the device time `ms`, sum over ranks of the work `units`).
 
@@ -297,6 +346,7 @@ def run_ours(args):
     admissible = B * H * (T * (T + 1) // 2 if w.causal else T * T)
     live = int(mask.sum().item())
     iters = it.float()
+    pass_hist = torch.bincount(it.reshape(-1).long(), minlength=1).tolist()
 
     stream = torch.cuda.current_stream(dev)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -379,6 +429,14 @@ def run_ours(args):
     torch.cuda.synchronize()
     ms_e2e, _ = combine_ranks(e0.elapsed_time(e1) / args.e2e_steps, exec_flops, world, dev)
 
+    comparator = None
+    if not args.no_comparator and w.dtype == "bf16":
+        comparator = time_dense_comparator(qd, kd, vd, dod, w.causal, min(args.steps, 20))
+        if "ms_per_step" in comparator:
+            comparator["ours_over_dense"] = ms_step / comparator["ms_per_step"]
+        comparator["what"] = ("torch SDPA softmax attention fwd+bwd on the same tensors "
+                              "(measurement context, not the method)")
+
     peaks, peak_kind = measured_peaks()
     sm_max = peaks.get("sm_max_mhz", 1965.0)
     fwd_tflops = fwd_flops / (ms_fwd * 1e-3) / 1e12
@@ -424,9 +482,12 @@ def run_ours(args):
             "executed_tflop_per_step": flops_all / 1e12,
             "effective_dense_tflops": world * dense_flops(w) / (ms_step * 1e-3) / 1e12,
             "pct_bf16_peak_executed": 100 * value / world / peaks["bf16_tflops"],
+            "pct_bf16_nominal_executed": 100 * value / world / NOMINAL_BF16_TFLOPS,
             "block_sparsity": 1.0 - live / admissible,
             "tau_passes": {"row_mean": iters.mean().item(), "row_max": int(iters.max().item()),
-                           "tile_mean": cf[2] / max(1, cf[3])},
+                           "tile_mean": cf[2] / max(1, cf[3]),
+                           "row_histogram": {str(k): c for k, c in enumerate(pass_hist) if c}},
+            "dense_softmax_comparator": comparator,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": flops_all / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,

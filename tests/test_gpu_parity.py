@@ -230,3 +230,9 @@ def test_workload_long_clustered():
 
 def test_workload_lm():
     _sampled_parity(inputs.WORKLOADS["lm"], early_keys=16)
+
+
+def test_workload_clustered4k_span_sweep():
+    # supplementary block-sparsity sweep at the iid shape (cluster span sets the sparsity)
+    for span in (128, 2048):
+        _sampled_parity(inputs.WORKLOADS["clustered4k"].replace(span=span), n_rows=32, early_keys=8)

@@ -117,3 +117,50 @@ class EntmaxAttention(torch.autograd.Function):
 def entmax_attention(q, k, v, alpha: float = 1.5, causal: bool = False):
     """Differentiable fused alpha-entmax attention."""
     return EntmaxAttention.apply(q, k, v, alpha, causal)
+
+
+# ------------------------------------------------------------ row-wise entmax
+SOLVERS = {"hist": capi.ENT_SOLVE_HIST, "halley": capi.ENT_SOLVE_HALLEY,
+           "bisect": capi.ENT_SOLVE_BISECT}
+
+
+def _check_rows(*ts):
+    t0 = ts[0]
+    if t0.dim() != 2:
+        raise ValueError(f"expected [rows, n] tensors, got shape {tuple(t0.shape)}")
+    if t0.dtype not in _DTYPES:
+        raise ValueError(f"dtype {t0.dtype} not supported (float32 or bfloat16)")
+    for t in ts:
+        if t.shape != t0.shape or t.dtype != t0.dtype or t.device != t0.device:
+            raise ValueError("z, dp must share shape, dtype and device")
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def entmax_rows_fwd(z, alpha: float = 1.5, solver: str = "hist", *, out=None):
+    """Row-wise alpha-entmax of z [rows, n]: returns (p, tau [rows], iters [rows] uint8)."""
+    _check_rows(z)
+    rows, n = z.shape
+    if out is None:
+        p = torch.empty_like(z)
+        tau = torch.empty(rows, dtype=torch.float32, device=z.device)
+        iters = torch.empty(rows, dtype=torch.uint8, device=z.device)
+    else:
+        p, tau, iters = out
+    st = capi.ent_entmax_rows_fwd(z.data_ptr(), rows, n, _DTYPES[z.dtype], alpha, SOLVERS[solver],
+                                  p.data_ptr(), tau.data_ptr(),
+                                  iters.data_ptr() if iters is not None else None,
+                                  _stream_handle(z.device))
+    _raise(st, "ent_entmax_rows_fwd")
+    return p, tau, iters
+
+
+def entmax_rows_bwd(z, tau, dp, alpha: float = 1.5, *, out=None):
+    """Gradient w.r.t. z of sum(dp * entmax(z)) for the tau the forward returned."""
+    _check_rows(z, dp)
+    rows, n = z.shape
+    dz = torch.empty_like(z) if out is None else out
+    st = capi.ent_entmax_rows_bwd(z.data_ptr(), tau.data_ptr(), dp.data_ptr(), rows, n,
+                                  _DTYPES[z.dtype], alpha, dz.data_ptr(), _stream_handle(z.device))
+    _raise(st, "ent_entmax_rows_bwd")
+    return dz

@@ -16,6 +16,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "entattn.h")
 
 ENT_OK, ENT_EINVAL, ENT_EUNSUPPORTED, ENT_ECUDA, ENT_ETIMEOUT = 0, 1, 2, 3, 4
 ENT_F32, ENT_BF16 = 0, 1
+ENT_SOLVE_HIST, ENT_SOLVE_HALLEY, ENT_SOLVE_BISECT = 0, 1, 2
 STATUS_NAMES = {0: "ENT_OK", 1: "ENT_EINVAL", 2: "ENT_EUNSUPPORTED", 3: "ENT_ECUDA",
                 4: "ENT_ETIMEOUT"}
 
@@ -54,6 +55,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ent_attn_read_status.restype = ci
     lib.ent_attn_last_error.argtypes = []
     lib.ent_attn_last_error.restype = ctypes.c_char_p
+    lib.ent_entmax_rows_max_n.argtypes = []
+    lib.ent_entmax_rows_max_n.restype = ci
+    lib.ent_entmax_rows_fwd.argtypes = [vp, ci, ci, ci, cf, ci, vp, vp, vp, vp]
+    lib.ent_entmax_rows_fwd.restype = ci
+    lib.ent_entmax_rows_bwd.argtypes = [vp, vp, vp, ci, ci, ci, cf, vp, vp]
+    lib.ent_entmax_rows_bwd.restype = ci
     _lib = lib
     return lib
 
@@ -61,7 +68,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
 def header_symbols(header: str = HEADER) -> list[str]:
     """Names of the functions include/entattn.h declares."""
     text = open(header).read()
-    return sorted(set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(ent_attn_\w+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(ent_(?:attn|entmax)_\w+)\s*\(", text, re.M)))
 
 
 def ent_attn_block_size() -> int:
@@ -91,6 +98,19 @@ def ent_attn_bwd(q, k, v, o, dout, tau, block_mask, B, H, N, d, dtype, alpha, ca
                  dv, ws, ws_bytes, stream) -> int:
     return load().ent_attn_bwd(q, k, v, o, dout, tau, block_mask, B, H, N, d, dtype,
                                float(alpha), int(causal), dq, dk, dv, ws, ws_bytes, stream)
+
+
+def ent_entmax_rows_max_n() -> int:
+    return load().ent_entmax_rows_max_n()
+
+
+def ent_entmax_rows_fwd(z, rows, n, dtype, alpha, method, p, tau, iters, stream) -> int:
+    return load().ent_entmax_rows_fwd(z, rows, n, dtype, float(alpha), int(method), p, tau, iters,
+                                      stream)
+
+
+def ent_entmax_rows_bwd(z, tau, dp, rows, n, dtype, alpha, dz, stream) -> int:
+    return load().ent_entmax_rows_bwd(z, tau, dp, rows, n, dtype, float(alpha), dz, stream)
 
 
 def ent_attn_read_status(ws, stream) -> tuple[int, list[int]]:

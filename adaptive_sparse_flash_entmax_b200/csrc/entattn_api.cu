@@ -185,6 +185,68 @@ ent_status ent_attn_bwd(const void* q, const void* k, const void* v, const void*
     return ENT_OK;
 }
 
+int ent_entmax_rows_max_n(void) { return 16384; }
+
+}  // extern "C"
+
+namespace {
+
+static_assert(ENT_SOLVE_HIST == ent::kSolveHist && ENT_SOLVE_HALLEY == ent::kSolveHalley &&
+                  ENT_SOLVE_BISECT == ent::kSolveBisect,
+              "solver codes of the header and the kernels agree");
+
+ent_status check_rows(int rows, int n, int dtype, float alpha) {
+    if (rows < 0 || n < 0) return fail(ENT_EINVAL, "negative size (rows=%d n=%d)", rows, n);
+    if (dtype != ENT_F32 && dtype != ENT_BF16) return fail(ENT_EINVAL, "unknown dtype %d", dtype);
+    if (!(alpha > 1.f && alpha <= 2.f)) return fail(ENT_EINVAL, "alpha=%g outside (1, 2]", (double)alpha);
+    if (n > ent_entmax_rows_max_n())
+        return fail(ENT_EUNSUPPORTED, "n=%d exceeds %d", n, ent_entmax_rows_max_n());
+    return ENT_OK;
+}
+
+ent::RowArgs row_args(int rows, int n, int dtype, float alpha) {
+    ent::RowArgs a{};
+    a.rows = rows; a.n = n; a.alpha = alpha;
+    a.cx = alpha - 1.f;
+    a.ftol = dtype == ENT_F32 ? 1e-6f : 1e-5f;
+    a.stol = dtype == ENT_F32 ? 4e-7f : 1e-6f;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+ent_status ent_entmax_rows_fwd(const void* z, int rows, int n, int dtype, float alpha, int method,
+                               void* p, float* tau, uint8_t* iters, void* stream) {
+    ent_status st = check_rows(rows, n, dtype, alpha);
+    if (st != ENT_OK) return st;
+    if (method != ENT_SOLVE_HIST && method != ENT_SOLVE_HALLEY && method != ENT_SOLVE_BISECT)
+        return fail(ENT_EINVAL, "unknown method %d", method);
+    if (rows == 0 || n == 0) return ENT_OK;
+    if (!z || !p || !tau) return fail(ENT_EINVAL, "null z/p/tau pointer");
+    ent::RowArgs a = row_args(rows, n, dtype, alpha);
+    a.z = z; a.p = p; a.tau = tau; a.iters = iters; a.method = method;
+    const int gm = gamma_mode(alpha, &a.gamma);
+    cudaError_t e = ent::rows_entmax(a, dtype == ENT_BF16, gm, false, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "row entmax launch");
+    return ENT_OK;
+}
+
+ent_status ent_entmax_rows_bwd(const void* z, const float* tau, const void* dp, int rows, int n,
+                               int dtype, float alpha, void* dz, void* stream) {
+    ent_status st = check_rows(rows, n, dtype, alpha);
+    if (st != ENT_OK) return st;
+    if (rows == 0 || n == 0) return ENT_OK;
+    if (!z || !tau || !dp || !dz) return fail(ENT_EINVAL, "null z/tau/dp/dz pointer");
+    ent::RowArgs a = row_args(rows, n, dtype, alpha);
+    a.z = z; a.tau_in = tau; a.dp = dp; a.dz = dz;
+    const int gm = gamma_mode(alpha, &a.gamma);
+    cudaError_t e = ent::rows_entmax(a, dtype == ENT_BF16, gm, true, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "row entmax backward launch");
+    return ENT_OK;
+}
+
 ent_status ent_attn_read_status(const void* ws, long long* counters, void* stream) {
     if (!ws) return fail(ENT_EINVAL, "null workspace");
     ent::WsHeader h;

@@ -41,6 +41,25 @@ struct BwdArgs {
     float alpha, gamma, cx, scale;
 };
 
+// Row-wise alpha-entmax of a [rows][n] score matrix (rows.cu).  Solver codes match
+// the public ENT_SOLVE_* values.
+enum RowSolve { kSolveHist = 0, kSolveHalley = 1, kSolveBisect = 2 };
+
+struct RowArgs {
+    const void* z;         // scores [rows][n]
+    void* p;               // forward: probabilities [rows][n]
+    float* tau;            // forward: tau per row (x units)
+    uint8_t* iters;        // forward, nullable: solver passes per row
+    const float* tau_in;   // backward: tau per row
+    const void* dp;        // backward: upstream gradient [rows][n]
+    void* dz;              // backward: gradient w.r.t. z [rows][n]
+    int rows, n, method;
+    float alpha, gamma;    // gamma = 1/(alpha-1)
+    float cx;              // alpha - 1: x = cx * z
+    float ftol, stol;      // stop rule, as in FwdArgs
+};
+cudaError_t rows_entmax(const RowArgs& a, int dtype_bf16, int gm, bool bwd, cudaStream_t s);
+
 // FP32 CUDA-core path: float32 inputs (scores by FFMA, no TF32 rounding).
 cudaError_t simt_fwd_f32(const FwdArgs& a, int d, int gm, cudaStream_t s);
 cudaError_t simt_bwd_f32(const BwdArgs& a, int d, int gm, cudaStream_t s);

@@ -153,6 +153,45 @@ ent_status ent_attn_read_status(const void *ws, long long *counters, void *strea
 /* Thread-local message describing the last non-OK status of this thread. */
 const char *ent_attn_last_error(void);
 
+/*
+ * Row-wise alpha-entmax of a score matrix, without attention ("AdaSplash:
+ * Adaptive Sparse Flash Attention", Background and Technical Deep Dive /
+ * Accelerated Alpha-Entmax Transformation; "AdaSplash-2: ...", Sparse Attention
+ * Makes Waves): for each row of z [rows][n] (row-major, contiguous),
+ *     p_j = ((alpha-1) z_j - tau)_+^(1/(alpha-1)),   sum_j p_j = 1,
+ * with tau the root of f(tau) = sum_j ((alpha-1) z_j - tau)_+^gamma - 1, in units of
+ * (alpha-1) z.  `method` picks the root finder (same stop rule as the attention
+ * forward: |f| <= 1e-6 (float32) / 1e-5 (bf16), or a step below 4e-7 / 1e-6 of
+ * max(1,|tau|), or the pass cap):
+ *   ENT_SOLVE_HIST    Halley-bisection from the bracket and start of a 64-bin
+ *                     histogram of the row (the attention path's solver);
+ *   ENT_SOLVE_HALLEY  Halley-bisection from the plain bracket
+ *                     [m - 1, m - n^(1-alpha)] (m = row max), midpoint start;
+ *   ENT_SOLVE_BISECT  bisection on the plain bracket (pass cap 48).
+ * Outputs (device, caller-owned): p [rows][n] in the dtype of z, tau float
+ * [rows], iters uint8 [rows] (nullable; solver passes per row).  Supported:
+ * 1 < alpha <= 2, 1 <= n <= ent_entmax_rows_max_n() (ENT_EUNSUPPORTED above);
+ * rows = 0 or n = 0 is a no-op.  No workspace; asynchronous on `stream`.
+ * Returns ENT_EINVAL for a bad argument (checked before any work is queued),
+ * ENT_ECUDA if a launch fails.
+ */
+#define ENT_SOLVE_HIST 0
+#define ENT_SOLVE_HALLEY 1
+#define ENT_SOLVE_BISECT 2
+int ent_entmax_rows_max_n(void);
+ent_status ent_entmax_rows_fwd(const void *z, int rows, int n, int dtype, float alpha,
+                               int method, void *p, float *tau, uint8_t *iters, void *stream);
+
+/*
+ * Vector-Jacobian product of ent_entmax_rows_fwd (derived from the definition):
+ * dz_j = g_j (dp_j - delta), g_j = ((alpha-1) z_j - tau)_+^(gamma-1) (0 off the
+ * support), delta = sum_j g_j dp_j / sum_j g_j.  z, dp, dz [rows][n] in one dtype;
+ * tau float [rows] as the forward returned it.  Same limits and errors as the
+ * forward.
+ */
+ent_status ent_entmax_rows_bwd(const void *z, const float *tau, const void *dp, int rows, int n,
+                               int dtype, float alpha, void *dz, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

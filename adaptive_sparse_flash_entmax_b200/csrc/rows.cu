@@ -67,6 +67,74 @@ __device__ __forceinline__ void bisect_update(RowSolver& st, float F0, int pass,
     st.tau = next;
 }
 
+// Bracket and start from a full 64-bin row histogram, computed by one warp: the
+// bounds of hist_start_fn (the same G(j) = sum_{k<j} c_k (j-k)^gamma at the edges,
+// c_k the count k bins below the top bin A), with lane l evaluating the edges
+// j = l and l + 32 by direct sums and ballots locating the two crossings (G grows
+// with j); the bin-centre model at lo and hi is a warp sum.  All lanes return
+// the same values.
+template <int GM>
+__device__ __forceinline__ void hist_bracket_warp(const unsigned int* hist, int A, float m, int n,
+                                                  float alpha, float gamma, const float* ptab,
+                                                  float& lo, float& hi, float& tau0) {
+    const int lane = threadIdx.x & 31;
+    auto cnt = [&](int k) { return hist[(A - k) & (kBins - 1)]; };
+    // G(j) <= 63^gamma  and  G(j) >= 63^gamma at edge j (exact integers for gamma 1..4)
+    auto test = [&](int j, bool& le, bool& ge) {
+        if (GM >= 1 && GM <= 4) {
+            unsigned long long g = 0;
+            for (int k = 0; k < j; ++k) {
+                const unsigned long long w = (unsigned long long)(j - k);
+                const unsigned long long pw = (GM == 1) ? w : (GM == 2) ? w * w : (GM == 3) ? w * w * w : w * w * w * w;
+                g += (unsigned long long)cnt(k) * pw;
+            }
+            const unsigned long long thr = (GM == 1) ? 63ull : (GM == 2) ? 3969ull : (GM == 3) ? 250047ull : 15752961ull;
+            le = g <= thr;
+            ge = g >= thr;
+        } else {
+            float g = 0.f;   // G(j) / 63^gamma
+            for (int k = 0; k < j; ++k) g = fmaf((float)cnt(k), ptab[j - k], g);
+            le = g <= 1.f;
+            ge = g >= 1.f;
+        }
+    };
+    bool le0, ge0, le1, ge1, le2 = false, ge2 = false;
+    test(lane, le0, ge0);
+    test(lane + 32, le1, ge1);
+    if (lane == 0) test(64, le2, ge2);
+    const int nle = __popc(__ballot_sync(0xffffffffu, le0)) + __popc(__ballot_sync(0xffffffffu, le1)) +
+                    __shfl_sync(0xffffffffu, (int)le2, 0);
+    const int nge = __popc(__ballot_sync(0xffffffffu, ge0)) + __popc(__ballot_sync(0xffffffffu, ge1)) +
+                    __shfl_sync(0xffffffffu, (int)ge2, 0);
+    const int h_j = nle - 1;                   // edges 0 .. h_j have G <= 63^gamma (G(0) = 0)
+    const int l_j = nge > 0 ? 65 - nge : -1;   // edges l_j .. 64 have G >= 63^gamma
+    const float slack = 4.f * 1.1920929e-7f * fmaxf(1.f, fabsf(m));
+    const float plain_lo = m - 1.f;
+    const float plain_hi = m - exp2f((1.f - alpha) * __log2f((float)n));
+    lo = (l_j >= 0 && l_j + 1 <= kBins) ? fmaxf((float)(A - l_j) / kBinsPerUnit - slack, plain_lo) : plain_lo;
+    hi = fminf((float)(A + 1 - h_j) / kBinsPerUnit + slack, plain_hi);
+    if (hi < lo) hi = lo;
+    float fcl = 0.f, fch = 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int k = lane + 32 * h;
+        const float c = (float)cnt(k);
+        const float centre = ((float)(A - k) + 0.5f) / kBinsPerUnit;
+        fcl = fmaf(c, entmax_p<GM>(centre - lo, gamma), fcl);
+        fch = fmaf(c, entmax_p<GM>(centre - hi, gamma), fch);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        fcl += __shfl_xor_sync(0xffffffffu, fcl, o);
+        fch += __shfl_xor_sync(0xffffffffu, fch, o);
+    }
+    fcl -= 1.f;
+    fch -= 1.f;
+    float t0 = 0.5f * (lo + hi);
+    if (fcl > 0.f && fch < 0.f) t0 = lo + (hi - lo) * (fcl / (fcl - fch));
+    tau0 = fminf(fmaxf(t0, lo), hi);
+}
+
 template <typename T, int E, int GM>
 __global__ void __launch_bounds__(kRowThreads) rows_fwd_kernel(const RowArgs a) {
     __shared__ float red[3][kRowWarps];
@@ -106,12 +174,14 @@ __global__ void __launch_bounds__(kRowThreads) rows_fwd_kernel(const RowArgs a) 
             if (b >= A - (kBins - 1)) atomicAdd(&hist[b & (kBins - 1)], 1u);
         }
         __syncthreads();
-        if (tid == 0) {
-            hist_start<GM>(hist, 1, A, m, a.n, a.alpha, gamma, ptab, sv.lo, sv.hi, sv.tau);
-            bc[0] = sv.tau;
+        if (tid < 32) {
+            hist_bracket_warp<GM>(hist, A, m, a.n, a.alpha, gamma, ptab, sv.lo, sv.hi, sv.tau);
+            if (tid == 0) { bc[0] = sv.tau; red[0][0] = sv.lo; red[1][0] = sv.hi; }
         }
         __syncthreads();
         sv.tau = bc[0];
+        sv.lo = red[0][0];
+        sv.hi = red[1][0];
     }
     for (int pass = 1;; ++pass) {
         float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0;

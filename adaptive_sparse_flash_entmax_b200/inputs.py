@@ -69,6 +69,12 @@ def rng(seed: int) -> np.random.Generator:
     return np.random.Generator(np.random.Philox(key=seed))
 
 
+def row_scores(rows: int, n: int, seed: int = 0, scale: float = 1.0) -> np.ndarray:
+    """[rows, n] float32 scores ~ N(0, scale^2) (Philox stream (seed, 7)) for the
+    row-wise entmax op: the distribution of s = q.k/sqrt(d) on the iid workload."""
+    return (scale * _normal(rng(seed * 16 + 7), (rows, n))).astype(np.float32)
+
+
 def round_to_bf16(a: np.ndarray) -> np.ndarray:
     """float32 array whose values are ``a`` rounded to bfloat16 (nearest, ties even)."""
     a = np.ascontiguousarray(a, dtype=np.float32)

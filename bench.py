@@ -45,6 +45,8 @@ def parse():
                    help="cluster span in keys (clustered workloads; block-sparsity sweep)")
     p.add_argument("--no-comparator", action="store_true",
                    help="skip timing the dense softmax comparator (torch SDPA)")
+    p.add_argument("--no-rowop", action="store_true",
+                   help="skip timing the row-wise entmax op")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--B", type=int, default=None, help="override the batch (profiling cases)")
     p.add_argument("--H", type=int, default=None, help="override the head count")
@@ -275,6 +277,38 @@ def time_dense_comparator(q, k, v, do, causal, steps):
     return out
 
 
+def time_row_entmax(dev, seed, hbm_gbs, rows=16384, n=4096, alpha=1.5):
+    """The row-wise entmax op on a [rows, n] bf16 score matrix, per root finder:
+    ms per call, solver passes, and HBM throughput (z read once, p written once)."""
+    import torch
+    from adaptive_sparse_flash_entmax_b200 import attention as A
+    z = torch.from_numpy(inputs.row_scores(rows, n, seed)).to(torch.bfloat16).to(dev)
+    p = torch.empty_like(z)
+    tau = torch.empty(rows, dtype=torch.float32, device=dev)
+    it = torch.empty(rows, dtype=torch.uint8, device=dev)
+    nbytes = 2 * rows * n * 2 + rows * 5
+    out = {"shape": f"[{rows}, {n}] bf16 N(0,1) scores, alpha {alpha}",
+           "bytes_per_call": nbytes}
+    for solver in ("hist", "halley", "bisect"):
+        for _ in range(3):
+            A.entmax_rows_fwd(z, alpha, solver, out=(p, tau, it))
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(20):
+            A.entmax_rows_fwd(z, alpha, solver, out=(p, tau, it))
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 20
+        itf = it.float()
+        out[solver] = {"ms": ms, "passes_mean": itf.mean().item(), "passes_max": int(itf.max().item()),
+                       "gbs": nbytes / (ms * 1e-3) / 1e9,
+                       "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / hbm_gbs}
+    out["bisect_over_halley_passes"] = out["bisect"]["passes_mean"] / out["halley"]["passes_mean"]
+    out["bisect_over_hist_ms"] = out["bisect"]["ms"] / out["hist"]["ms"]
+    return out
+
+
 def combine_ranks(ms: float, units: float, world: int, device) -> tuple:
     """(max over ranks of the device time `ms`, sum over ranks of the work `units`).
 
@@ -439,6 +473,9 @@ def run_ours(args):
 
     peaks, peak_kind = measured_peaks()
     sm_max = peaks.get("sm_max_mhz", 1965.0)
+    rowop = None
+    if not args.no_rowop:
+        rowop = time_row_entmax(dev, args.seed, peaks["hbm_gbs"])
     fwd_tflops = fwd_flops / (ms_fwd * 1e-3) / 1e12
     if w.dtype == "bf16":
         # tcgen05 forward: executed MMA flops against the sustained bf16 tensor peak
@@ -488,6 +525,7 @@ def run_ours(args):
                            "tile_mean": cf[2] / max(1, cf[3]),
                            "row_histogram": {str(k): c for k, c in enumerate(pass_hist) if c}},
             "dense_softmax_comparator": comparator,
+            "rowwise_entmax": rowop,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": flops_all / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,

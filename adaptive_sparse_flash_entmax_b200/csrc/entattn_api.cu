@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -46,6 +47,18 @@ int gamma_mode(float alpha, float* gamma_out) {
         return (int)r;
     }
     *gamma_out = gamma;
+    return 0;
+}
+
+// Histogram insert budget of a bf16 forward tile (after its first block).  The
+// default 0 starts every row from the plain bracket [m-1, m - n^(1-alpha)]: on B200
+// the histogram's inserts and per-row bracket cost more than the ~2 solver passes
+// they save, on every workload measured (the tiles then run ~4 cheap passes).
+// ENTATTN_HIST_BUDGET selects the histogram start instead: a positive budget builds
+// it until the tile has made that many inserts, a negative one always.
+int hist_budget() {
+    const char* v = getenv("ENTATTN_HIST_BUDGET");
+    if (v && *v) return atoi(v);
     return 0;
 }
 
@@ -127,6 +140,7 @@ ent_status ent_attn_fwd(const void* q, const void* k, const void* v, int B, int 
     // far below their rounding; float32 outputs get 1e-6.
     a.ftol = dtype == ENT_F32 ? 1e-6f : 1e-5f;
     a.stol = dtype == ENT_F32 ? 4e-7f : 1e-6f;
+    a.hist_budget = hist_budget();
     if (dtype == ENT_F32) {
         e = ent::simt_fwd_f32(a, d, gm, s);
     } else {

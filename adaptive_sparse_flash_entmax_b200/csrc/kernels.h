@@ -21,6 +21,8 @@ struct FwdArgs {
     float cx;              // (alpha-1)/sqrt(d): x = cx * (q . k)
     float scale;           // 1/sqrt(d)
     float ftol, stol;      // solver stop rule: |f| <= ftol, or a step <= stol*max(1,|tau|)
+    int hist_budget;       // tensor-core path: histogram inserts a tile may make after its
+                           // first block (0: no histogram, < 0: no limit)
 };
 
 struct BwdArgs {

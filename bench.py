@@ -47,6 +47,9 @@ def parse():
                    help="skip timing the dense softmax comparator (torch SDPA)")
     p.add_argument("--no-rowop", action="store_true",
                    help="skip timing the row-wise entmax op")
+    p.add_argument("--hist-budget", type=int, default=None,
+                   help="ablation: histogram insert budget per forward tile (0: no histogram, "
+                        "i.e. every row from the plain bracket; -1: no limit)")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--B", type=int, default=None, help="override the batch (profiling cases)")
     p.add_argument("--H", type=int, default=None, help="override the head count")
@@ -86,6 +89,11 @@ def config_of(w, n_gpus, extra=None):
              4 * w.B * w.H * w.N * w.d * (2 if w.dtype == 'bf16' else 4) >> 20)}
     if w.kind == "clustered":
         c["cluster_span"] = w.span
+    hb = os.environ.get("ENTATTN_HIST_BUDGET")
+    c["tau_start"] = ("plain bracket" if not hb or int(hb) == 0 else
+                      f"histogram (insert budget {hb})")
+    if hb:
+        c["hist_budget"] = int(hb)
     if extra:
         c.update(extra)
     return c
@@ -327,6 +335,8 @@ def combine_ranks(ms: float, units: float, world: int, device) -> tuple:
 
 
 def run_ours(args):
+    if args.hist_budget is not None:   # read by the library at each forward call
+        os.environ["ENTATTN_HIST_BUDGET"] = str(args.hist_budget)
     import torch
     import torch.distributed as dist
 

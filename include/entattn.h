@@ -82,6 +82,13 @@ size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype);
  * after the histogram pass.  Per 128-row query tile the kernel runs one
  * statistics pass (row max and score histogram), solver passes until every
  * row of the tile has converged, and one P.V pass over the live key blocks.
+ * bf16 inputs start every row's solver from the plain bracket [m-1, m - n^(1-alpha)]
+ * (measured faster on B200 than the histogram start, whose inserts cost more than
+ * the passes they save).  The environment variable ENTATTN_HIST_BUDGET, read at each
+ * call, selects the histogram start of the statistics pass instead: a tile builds
+ * the histogram until it has made that many inserts after its first block (a
+ * negative value: no limit).  float32 inputs always use the histogram start.  The
+ * result is the same to the solver's stop rule either way.
  */
 ent_status ent_attn_fwd(const void *q, const void *k, const void *v,
                         int B, int H, int N, int d, int dtype,

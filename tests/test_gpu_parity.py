@@ -236,3 +236,19 @@ def test_workload_clustered4k_span_sweep():
     # supplementary block-sparsity sweep at the iid shape (cluster span sets the sparsity)
     for span in (128, 2048):
         _sampled_parity(inputs.WORKLOADS["clustered4k"].replace(span=span), n_rows=32, early_keys=8)
+
+
+@pytest.mark.parametrize("budget", ["-1", "6144"])
+def test_histogram_start(monkeypatch, budget):
+    # the histogram start of the statistics pass (selected by ENTATTN_HIST_BUDGET, read at
+    # each forward call): the same results as the plain-bracket default
+    monkeypatch.setenv("ENTATTN_HIST_BUDGET", budget)
+    for N, d, causal, alpha in [(300, 64, True, 1.5), (384, 128, False, 2.0),
+                                (128, 64, True, 1.25), (384, 128, True, 1.7)]:
+        w, (q, k, v, do) = inputs.small_case(B=1, H=2, N=N, d=d, causal=causal, alpha=alpha,
+                                             beta=2.0, seed=N + d + 1)
+        full_parity(q, k, v, do, alpha, causal, "bf16")
+    w, (q, k, v, do) = inputs.small_case(B=1, H=2, N=1000, d=128, causal=True, beta=4.0,
+                                         kind="clustered", seed=5)
+    full_parity(q, k, v, do, w.alpha, w.causal, "bf16", bwd=False)
+    _sampled_parity(inputs.WORKLOADS["alpha"], early_keys=8)

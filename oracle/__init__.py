@@ -57,6 +57,8 @@ def _L():
                                      c_int, c_int, _dp, _dp, _dp, c_int]
         lib.orc_attn_fwd_rows.argtypes = [_dp, _dp, _dp, c_int, c_int, c_int, c_int, c_double,
                                           c_int, c_int, _i64p, c_int, _dp, _dp, _dp, c_int]
+        lib.orc_attn_otilde_rows.argtypes = [_dp, _dp, _dp, c_int, c_int, c_int, c_int,
+                                             c_double, c_int, _i64p, c_int, _dp, c_int]
         lib.orc_attn_bwd.argtypes = [_dp, _dp, _dp, _dp, c_int, c_int, c_int, c_int, c_double,
                                      c_int, _dp, _dp, _dp, _dp, _dp, c_int]
         lib.orc_attn_bwd_head_sampled.argtypes = [_dp, _dp, _dp, _dp, c_int, c_int, c_double,
@@ -163,6 +165,18 @@ def attn_fwd_rows(q, k, v, alpha, causal, rows, blk=128, nthreads=0):
                                   blk, _ptr(rows, _i64p), rows.size, _ptr(o), _ptr(tau),
                                   _ptr(bmax), nthreads), "attn_fwd_rows")
     return o, tau, bmax
+
+
+def attn_otilde_rows(q, k, v, alpha, causal, rows, nthreads=0):
+    """otilde_i = sum_j g_ij v_j / sum_j g_ij for flat row ids (b*H+h)*N+i: [R, d]."""
+    q, k, v = _d(q), _d(k), _d(v)
+    B, H, N, d = q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    ot = np.zeros((rows.size, d))
+    _check(_L().orc_attn_otilde_rows(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, alpha, int(causal),
+                                     _ptr(rows, _i64p), rows.size, _ptr(ot), nthreads),
+           "attn_otilde_rows")
+    return ot
 
 
 def attn_bwd(q, k, v, do, alpha, causal, nthreads=0):

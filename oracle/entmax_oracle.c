@@ -330,6 +330,54 @@ int orc_attn_fwd_rows(const double *q, const double *k, const double *v,
     return bad ? -1 : 0;
 }
 
+/*
+ * The g-weighted mean of the value rows for a list of rows (rows[r] = (b*H +
+ * h)*N + i): otilde_i = sum_j g_ij v_j / sum_j g_ij, g = (x - tau)_+^(gamma-1)
+ * at the row's exact tau.  It follows from the backward's definition of delta
+ * (delta_i = sum_j g_ij dP_ij / sum_j g_ij) and dP = dO V^T: delta_i =
+ * dO_i . otilde_i, so a forward that returns otilde lets the backward skip
+ * its delta pass over the keys.  Plain definition, row by row.
+ */
+int orc_attn_otilde_rows(const double *q, const double *k, const double *v,
+                         int B, int H, int N, int d, double alpha, int causal,
+                         const int64_t *rows, int nrows, double *ot_rows, int nthreads)
+{
+    if (B < 0 || H < 0 || N < 1 || d < 1 || !(alpha > 1.0)) return -1;
+    const double gamma = 1.0 / (alpha - 1.0);
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)N);
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < nrows; ++r) {
+            const int64_t flat = rows[r];
+            if (flat < 0 || flat >= (int64_t)B * H * N) { bad = 1; continue; }
+            const int64_t bh = flat / N;
+            const int i = (int)(flat % N);
+            const int n = n_admissible(i, N, causal);
+            const double *vh = v + (size_t)bh * N * d;
+            score_row(q + (size_t)flat * d, k + (size_t)bh * N * d, n, d, s);
+            double tau;
+            orc_entmax_tau(s, n, alpha, &tau);
+            double *ot = ot_rows + (size_t)r * d;
+            double sg = 0.0;
+            for (int c = 0; c < d; ++c) ot[c] = 0.0;
+            for (int j = 0; j < n; ++j) {
+                const double g = entmax_g((alpha - 1.0) * s[j] - tau, gamma);
+                if (g == 0.0) continue;
+                sg += g;
+                for (int c = 0; c < d; ++c) ot[c] += g * vh[(size_t)j * d + c];
+            }
+            for (int c = 0; c < d; ++c) ot[c] = (sg > 0.0) ? ot[c] / sg : 0.0;
+        }
+        free(s);
+    }
+    return bad ? -1 : 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Attention, backward.                                                      */
 /* ------------------------------------------------------------------------ */

@@ -323,6 +323,52 @@ def test_backward_sum_rules(orc):
     np.testing.assert_allclose(dv.sum(axis=2), do.sum(axis=2), atol=1e-11)
 
 
+# ------------------------------------------------------------ otilde (g-weighted value mean)
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0])
+def test_otilde_vs_brute_force(orc, causal, alpha):
+    """otilde_i = sum_j g_ij v_j / sum_j g_ij with g = (x - tau)_+^(gamma - 1), tau and the
+    support from the brute-force enumeration."""
+    g = np.random.default_rng(31)
+    q, k, v = (g.normal(size=(1, 2, 7, 3)) for _ in range(3))
+    rows = np.arange(14)
+    ot = orc.attn_otilde_rows(q, k, v, alpha, causal, rows)
+    S = np.einsum("bhid,bhjd->bhij", q, k) / np.sqrt(3)
+    for flat in rows:
+        h, i = divmod(int(flat), 7)
+        n = i + 1 if causal else 7
+        (t, supp), = brute_force_tau(S[0, h, i, :n], alpha)
+        u = (alpha - 1) * S[0, h, i, :n] - t
+        w = np.zeros(n)
+        idx = sorted(supp)
+        w[idx] = u[idx] ** (1 / (alpha - 1) - 1)
+        np.testing.assert_allclose(ot[flat], w @ v[0, h, :n] / w.sum(), atol=1e-11)
+
+
+def test_otilde_sparsemax_is_support_mean(orc):
+    """At alpha = 2, g is the support indicator: otilde is the plain mean of the values
+    on the support, which the sort-based closed form of tau fixes."""
+    g = np.random.default_rng(32)
+    q, k, v = (g.normal(size=(1, 1, 40, 8)) for _ in range(3))
+    ot = orc.attn_otilde_rows(q, k, v, 2.0, False, np.arange(40))
+    S = q[0, 0] @ k[0, 0].T / np.sqrt(8)
+    for i in range(40):
+        supp = S[i] > orc.sparsemax_tau_sort(S[i])
+        np.testing.assert_allclose(ot[i], v[0, 0][supp].mean(axis=0), atol=1e-11)
+
+
+def test_otilde_gives_backward_delta(orc):
+    """dO_i . otilde_i equals the backward's delta_i = sum_j g_ij dP_ij / sum_j g_ij, which
+    the backward computes through dP = dO V^T (another contraction order)."""
+    g = np.random.default_rng(33)
+    q, k, v, do = (g.normal(size=(2, 2, 33, 8)) for _ in range(4))
+    for alpha, causal in ((1.5, True), (1.25, False), (2.0, True)):
+        _, _, _, _, delta = orc.attn_bwd(q, k, v, do, alpha, causal)
+        ot = orc.attn_otilde_rows(q, k, v, alpha, causal, np.arange(2 * 2 * 33))
+        np.testing.assert_allclose(np.einsum("rd,rd->r", do.reshape(-1, 8), ot),
+                                   delta.reshape(-1), atol=1e-11)
+
+
 # ------------------------------------------------------------ iteration counts
 def test_iterative_solvers_converge_and_counts(orc):
     """All three root-finders land on the bisection tau; pass counts follow the

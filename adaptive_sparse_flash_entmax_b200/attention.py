@@ -43,8 +43,12 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def entmax_attn_fwd(q, k, v, alpha: float = 1.5, causal: bool = False, *, with_iters=False,
-                    ws: torch.Tensor | None = None, out=None):
-    """Forward: returns (o, tau, block_mask, iters_or_None)."""
+                    ws: torch.Tensor | None = None, out=None, otilde=None):
+    """Forward: returns (o, tau, block_mask, iters_or_None).
+
+    ``otilde``: a float32 tensor shaped like q to call ``ent_attn_fwd_otilde`` instead,
+    which also fills it with sum_j g_ij v_j / sum_j g_ij (the backward's delta is then
+    dO . otilde, see ``entmax_attn_bwd``)."""
     _check(q, k, v)
     B, H, N, d = q.shape
     dt = _DTYPES[q.dtype]
@@ -59,17 +63,31 @@ def entmax_attn_fwd(q, k, v, alpha: float = 1.5, causal: bool = False, *, with_i
     need = capi.ent_attn_fwd_workspace_size(B, H, N, d, dt)
     if ws is None or ws.numel() < need:
         ws = workspace(need, q.device)
-    st = capi.ent_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, dt, alpha,
-                           causal, o.data_ptr(), tau.data_ptr(), mask.data_ptr(),
-                           iters.data_ptr() if iters is not None else None, ws.data_ptr(),
-                           ws.numel(), _stream_handle(q.device))
-    _raise(st, "ent_attn_fwd")
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, dt, alpha, causal, o.data_ptr(),
+            tau.data_ptr(), mask.data_ptr(), iters.data_ptr() if iters is not None else None)
+    tail = (ws.data_ptr(), ws.numel(), _stream_handle(q.device))
+    if otilde is None:
+        st = capi.ent_attn_fwd(*args, *tail)
+        _raise(st, "ent_attn_fwd")
+    else:
+        _check_otilde(otilde, q)
+        st = capi.ent_attn_fwd_otilde(*args, otilde.data_ptr(), *tail)
+        _raise(st, "ent_attn_fwd_otilde")
     return o, tau, mask, iters
 
 
+def _check_otilde(otilde, q):
+    if (otilde.dtype != torch.float32 or otilde.shape != q.shape or otilde.device != q.device
+            or not otilde.is_contiguous()):
+        raise ValueError("otilde must be a contiguous float32 tensor shaped like q, on its device")
+
+
 def entmax_attn_bwd(q, k, v, o, dout, tau, block_mask, alpha: float = 1.5, causal: bool = False,
-                    *, ws: torch.Tensor | None = None, out=None):
-    """Backward: returns (dq, dk, dv)."""
+                    *, ws: torch.Tensor | None = None, out=None, otilde=None):
+    """Backward: returns (dq, dk, dv).
+
+    ``otilde``: the tensor a forward with ``otilde=`` filled; the call then goes to
+    ``ent_attn_bwd_otilde`` (delta = dO . otilde, no delta pass over the keys)."""
     _check(q, k, v, dout)
     B, H, N, d = q.shape
     dt = _DTYPES[q.dtype]
@@ -80,12 +98,18 @@ def entmax_attn_bwd(q, k, v, o, dout, tau, block_mask, alpha: float = 1.5, causa
     need = capi.ent_attn_bwd_workspace_size(B, H, N, d, dt)
     if ws is None or ws.numel() < need:
         ws = workspace(need, q.device)
-    st = capi.ent_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                           o.data_ptr() if o is not None else None, dout.data_ptr(),
-                           tau.data_ptr(), block_mask.data_ptr(), B, H, N, d, dt, alpha, causal,
-                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(),
-                           _stream_handle(q.device))
-    _raise(st, "ent_attn_bwd")
+    tail = (dout.data_ptr(), tau.data_ptr(), block_mask.data_ptr(), B, H, N, d, dt, alpha, causal,
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(),
+            _stream_handle(q.device))
+    if otilde is None:
+        st = capi.ent_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                               o.data_ptr() if o is not None else None, *tail)
+        _raise(st, "ent_attn_bwd")
+    else:
+        _check_otilde(otilde, q)
+        st = capi.ent_attn_bwd_otilde(q.data_ptr(), k.data_ptr(), v.data_ptr(), otilde.data_ptr(),
+                                      *tail)
+        _raise(st, "ent_attn_bwd_otilde")
     return dq, dk, dv
 
 
@@ -97,26 +121,36 @@ def read_status(ws: torch.Tensor) -> list[int]:
 
 
 class EntmaxAttention(torch.autograd.Function):
-    """Autograd wrapper: O = entmax_alpha(Q K^T / sqrt(d)) V."""
+    """Autograd wrapper: O = entmax_alpha(Q K^T / sqrt(d)) V.
+
+    With ``delta="otilde"`` the forward also returns otilde (float32, shaped like q) and
+    saves it, and the backward takes delta = dO . otilde instead of a delta pass over the
+    keys; ``delta="recompute"`` saves nothing extra and recomputes delta from the scores."""
 
     @staticmethod
-    def forward(ctx, q, k, v, alpha, causal):
+    def forward(ctx, q, k, v, alpha, causal, delta):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        o, tau, mask, _ = entmax_attn_fwd(q, k, v, alpha, causal)
-        ctx.save_for_backward(q, k, v, o, tau, mask)
+        ot = None
+        if delta == "otilde" and any(ctx.needs_input_grad[:3]):
+            ot = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        elif delta not in ("otilde", "recompute"):
+            raise ValueError(f"delta must be 'otilde' or 'recompute', not {delta!r}")
+        o, tau, mask, _ = entmax_attn_fwd(q, k, v, alpha, causal, otilde=ot)
+        ctx.save_for_backward(q, k, v, o, tau, mask, ot)
         ctx.alpha, ctx.causal = alpha, causal
         return o
 
     @staticmethod
     def backward(ctx, do):
-        q, k, v, o, tau, mask = ctx.saved_tensors
-        dq, dk, dv = entmax_attn_bwd(q, k, v, o, do.contiguous(), tau, mask, ctx.alpha, ctx.causal)
-        return dq, dk, dv, None, None
+        q, k, v, o, tau, mask, ot = ctx.saved_tensors
+        dq, dk, dv = entmax_attn_bwd(q, k, v, o, do.contiguous(), tau, mask, ctx.alpha, ctx.causal,
+                                     otilde=ot)
+        return dq, dk, dv, None, None, None
 
 
-def entmax_attention(q, k, v, alpha: float = 1.5, causal: bool = False):
-    """Differentiable fused alpha-entmax attention."""
-    return EntmaxAttention.apply(q, k, v, alpha, causal)
+def entmax_attention(q, k, v, alpha: float = 1.5, causal: bool = False, delta: str = "otilde"):
+    """Differentiable fused alpha-entmax attention (``delta``: see EntmaxAttention)."""
+    return EntmaxAttention.apply(q, k, v, alpha, causal, delta)
 
 
 # ------------------------------------------------------------ row-wise entmax

@@ -51,6 +51,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ent_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp, vp,
                                  vp, vp, sz, vp]
     lib.ent_attn_bwd.restype = ci
+    lib.ent_attn_fwd_otilde.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp, vp, vp, vp, vp,
+                                        vp, sz, vp]
+    lib.ent_attn_fwd_otilde.restype = ci
+    lib.ent_attn_bwd_otilde.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp,
+                                        vp, vp, vp, sz, vp]
+    lib.ent_attn_bwd_otilde.restype = ci
     lib.ent_attn_read_status.argtypes = [vp, ctypes.POINTER(ctypes.c_longlong), vp]
     lib.ent_attn_read_status.restype = ci
     lib.ent_attn_last_error.argtypes = []
@@ -98,6 +104,18 @@ def ent_attn_bwd(q, k, v, o, dout, tau, block_mask, B, H, N, d, dtype, alpha, ca
                  dv, ws, ws_bytes, stream) -> int:
     return load().ent_attn_bwd(q, k, v, o, dout, tau, block_mask, B, H, N, d, dtype,
                                float(alpha), int(causal), dq, dk, dv, ws, ws_bytes, stream)
+
+
+def ent_attn_fwd_otilde(q, k, v, B, H, N, d, dtype, alpha, causal, o, tau, block_mask, iters,
+                        otilde, ws, ws_bytes, stream) -> int:
+    return load().ent_attn_fwd_otilde(q, k, v, B, H, N, d, dtype, float(alpha), int(causal), o,
+                                      tau, block_mask, iters, otilde, ws, ws_bytes, stream)
+
+
+def ent_attn_bwd_otilde(q, k, v, otilde, dout, tau, block_mask, B, H, N, d, dtype, alpha, causal,
+                        dq, dk, dv, ws, ws_bytes, stream) -> int:
+    return load().ent_attn_bwd_otilde(q, k, v, otilde, dout, tau, block_mask, B, H, N, d, dtype,
+                                      float(alpha), int(causal), dq, dk, dv, ws, ws_bytes, stream)
 
 
 def ent_entmax_rows_max_n() -> int:

@@ -107,10 +107,15 @@ size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype) {
 
 const char* ent_attn_last_error(void) { return g_err.c_str(); }
 
-ent_status ent_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d,
-                        int dtype, float alpha, int causal, void* o, float* tau,
-                        uint8_t* block_mask, uint8_t* iters, void* ws, size_t ws_bytes,
-                        void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Forward of ent_attn_fwd and, with a non-null otilde, of ent_attn_fwd_otilde.
+ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                    int dtype, float alpha, int causal, void* o, float* tau, uint8_t* block_mask,
+                    uint8_t* iters, float* otilde, bool want_otilde, void* ws, size_t ws_bytes,
+                    void* stream) {
     ent_status st = check_common(B, H, N, d, dtype, alpha, causal);
     if (st != ENT_OK) return st;
     if (!ws) return fail(ENT_EINVAL, "null workspace");
@@ -123,13 +128,16 @@ ent_status ent_attn_fwd(const void* q, const void* k, const void* v, int B, int 
         return fail(ENT_EINVAL, "null q/k/v/o/tau/block_mask pointer");
     if (!empty && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)))
         return fail(ENT_EINVAL, "q/k/v/o must be 16-byte aligned");
+    if (!empty && want_otilde && (!otilde || !aligned16(otilde)))
+        return fail(ENT_EINVAL, "otilde must be a non-null 16-byte aligned pointer");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace header");
     if (empty) return ENT_OK;
 
-    ent::FwdArgs a;
+    ent::FwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.o = o; a.tau = tau; a.mask = block_mask; a.iters = iters;
+    a.otilde = want_otilde ? otilde : nullptr;
     a.hdr = static_cast<ent::WsHeader*>(ws);
     a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal;
     a.alpha = alpha;
@@ -152,11 +160,12 @@ ent_status ent_attn_fwd(const void* q, const void* k, const void* v, int B, int 
     return ENT_OK;
 }
 
-ent_status ent_attn_bwd(const void* q, const void* k, const void* v, const void* o,
-                        const void* dout, const float* tau, const uint8_t* block_mask, int B,
-                        int H, int N, int d, int dtype, float alpha, int causal, void* dq,
-                        void* dk, void* dv, void* ws, size_t ws_bytes, void* stream) {
-    (void)o;
+// Backward of ent_attn_bwd and, with a non-null otilde, of ent_attn_bwd_otilde.
+ent_status bwd_impl(const void* q, const void* k, const void* v, const float* otilde,
+                    bool want_otilde, const void* dout, const float* tau,
+                    const uint8_t* block_mask, int B, int H, int N, int d, int dtype, float alpha,
+                    int causal, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                    void* stream) {
     ent_status st = check_common(B, H, N, d, dtype, alpha, causal);
     if (st != ENT_OK) return st;
     if (!ws) return fail(ENT_EINVAL, "null workspace");
@@ -170,14 +179,17 @@ ent_status ent_attn_bwd(const void* q, const void* k, const void* v, const void*
     if (!empty && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) ||
                    !aligned16(dq) || !aligned16(dk) || !aligned16(dv)))
         return fail(ENT_EINVAL, "q/k/v/dout/dq/dk/dv must be 16-byte aligned");
+    if (!empty && want_otilde && (!otilde || !aligned16(otilde)))
+        return fail(ENT_EINVAL, "otilde must be a non-null 16-byte aligned pointer");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace header");
     if (empty) return ENT_OK;
 
-    ent::BwdArgs a;
+    ent::BwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.dout = dout; a.tau = tau; a.mask = block_mask;
     a.dq = dq; a.dk = dk; a.dv = dv;
+    a.otilde = want_otilde ? otilde : nullptr;
     char* base = static_cast<char*>(ws);
     a.hdr = reinterpret_cast<ent::WsHeader*>(base);
     a.delta = reinterpret_cast<float*>(base + L.delta);
@@ -197,6 +209,44 @@ ent_status ent_attn_bwd(const void* q, const void* k, const void* v, const void*
     }
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return ENT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ent_status ent_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                        int dtype, float alpha, int causal, void* o, float* tau,
+                        uint8_t* block_mask, uint8_t* iters, void* ws, size_t ws_bytes,
+                        void* stream) {
+    return fwd_impl(q, k, v, B, H, N, d, dtype, alpha, causal, o, tau, block_mask, iters, nullptr,
+                    false, ws, ws_bytes, stream);
+}
+
+ent_status ent_attn_fwd_otilde(const void* q, const void* k, const void* v, int B, int H, int N,
+                               int d, int dtype, float alpha, int causal, void* o, float* tau,
+                               uint8_t* block_mask, uint8_t* iters, float* otilde, void* ws,
+                               size_t ws_bytes, void* stream) {
+    return fwd_impl(q, k, v, B, H, N, d, dtype, alpha, causal, o, tau, block_mask, iters, otilde,
+                    true, ws, ws_bytes, stream);
+}
+
+ent_status ent_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* tau, const uint8_t* block_mask, int B,
+                        int H, int N, int d, int dtype, float alpha, int causal, void* dq,
+                        void* dk, void* dv, void* ws, size_t ws_bytes, void* stream) {
+    (void)o;
+    return bwd_impl(q, k, v, nullptr, false, dout, tau, block_mask, B, H, N, d, dtype, alpha,
+                    causal, dq, dk, dv, ws, ws_bytes, stream);
+}
+
+ent_status ent_attn_bwd_otilde(const void* q, const void* k, const void* v, const float* otilde,
+                               const void* dout, const float* tau, const uint8_t* block_mask,
+                               int B, int H, int N, int d, int dtype, float alpha, int causal,
+                               void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                               void* stream) {
+    return bwd_impl(q, k, v, otilde, true, dout, tau, block_mask, B, H, N, d, dtype, alpha, causal,
+                    dq, dk, dv, ws, ws_bytes, stream);
 }
 
 int ent_entmax_rows_max_n(void) { return 16384; }
@@ -349,9 +399,10 @@ extern "C" ent_status ent_attn_bwd_noalloc(const void* q, const void* k, const v
     if (e != cudaSuccess) return cuda_fail(e, "clearing the fixed scratch header");
     if (empty) return ENT_OK;
 
-    ent::BwdArgs a;
+    ent::BwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.dout = dout; a.tau = tau; a.mask = block_mask;
     a.dq = dq; a.dk = dk; a.dv = dv;
+    a.otilde = nullptr;
     char* b = static_cast<char*>(base);
     a.hdr = reinterpret_cast<ent::WsHeader*>(b);
     a.delta = reinterpret_cast<float*>(b + kHdr);

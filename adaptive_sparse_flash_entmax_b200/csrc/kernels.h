@@ -23,6 +23,7 @@ struct FwdArgs {
     float ftol, stol;      // solver stop rule: |f| <= ftol, or a step <= stol*max(1,|tau|)
     int hist_budget;       // tensor-core path: histogram inserts a tile may make after its
                            // first block (0: no histogram, < 0: no limit)
+    float* otilde;         // nullable [BH][N][d] fp32: sum_j g_ij v_j / sum_j g_ij
 };
 
 struct BwdArgs {
@@ -35,6 +36,8 @@ struct BwdArgs {
     void* dq;
     void* dk;
     void* dv;
+    const float* otilde;   // nullable: the forward's otilde; then delta_i = dO_i . otilde_i
+                           // and the delta pass over the keys is skipped
     float* delta;          // workspace [BH*N]
     float* dq_acc;         // workspace [BH*N*d] fp32 (tensor-core path)
     int* lists;            // workspace: per-tile / per-block live lists (tensor-core path)

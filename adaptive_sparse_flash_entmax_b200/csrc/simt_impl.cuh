@@ -158,42 +158,57 @@ __global__ void __launch_bounds__(128, 1) simt_fwd_kernel(FwdArgs a) {
     }
     const int npass = pass;   // solver passes after the statistics pass
 
-    // P.V over live blocks.
-    float acc[D];
-#pragma unroll
-    for (int c = 0; c < D; ++c) acc[c] = 0.f;
+    // P.V over live blocks; with otilde a second sweep accumulates G.V and sum_j g
+    // (g = u^(gamma-1)) for otilde = G.V / sum_j g.
     int nlive = 0;
-    for (int b = 0; b < nblk; ++b) {
-        if (!live[b]) continue;   // CTA-uniform (shared flag, written before the last barrier)
-        ++nlive;
-        for (int sb = 0; sb < kBlk / kSub; ++sb) {
-            const int j0 = b * kBlk + sb * kSub;
-            if (j0 >= N || (a.causal && j0 > last_row)) break;
-            __syncthreads();
-            load_rows_f32<TIn, D>(Ks, D, k, j0, kSub, N, tid, 128);
-            load_rows_f32<TIn, D>(Vs, D, v, j0, kSub, N, tid, 128);
-            __syncthreads();
-            float r[kSub];
-            dot_rows<D, kSub>(r, qrow, Ks);
-            const int nv = key_end - j0;
+    const int nsweep = a.otilde ? 2 : 1;
+#pragma unroll 1
+    for (int sweep = 0; sweep < nsweep; ++sweep) {
+        float acc[D];
 #pragma unroll
-            for (int jj = 0; jj < kSub; ++jj) {
-                const float p = (jj < nv) ? entmax_p<GM>(__fmaf_rn(cx, r[jj], -st.tau), gamma) : 0.f;
+        for (int c = 0; c < D; ++c) acc[c] = 0.f;
+        float wsum = 0.f;
+        for (int b = 0; b < nblk; ++b) {
+            if (!live[b]) continue;   // CTA-uniform (shared flag, written before the last barrier)
+            if (sweep == 0) ++nlive;
+            for (int sb = 0; sb < kBlk / kSub; ++sb) {
+                const int j0 = b * kBlk + sb * kSub;
+                if (j0 >= N || (a.causal && j0 > last_row)) break;
+                __syncthreads();
+                load_rows_f32<TIn, D>(Ks, D, k, j0, kSub, N, tid, 128);
+                load_rows_f32<TIn, D>(Vs, D, v, j0, kSub, N, tid, 128);
+                __syncthreads();
+                float r[kSub];
+                dot_rows<D, kSub>(r, qrow, Ks);
+                const int nv = key_end - j0;
 #pragma unroll
-                for (int c = 0; c < D; c += 4) {
-                    const float4 vv = *reinterpret_cast<const float4*>(Vs + jj * D + c);
-                    acc[c] = fmaf(p, vv.x, acc[c]);
-                    acc[c + 1] = fmaf(p, vv.y, acc[c + 1]);
-                    acc[c + 2] = fmaf(p, vv.z, acc[c + 2]);
-                    acc[c + 3] = fmaf(p, vv.w, acc[c + 3]);
+                for (int jj = 0; jj < kSub; ++jj) {
+                    const float u = __fmaf_rn(cx, r[jj], -st.tau);
+                    const float p = (jj >= nv) ? 0.f : (sweep == 0) ? entmax_p<GM>(u, gamma) : entmax_g<GM>(u, gamma);
+                    wsum += p;
+#pragma unroll
+                    for (int c = 0; c < D; c += 4) {
+                        const float4 vv = *reinterpret_cast<const float4*>(Vs + jj * D + c);
+                        acc[c] = fmaf(p, vv.x, acc[c]);
+                        acc[c + 1] = fmaf(p, vv.y, acc[c + 1]);
+                        acc[c + 2] = fmaf(p, vv.z, acc[c + 2]);
+                        acc[c + 3] = fmaf(p, vv.w, acc[c + 3]);
+                    }
                 }
             }
         }
+        if (row_valid && sweep == 0) {
+            TIn* o = static_cast<TIn*>(a.o) + head + (size_t)i * D;
+#pragma unroll
+            for (int c = 0; c < D; ++c) store_f(o, c, acc[c]);
+        } else if (row_valid) {
+            float* ot = a.otilde + head + (size_t)i * D;
+            const float rs = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+            for (int c = 0; c < D; ++c) ot[c] = acc[c] * rs;
+        }
     }
     if (row_valid) {
-        TIn* o = static_cast<TIn*>(a.o) + head + (size_t)i * D;
-#pragma unroll
-        for (int c = 0; c < D; ++c) store_f(o, c, acc[c]);
         a.tau[(size_t)bh * N + i] = st.tau;
         if (a.iters) a.iters[(size_t)bh * N + i] = (unsigned char)st.iters;
     }
@@ -204,6 +219,7 @@ __global__ void __launch_bounds__(128, 1) simt_fwd_kernel(FwdArgs a) {
         atomicAdd(&a.hdr->counters[kCtrPvBlocks], (unsigned long long)nlive);
         atomicAdd(&a.hdr->counters[kCtrPasses], (unsigned long long)npass);
         atomicAdd(&a.hdr->counters[kCtrTiles], 1ull);
+        if (a.otilde) atomicAdd(&a.hdr->counters[kCtrGvBlocks], (unsigned long long)nlive);
     }
 }
 
@@ -246,11 +262,21 @@ __global__ void __launch_bounds__(128, 1) simt_bwd_dq_kernel(BwdArgs a) {
     float acc[D];
 #pragma unroll
     for (int c = 0; c < D; ++c) acc[c] = 0.f;
-    int nvis = 0;
-    for (int phase = 0; phase < 2; ++phase) {
+    int nvis = 0, nphase0 = 0;
+    if (a.otilde) {
+        // delta_i = dO_i . otilde_i (dP = dO V^T), so the delta phase is not needed
+        __syncthreads();   // the dO tile is loaded cooperatively
+        if (row_valid) {
+            const float* ot = a.otilde + head + (size_t)i * D;
+            for (int c = 0; c < D; ++c) delta = fmaf(dorow[c], ot[c], delta);
+            a.delta[(size_t)bh * N + i] = delta;
+        }
+    }
+    for (int phase = a.otilde ? 1 : 0; phase < 2; ++phase) {
         for (int b = 0; b < nblk; ++b) {
             if (!mrow[b]) continue;   // CTA-uniform
             ++nvis;
+            if (phase == 0) ++nphase0;
             for (int sb = 0; sb < kBlk / kSubB; ++sb) {
                 const int j0 = b * kBlk + sb * kSubB;
                 if (j0 >= N || (a.causal && j0 > last_row)) break;
@@ -293,7 +319,8 @@ __global__ void __launch_bounds__(128, 1) simt_bwd_dq_kernel(BwdArgs a) {
         for (int c = 0; c < D; ++c) store_f(dq, c, acc[c] * a.scale);
     }
     // block GEMMs: the delta phase computes S and dP (2), the dQ phase S, dP and dS K (3)
-    if (tid == 0) atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(nvis / 2) * 5);
+    if (tid == 0)
+        atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(2 * nphase0 + 3 * (nvis - nphase0)));
 }
 
 // dV (WHICH = 0) or dK (WHICH = 1) for one 128-key block (thread = key).

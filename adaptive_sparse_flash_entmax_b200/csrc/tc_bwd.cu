@@ -15,7 +15,9 @@
 //   dq kernel   one CTA per 128-row query tile, one live 128-key block per job.
 //               Phase A: S = Q K^T, dP = dO V^T -> delta per row (also written
 //               to the workspace).  Phase B: again S and dP, dS as a pair of
-//               bf16 parts (hi + lo) and dQ += dS K (K read MN-major).
+//               bf16 parts (hi + lo) and dQ += dS K (K read MN-major).  Given
+//               the forward's otilde = sum_j g_ij v_j / sum_j g_ij, delta_i =
+//               dO_i . otilde_i (since dP = dO V^T) and phase A is skipped.
 //   dkv kernel  one CTA per 128-key block, Q/dO in 64-row sub-tiles of the
 //               live query tiles (so that two S^T/dP^T pairs fit in TMEM
 //               beside dV and dK), P^T and dS^T over their own S^T and dP^T
@@ -173,8 +175,11 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
-    const int nA = misc->njobs;      // phase A jobs 0..nA-1, phase B jobs nA..2nA-1, same blocks
-    const int total = 2 * nA;
+    // phase A jobs 0..nA-1 (none when delta comes from otilde), phase B jobs nA..nA+nB-1,
+    // both over the same live blocks
+    const int nB = misc->njobs;
+    const int nA = a.otilde ? 0 : nB;
+    const int total = nA + nB;
     // pair of job j and the number of earlier jobs on that pair
     auto pair_of = [&](int j) { return j < nA ? (j & 1) : 0; };
     auto use_of = [&](int j) { return j < nA ? (j >> 1) : ((nA + 1) >> 1) + (j - nA); };
@@ -257,11 +262,11 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int j = 0; j < nA && ok; ++j) ok = issue_sdp(j);
             // phase B: S and dP of job i go in ahead of dQ of job i-1, so the tensor
             // pipe has work while the elementwise warps turn job i-1 into dS
-            for (int i = 0; i < nA && ok; ++i) {
+            for (int i = 0; i < nB && ok; ++i) {
                 ok = issue_sdp(nA + i);
                 if (ok && i > 0) ok = issue_dq(i - 1);
             }
-            if (ok && nA > 0) ok = issue_dq(nA - 1);
+            if (ok && nB > 0) ok = issue_dq(nB - 1);
             if (ok) umma_commit(acc_full);
             umma_commit(mma_done);
             drain_wait(mma_done, 0);
@@ -325,17 +330,42 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             sg += a0.x + a0.y;
             sgdp += b0.x + b0.y;
         }
+        constexpr int DH = D / 2;
+        float dpart = 0.f;   // with otilde: this half's share of dO_i . otilde_i
+        if (a.otilde && row_valid) {
+            const __nv_bfloat16* dor = static_cast<const __nv_bfloat16*>(a.dout) + ((size_t)bh * N + i) * D + half * DH;
+            const float* otr = a.otilde + ((size_t)bh * N + i) * D + half * DH;
+            float2 acc2 = make_float2(0.f, 0.f);
+#pragma unroll 4
+            for (int c = 0; c < DH; c += 8) {
+                const uint4 g8 = *reinterpret_cast<const uint4*>(dor + c);
+                const float4 o0 = *reinterpret_cast<const float4*>(otr + c);
+                const float4 o1 = *reinterpret_cast<const float4*>(otr + c + 4);
+                const uint32_t w[4] = {g8.x, g8.y, g8.z, g8.w};
+                const float2 ov[4] = {make_float2(o0.x, o0.y), make_float2(o0.z, o0.w),
+                                      make_float2(o1.x, o1.y), make_float2(o1.z, o1.w)};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc2 = __ffma2_rn(__bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e])), ov[e], acc2);
+            }
+            dpart = acc2.x + acc2.y;
+        }
         // every elementwise thread reaches this barrier once, also after an abort
-        xch[(0 * 2 + half) * 128 + row] = sg;
+        xch[(0 * 2 + half) * 128 + row] = a.otilde ? dpart : sg;
         xch[(1 * 2 + half) * 128 + row] = sgdp;
         named_bar(1, kEw);
-        const float SG = sg + xch[(0 * 2 + (half ^ 1)) * 128 + row];
-        const float SGDP = sgdp + xch[(1 * 2 + (half ^ 1)) * 128 + row];
-        const float delta = (SG > 0.f) ? SGDP / SG : 0.f;
+        float delta;
+        if (a.otilde) {
+            delta = dpart + xch[(0 * 2 + (half ^ 1)) * 128 + row];
+        } else {
+            const float SG = sg + xch[(0 * 2 + (half ^ 1)) * 128 + row];
+            const float SGDP = sgdp + xch[(1 * 2 + (half ^ 1)) * 128 + row];
+            delta = (SG > 0.f) ? SGDP / SG : 0.f;
+        }
         if (row_valid && half == 0) a.delta[(size_t)bh * N + i] = delta;
         // phase B: dS = g (dP - delta) as bf16 hi + lo into TMEM
         const float2 nd2 = make_float2(-delta, -delta), m1 = make_float2(-1.f, -1.f);
-        for (int ib = 0; ib < nA && ok; ++ib) {
+        for (int ib = 0; ib < nB && ok; ++ib) {
             const int j = nA + ib;
             if (!(ok = mbar_wait(&s_full[0], use_of(j) & 1, ab, 26))) break;
             tc_fence_after();
@@ -363,9 +393,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(ds_full);
         }
-        constexpr int DH = D / 2;
         float acc[DH];
-        if (ok && nA > 0) {
+        if (ok && nB > 0) {
             ok = mbar_wait(acc_full, 0, ab, 28);
             tc_fence_after();
             const uint32_t ob = lane0 + 256 + half * DH;
@@ -379,7 +408,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         if (row_valid) store_out_row(a.dq, ((size_t)bh * N + i) * D + half * DH, acc, DH, a.scale);
         if (threadIdx.x == 64)   // block products: phase A S, dP (2) + phase B S, dP, dQ hi, lo (4)
-            atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(6 * nA));
+            atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(2 * nA + 4 * nB));
     }
 
     tc_fence_before();

@@ -43,13 +43,15 @@ namespace {
 
 constexpr int kSlots = 4;          // single tile slots of the P.V pass (K or V blocks)
 constexpr int kDSlots = 2;         // double slots of the score passes (two K blocks), same memory
-constexpr int kSbuf = 3;           // 128-column S accumulators in TMEM (P.V pass)
+constexpr int kSbuf = 3;           // 128-column S accumulators in TMEM (P.V pass; two when
+                                   // the G.V accumulator of a d = 128 forward takes the third)
 constexpr int kThreads = 320;      // 10 warps
 constexpr int kEw = 256;           // elementwise threads (warps 2-9): two per query row
 constexpr int kEwWarps = 8;
 constexpr int kAtom = 128 * 128;   // bytes of a [128 rows x 64 bf16] swizzled atom
 constexpr int kTmemCols = 512;     // score passes: S [0,256), [256,512); P.V pass: S0 [0,128),
-                                   // S1 [128,256), O [256, 256+D), S2 [384, 512)
+                                   // S1 [128,256), O [256, 256+D), then either S2 [384, 512)
+                                   // or, with otilde, G.V [256+D, 256+2D) (and S2 when D = 64)
 constexpr int kDecSolve = 1, kDecPv = 2;
 // Largest upward Halley step taken without a verifying pass, relative to max(1,|tau|).
 constexpr float kAcceptStep = 5e-4f;
@@ -97,7 +99,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 
 }  // namespace
 
-template <int D, int GM>
+// OT: also accumulate G.V (g = u^(gamma-1) as bf16 beside P in TMEM) and write
+// otilde = G.V / sum_j g, from which the backward takes delta without a pass over the keys.
+template <int D, int GM, bool OT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
@@ -132,6 +136,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int bh = blockIdx.y;
     const int nblk = a.causal ? t + 1 : T;
     const Abort ab{&misc->abort, a.hdr};
+    constexpr int SB = (OT && D == 128) ? 2 : kSbuf;   // S buffers of the P.V pass
+    constexpr uint32_t kOtCol = 256 + D;                // G.V accumulator (OT)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSlots; ++s) { mbar_init(&kfull[s], 1); mbar_init(&kempty[s], 1); }
@@ -291,20 +297,20 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const int job = 0, sj = 0;
                 for (int i = 0; i <= njobs && ok; ++i) {
                     if (i < njobs) {
-                        const int jb = job + i, sb = jb % kSbuf;
+                        const int jb = job + i, sb = jb % SB;
                         if (!(ok = wait_tile(sj + 2 * i))) break;
-                        ok = (i < kSbuf) ? mbar_wait(&s_empty[sb], ((jb / kSbuf) & 1) ^ 1, ab, 5)
-                                         : mbar_wait(&pv_sfree[sb], ((i / kSbuf) - 1) & 1, ab, 5);
+                        ok = (i < SB) ? mbar_wait(&s_empty[sb], ((jb / SB) & 1) ^ 1, ab, 5)
+                                      : mbar_wait(&pv_sfree[sb], ((i / SB) - 1) & 1, ab, 5);
                         if (!ok) break;
                         tc_fence_after();
                         issue_s(sb, sj + 2 * i);
                     }
                     if (i > 0) {
-                        const int ip = i - 1, sb = (job + ip) % kSbuf, tv = sj + 2 * ip + 1;
+                        const int ip = i - 1, sb = (job + ip) % SB, tv = sj + 2 * ip + 1;
                         if (!(ok = wait_tile(tv))) break;
-                        // one p_full per buffer: P(i+3) cannot complete before P.V(i) frees
+                        // one p_full per buffer: P(i+SB) cannot complete before P.V(i) frees
                         // the buffer, so the elementwise warps never lap this wait
-                        if (!(ok = mbar_wait(&p_full[sb], (ip / kSbuf) & 1, ab, 6))) break;
+                        if (!(ok = mbar_wait(&p_full[sb], (ip / SB) & 1, ab, 6))) break;
                         tc_fence_after();
                         const uint64_t dv = dring_mn + ((uint32_t)((tv % kSlots) * L::kTile) >> 4);
                         const uint32_t ap = tmem + sbuf_col(sb);
@@ -315,6 +321,15 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
                             umma_bf16_ts(tmem + 256, ap + acol, dv + ((kk * 16 * 128) >> 4), idesc_pv,
                                          (ip > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        if constexpr (OT) {
+                            // G (bf16 pairs) sits in the 32 columns after each half's P
+#pragma unroll
+                            for (int kk = 0; kk < kBlk / 16; ++kk) {
+                                const uint32_t acol = (kk >> 2) * 64 + 32 + (kk & 3) * 8;
+                                umma_bf16_ts(tmem + kOtCol, ap + acol, dv + ((kk * 16 * 128) >> 4),
+                                             idesc_pv, (ip > 0 || kk > 0) ? 1u : 0u);
+                            }
                         }
                         umma_commit(&pv_sfree[sb]);
                         umma_commit(&kempty[tv % kSlots]);
@@ -579,13 +594,14 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (all) break;
         }
         const int npass = pass;
+        [[maybe_unused]] float2 sg2 = make_float2(0.f, 0.f);   // sum_j g of this half-row (OT)
         if (ok) {
             named_bar(1, kEw);   // job_list / njobs of the P.V pass visible to the group
             nlive = misc->njobs;
             for (int li = 0; li < nlive; ++li) {
                 const int b = job_list[li];
-                const int sb = li % kSbuf;   // the P.V pass counts its own jobs
-                if (!(ok = mbar_wait(&s_full[sb], (li / kSbuf) & 1, ab, 9))) break;
+                const int sb = li % SB;   // the P.V pass counts its own jobs
+                if (!(ok = mbar_wait(&s_full[sb], (li / SB) & 1, ab, 9))) break;
                 tc_fence_after();
                 float s[64];
                 tmem_ld32(lane_base + sbuf_col(sb) + c0, &s[0]);
@@ -598,15 +614,31 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int c = 0; c < 64; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
                 }
                 uint32_t pk[32];
+                [[maybe_unused]] uint32_t gk[32];
                 const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-sv.tau, -sv.tau);
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
-                    const float2 p2 = entmax_p_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma);
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(p2.x, p2.y);
-                    pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+                    const float2 u2 = __ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2);
+                    if constexpr (OT) {
+                        float2 p2, g2;
+                        entmax_pg_x2<GM>(u2, gamma, p2, g2);
+                        const __nv_bfloat162 hp = __floats2bfloat162_rn(p2.x, p2.y);
+                        const __nv_bfloat162 hg = __floats2bfloat162_rn(g2.x, g2.y);
+                        pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
+                        gk[c >> 1] = *reinterpret_cast<const uint32_t*>(&hg);
+                        // sum the rounded weights the G.V product uses: otilde is then
+                        // a weighted mean whose weights sum to one
+                        sg2 = __fadd2_rn(sg2, __bfloat1622float2(hg));
+                    } else {
+                        const float2 p2 = entmax_p_x2<GM>(u2, gamma);
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p2.x, p2.y);
+                        pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+                    }
                 }
                 // P over this thread's own S columns: keys c0 .. c0+63 -> columns c0 .. c0+31
+                // (and G, with otilde, -> columns c0+32 .. c0+63)
                 tmem_st32(lane_base + sbuf_col(sb) + c0, pk);
+                if constexpr (OT) tmem_st32(lane_base + sbuf_col(sb) + c0 + 32, gk);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -645,6 +677,31 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (a.iters) a.iters[(size_t)bh * N + i] = (uint8_t)sv.iters;
             }
         }
+        if constexpr (OT) {
+            // otilde = G.V / sum_j g; the halves' sums meet in shared memory (every
+            // elementwise thread reaches this barrier once, also after an abort)
+            X(0, half) = sg2.x + sg2.y;
+            named_bar(1, kEw);
+            const float sg = X(0, 0) + X(0, 1);
+            if (ok && nlive > 0) {
+#pragma unroll
+                for (int c = 0; c < DH / 32; ++c)
+                    tmem_ld32(lane_base + kOtCol + half * DH + c * 32, &o[c * 32]);
+                tmem_wait_ld();
+                reg_fence<DH>(o);
+            } else {
+#pragma unroll
+                for (int c = 0; c < DH; ++c) o[c] = 0.f;
+            }
+            const float rs = sg > 0.f ? 1.f / sg : 0.f;
+            if (row_valid) {
+                float* orow = a.otilde + ((size_t)bh * N + i) * D + half * DH;
+#pragma unroll
+                for (int c = 0; c < DH; c += 4)
+                    *reinterpret_cast<float4*>(orow + c) =
+                        make_float4(o[c] * rs, o[c + 1] * rs, o[c + 2] * rs, o[c + 3] * rs);
+            }
+        }
         uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
         for (int bb = ew; bb < T; bb += kEw) mrow[bb] = (bb < nblk) ? live[bb] : 0;
         if (ew == 0) {
@@ -652,6 +709,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             atomicAdd(&a.hdr->counters[kCtrPvBlocks], (unsigned long long)nlive);
             atomicAdd(&a.hdr->counters[kCtrPasses], (unsigned long long)npass);
             atomicAdd(&a.hdr->counters[kCtrTiles], 1ull);
+            if (OT) atomicAdd(&a.hdr->counters[kCtrGvBlocks], (unsigned long long)nlive);
         }
     }
 
@@ -704,7 +762,7 @@ template <int D, int GM>
 static cudaError_t launch_tc_fwd(const CUtensorMap& mq, const CUtensorMap& mk,
                                  const CUtensorMap& mv, const FwdArgs& a, cudaStream_t s) {
     const size_t sm = Layout<D>::bytes(a.T);
-    auto kern = tc_fwd_kernel<D, GM>;
+    auto kern = a.otilde ? tc_fwd_kernel<D, GM, true> : tc_fwd_kernel<D, GM, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(mq, mk, mv, a);

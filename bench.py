@@ -50,6 +50,9 @@ def parse():
     p.add_argument("--hist-budget", type=int, default=None,
                    help="ablation: histogram insert budget per forward tile (0: no histogram, "
                         "i.e. every row from the plain bracket; -1: no limit)")
+    p.add_argument("--delta", choices=["otilde", "recompute"], default="otilde",
+                   help="backward delta: from the forward's otilde (ent_attn_fwd_otilde + "
+                        "ent_attn_bwd_otilde) or recomputed by a pass over the keys")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--B", type=int, default=None, help="override the batch (profiling cases)")
     p.add_argument("--H", type=int, default=None, help="override the head count")
@@ -368,23 +371,27 @@ def run_ours(args):
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
     wsf = A.workspace(capi.ent_attn_fwd_workspace_size(B, H, N, d, dt_code), dev)
     wsb = A.workspace(capi.ent_attn_bwd_workspace_size(B, H, N, d, dt_code), dev)
+    # otilde = G V / sum g (float32, like q) when the backward takes delta from it
+    ot = torch.empty(qd.shape, dtype=torch.float32, device=dev) if args.delta == "otilde" else None
 
     def step():
-        A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, None))
+        A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, None),
+                          otilde=ot)
         A.entmax_attn_bwd(qd, kd, vd, o, dod, tau, mask, w.alpha, w.causal, ws=wsb,
-                          out=(dq, dk, dv))
+                          out=(dq, dk, dv), otilde=ot)
 
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
     # counters, sparsity and solver passes of one step (untimed)
     it = torch.empty((B, H, N), dtype=torch.uint8, device=dev)
-    A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, it))
+    A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, it), otilde=ot)
     cf = A.read_status(wsf)
-    A.entmax_attn_bwd(qd, kd, vd, o, dod, tau, mask, w.alpha, w.causal, ws=wsb, out=(dq, dk, dv))
+    A.entmax_attn_bwd(qd, kd, vd, o, dod, tau, mask, w.alpha, w.causal, ws=wsb, out=(dq, dk, dv),
+                      otilde=ot)
     cb = A.read_status(wsb)
     blk = 2.0 * 128 * 128 * d
-    fwd_flops = blk * (cf[0] + 2 * cf[1])
+    fwd_flops = blk * (cf[0] + 2 * cf[1] + cf[5])
     bwd_flops = blk * cb[4]
     exec_flops = fwd_flops + bwd_flops
     admissible = B * H * (T * (T + 1) // 2 if w.causal else T * T)
@@ -403,10 +410,11 @@ def run_ours(args):
         t_start.record(stream)
         for s in range(args.steps):
             ev[s][0].record(stream)
-            A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, None))
+            A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, None),
+                              otilde=ot)
             ev[s][1].record(stream)
             A.entmax_attn_bwd(qd, kd, vd, o, dod, tau, mask, w.alpha, w.causal, ws=wsb,
-                              out=(dq, dk, dv))
+                              out=(dq, dk, dv), otilde=ot)
             ev[s][2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -450,8 +458,9 @@ def run_ours(args):
                     s_cmp.wait_event(done_out[i - 2])  # outputs of this buffer set copied out
                 qq, kk, vv, dd = din[bset]
                 oo, tt, mm, g1, g2, g3 = dout[bset]
-                A.entmax_attn_fwd(qq, kk, vv, w.alpha, w.causal, ws=wsf, out=(oo, tt, mm, None))
-                A.entmax_attn_bwd(qq, kk, vv, oo, dd, tt, mm, w.alpha, w.causal, ws=wsb,
+                A.entmax_attn_fwd(qq, kk, vv, w.alpha, w.causal, ws=wsf, out=(oo, tt, mm, None),
+                                  otilde=ot)
+                A.entmax_attn_bwd(qq, kk, vv, oo, dd, tt, mm, w.alpha, w.causal, ws=wsb, otilde=ot,
                                   out=(g1, g2, g3))
                 done_cmp.append(torch.cuda.Event())
                 done_cmp[-1].record(s_cmp)
@@ -524,7 +533,9 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32" if w.dtype == "f32" else "bf16 inputs, f32 accumulate",
             "data": "synthetic",
-            "config": config_of(w, world),
+            "config": config_of(w, world, {"delta": (
+                "from the forward's otilde = G V / sum g (ent_attn_fwd_otilde, ent_attn_bwd_otilde)"
+                if ot is not None else "recomputed by a pass over the live keys")}),
             "ms_fwd": ms_fwd, "ms_bwd": ms_bwd,
             "executed_tflop_per_step": flops_all / 1e12,
             "effective_dense_tflops": world * dense_flops(w) / (ms_step * 1e-3) / 1e12,

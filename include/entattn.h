@@ -113,6 +113,37 @@ ent_status ent_attn_bwd(const void *q, const void *k, const void *v, const void 
                         void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Forward that also returns otilde, float32 [B,H,N,d] (caller-owned, 16-byte
+ * aligned): the g-weighted mean of the value rows at the returned tau,
+ *     otilde_i = sum_j g_ij v_j / sum_j g_ij,   g = (x - tau)_+^(1/(alpha-1) - 1).
+ * Everything else is ent_attn_fwd's (same outputs, same workspace size).  The
+ * backward's delta_i = sum_j g_ij dP_ij / sum_j g_ij equals dO_i . otilde_i
+ * because dP = dO V^T (derived from the definition), so ent_attn_bwd_otilde
+ * needs no delta pass over the keys.  The P.V pass then also accumulates G V
+ * (one more 128x128xd block product per live block, counter [5]); on the
+ * bf16 path g is rounded to bf16 for that product, as P is.  A null otilde is
+ * ENT_EINVAL.
+ */
+ent_status ent_attn_fwd_otilde(const void *q, const void *k, const void *v,
+                               int B, int H, int N, int d, int dtype,
+                               float alpha, int causal,
+                               void *o, float *tau, uint8_t *block_mask, uint8_t *iters,
+                               float *otilde, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Backward given otilde from ent_attn_fwd_otilde of the same q, k, v (with
+ * the tau and block_mask of that call): delta_i = dO_i . otilde_i, then dq,
+ * dk, dv exactly as ent_attn_bwd computes them, without the delta pass (two
+ * block products per live block fewer).  Same workspace size as
+ * ent_attn_bwd.  A null otilde is ENT_EINVAL.
+ */
+ent_status ent_attn_bwd_otilde(const void *q, const void *k, const void *v, const float *otilde,
+                               const void *dout, const float *tau, const uint8_t *block_mask,
+                               int B, int H, int N, int d, int dtype, float alpha, int causal,
+                               void *dq, void *dk, void *dv,
+                               void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Backward without a workspace argument.  The pages have no counterpart: this
  * is a library convenience.  It computes exactly what ent_attn_bwd computes
  * (same kernels, same arguments minus ws / ws_bytes) for callers that cannot
@@ -150,8 +181,9 @@ ent_status ent_attn_bwd_noalloc(const void *q, const void *k, const void *v, con
  *   [2] solver passes summed over query tiles,
  *   [3] query tiles processed,
  *   [4] block products issued by the backward kernels (all of them),
- *   [5]..[7] reserved (0).
- * Executed flops of a call = 2*128*128*d * ([0] + 2*[1] + [4]).
+ *   [5] G.V block products of ent_attn_fwd_otilde (one per live block),
+ *   [6]..[7] reserved (0).
+ * Executed flops of a call = 2*128*128*d * ([0] + 2*[1] + [4] + [5]).
  * Returns ENT_OK, ENT_ETIMEOUT if a bounded wait gave up, ENT_ECUDA on a
  * CUDA error.
  */

@@ -50,9 +50,10 @@ def parse():
     p.add_argument("--hist-budget", type=int, default=None,
                    help="ablation: histogram insert budget per forward tile (0: no histogram, "
                         "i.e. every row from the plain bracket; -1: no limit)")
-    p.add_argument("--delta", choices=["otilde", "recompute"], default="otilde",
+    p.add_argument("--delta", choices=["auto", "otilde", "recompute"], default="auto",
                    help="backward delta: from the forward's otilde (ent_attn_fwd_otilde + "
-                        "ent_attn_bwd_otilde) or recomputed by a pass over the keys")
+                        "ent_attn_bwd_otilde), recomputed by a pass over the keys, or auto: "
+                        "otilde unless an untimed forward finds >= 50%% of the blocks empty")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--B", type=int, default=None, help="override the batch (profiling cases)")
     p.add_argument("--H", type=int, default=None, help="override the head count")
@@ -180,10 +181,10 @@ def measured_peaks():
                 "sm_max_mhz": 1965.0}, "fallback"
 
 
-def profiled_traffic(w, kernel):
-    """DRAM bytes per launch of `kernel` on this workload from the committed ncu
-    summary (profiles/traffic.json), or None when the kernel source changed since
-    the capture (the summary stores a hash of the source file)."""
+def profiled_traffic(w, kernel, variant="plain"):
+    """DRAM bytes per launch of `kernel` (variant "plain" or "otilde") on this workload
+    from the committed ncu summary (profiles/traffic.json), or None when the kernel
+    source changed since the capture (the summary stores a hash of the source file)."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
@@ -192,6 +193,8 @@ def profiled_traffic(w, kernel):
         return None
     for r in rec.get("captures", []):
         if r.get("kernel") != kernel or r.get("workload") != w.name:
+            continue
+        if r.get("variant", "plain") != variant:
             continue
         if any(r.get(k) != getattr(w, k) for k in ("B", "H", "N", "d", "alpha", "beta")):
             continue
@@ -371,8 +374,19 @@ def run_ours(args):
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
     wsf = A.workspace(capi.ent_attn_fwd_workspace_size(B, H, N, d, dt_code), dev)
     wsb = A.workspace(capi.ent_attn_bwd_workspace_size(B, H, N, d, dt_code), dev)
+    admissible = B * H * (T * (T + 1) // 2 if w.causal else T * T)
+    delta_mode, delta_why = args.delta, "requested"
+    if delta_mode == "auto":
+        # Measured on B200: delta from otilde makes the dense-block workloads 2-4 % faster
+        # per step (the backward drops S and dP of every live block, the forward adds one
+        # G V product per live block); at 95 % block sparsity the saving no longer pays
+        # for the forward's extra work.  One untimed forward measures the sparsity.
+        A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, None))
+        sp0 = 1.0 - int(mask.sum().item()) / admissible
+        delta_mode = "otilde" if sp0 < 0.5 else "recompute"
+        delta_why = f"auto: block sparsity {sp0:.3f} of an untimed forward (otilde below 0.5)"
     # otilde = G V / sum g (float32, like q) when the backward takes delta from it
-    ot = torch.empty(qd.shape, dtype=torch.float32, device=dev) if args.delta == "otilde" else None
+    ot = torch.empty(qd.shape, dtype=torch.float32, device=dev) if delta_mode == "otilde" else None
 
     def step():
         A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=wsf, out=(o, tau, mask, None),
@@ -394,7 +408,6 @@ def run_ours(args):
     fwd_flops = blk * (cf[0] + 2 * cf[1] + cf[5])
     bwd_flops = blk * cb[4]
     exec_flops = fwd_flops + bwd_flops
-    admissible = B * H * (T * (T + 1) // 2 if w.causal else T * T)
     live = int(mask.sum().item())
     iters = it.float()
     pass_hist = torch.bincount(it.reshape(-1).long(), minlength=1).tolist()
@@ -499,7 +512,8 @@ def run_ours(args):
     if w.dtype == "bf16":
         # tcgen05 forward: executed MMA flops against the sustained bf16 tensor peak
         # (the kernel is timed inside a long step)
-        roof = {"kernel": "tc_fwd_kernel: statistics + solver + P.V passes (tcgen05/TMEM/TMA)",
+        roof = {"kernel": "tc_fwd_kernel: statistics + solver + P.V passes (tcgen05/TMEM/TMA)"
+                          + ("; G.V for otilde" if ot is not None else ""),
                 "bound": "tensor", "achieved": fwd_tflops,
                 "peak": peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]),
                 "unit": "TFLOP/s",
@@ -512,7 +526,8 @@ def run_ours(args):
                 "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x %.0f MHz" % sm_max}
         launches = 4    # forward + three backward kernels
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = profiled_traffic(w, roof["kernel"].split(":")[0])
+    roof["traffic"] = profiled_traffic(w, roof["kernel"].split(":")[0],
+                                       "otilde" if ot is not None else "plain")
     value = flops_all / (ms_step * 1e-3) / 1e12
     line = None
     if rank == 0:
@@ -535,7 +550,7 @@ def run_ours(args):
             "data": "synthetic",
             "config": config_of(w, world, {"delta": (
                 "from the forward's otilde = G V / sum g (ent_attn_fwd_otilde, ent_attn_bwd_otilde)"
-                if ot is not None else "recomputed by a pass over the live keys")}),
+                if ot is not None else "recomputed by a pass over the live keys") + f" [{delta_why}]"}),
             "ms_fwd": ms_fwd, "ms_bwd": ms_bwd,
             "executed_tflop_per_step": flops_all / 1e12,
             "effective_dense_tflops": world * dense_flops(w) / (ms_step * 1e-3) / 1e12,

@@ -99,12 +99,13 @@ struct RowSolver {
 // within the closed bracket [lo, hi] (a point that rounding put a few ulps
 // outside is clamped onto it: a root on a bracket end, such as tau = m - 1 for
 // a one-element support, must stay reachable); otherwise the bracket is bisected.
-// `accept` > 0 also stops on an upward Halley step of at most accept*max(1,|tau|),
-// taking the new point without evaluating it: the root is then within the step of
-// it (Halley's error is cubic in the step between support changes), and since tau
-// only grew the support only shrank, so the live blocks marked in this pass still
-// cover every block with p > 0 (a block marked live whose elements all lie in
-// (tau_old, tau_new] has max(x - tau) > -accept*max(1,|tau|)).
+// `accept` > 0 also stops on an upward Halley step of at most `accept` (absolute, in
+// x units), taking the new point without evaluating it: the root is then within the
+// step of it (Halley's error is cubic in the step between support changes), and since
+// tau only grew the support only shrank, so the live blocks marked in this pass still
+// cover every block with p > 0.  A block marked live whose elements all lie in
+// (tau_old, tau_new] has max(x - tau) > -accept, so with accept below the 1e-3 band of
+// the mask contract the mask stays exact outside that band at any |tau|.
 __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1, float F2,
                                               float gamma, bool gamma_is_one, int pass,
                                               float ftol, float stol, float accept = 0.f) {
@@ -120,7 +121,7 @@ __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1,
     const bool halley = isfinite(h) && h >= st.lo - tol && h <= st.hi + tol;
     const float next = halley ? fminf(fmaxf(h, st.lo), st.hi) : 0.5f * (st.lo + st.hi);
     if (fabsf(next - st.tau) <= tol) { st.done = 1; st.iters = pass; return; }
-    if (halley && next > st.tau && next - st.tau <= accept * scale) {
+    if (halley && next > st.tau && next - st.tau <= accept) {
         st.tau = next; st.done = 1; st.iters = pass; return;
     }
     st.tau = next;

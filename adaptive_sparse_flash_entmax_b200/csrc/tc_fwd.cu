@@ -53,7 +53,8 @@ constexpr int kTmemCols = 512;     // score passes: S [0,256), [256,512); P.V pa
                                    // S1 [128,256), O [256, 256+D), then either S2 [384, 512)
                                    // or, with otilde, G.V [256+D, 256+2D) (and S2 when D = 64)
 constexpr int kDecSolve = 1, kDecPv = 2;
-// Largest upward Halley step taken without a verifying pass, relative to max(1,|tau|).
+// Largest upward Halley step taken without a verifying pass (x units; below the 1e-3
+// band within which the block mask may differ from the exact one).
 constexpr float kAcceptStep = 5e-4f;
 
 __host__ __device__ constexpr uint32_t sbuf_col(int sb) { return sb < 2 ? sb * 128 : 384; }

@@ -184,8 +184,7 @@ def measured_peaks():
 def profiled_traffic(w, kernel, variant="plain"):
     """DRAM bytes per launch of `kernel` (variant "plain" or "otilde") on this workload
     from the committed ncu summary (profiles/traffic.json), or None when the kernel
-    source changed since the capture (the summary stores a hash of the source file)."""
-    import hashlib
+    source changed since the capture (the summary stores a hash of its source files)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)
@@ -198,14 +197,23 @@ def profiled_traffic(w, kernel, variant="plain"):
             continue
         if any(r.get(k) != getattr(w, k) for k in ("B", "H", "N", "d", "alpha", "beta")):
             continue
-        src = os.path.join(ROOT, r["source"])
-        try:
-            digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
-        except OSError:
-            return None
-        if digest == r.get("sha256"):
+        if sources_digest(r.get("sources") or [r["source"]]) == r.get("sha256"):
             return r["dram_bytes_per_launch"]
     return None
+
+
+def sources_digest(paths):
+    """sha256 over the bytes of the given repository files, in order (None if one is
+    missing): the kernel file and the headers it includes."""
+    import hashlib
+    h = hashlib.sha256()
+    for rel in paths:
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        except OSError:
+            return None
+    return h.hexdigest()
 
 
 # --------------------------------------------------------------------- oracle
@@ -251,6 +259,29 @@ def run_reference(args):
 
 # --------------------------------------------------------------------- ours
 NOMINAL_BF16_TFLOPS = 2250.0   # dense bf16 tensor peak, nominal
+
+
+def element_density(q, k, tau, alpha, causal, heads=2, chunk=512):
+    """Fraction of admissible (query, key) pairs with p > 0 over the first `heads` heads
+    (scores recomputed in float32 with torch from the same inputs; measurement only)."""
+    import torch
+    B, H, N, d = q.shape
+    cx = (alpha - 1.0) / d ** 0.5
+    cols = torch.arange(N, device=q.device)
+    nnz = adm = 0
+    for bh in range(min(heads, B * H)):
+        b, h = divmod(bh, H)
+        K = k[b, h].float()
+        for r0 in range(0, N, chunk):
+            r1 = min(N, r0 + chunk)
+            rows = torch.arange(r0, r1, device=q.device)
+            x = cx * (q[b, h, r0:r1].float() @ K.T)
+            live = x > tau[b, h, r0:r1, None]
+            if causal:
+                live &= cols[None, :] <= rows[:, None]
+            nnz += int(live.sum().item())
+            adm += int(((rows + 1).sum().item()) if causal else (r1 - r0) * N)
+    return nnz / adm
 
 
 def time_dense_comparator(q, k, v, do, causal, steps):
@@ -409,6 +440,7 @@ def run_ours(args):
     bwd_flops = blk * cb[4]
     exec_flops = fwd_flops + bwd_flops
     live = int(mask.sum().item())
+    density = element_density(qd, kd, tau, w.alpha, w.causal)
     iters = it.float()
     pass_hist = torch.bincount(it.reshape(-1).long(), minlength=1).tolist()
 
@@ -557,6 +589,8 @@ def run_ours(args):
             "pct_bf16_peak_executed": 100 * value / world / peaks["bf16_tflops"],
             "pct_bf16_nominal_executed": 100 * value / world / NOMINAL_BF16_TFLOPS,
             "block_sparsity": 1.0 - live / admissible,
+            "element_density": {"value": density,
+                                "what": "fraction of admissible pairs with p > 0, first 2 heads"},
             "tau_passes": {"row_mean": iters.mean().item(), "row_max": int(iters.max().item()),
                            "tile_mean": cf[2] / max(1, cf[3]),
                            "row_histogram": {str(k): c for k, c in enumerate(pass_hist) if c}},

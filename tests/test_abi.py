@@ -2,6 +2,8 @@
 symbol the header declares, and rejects bad arguments before touching CUDA."""
 import ctypes
 import os
+import shutil
+import subprocess
 
 import pytest
 
@@ -90,3 +92,40 @@ def test_missing_library_fails_loudly(tmp_path):
             capi.load(str(tmp_path / "libentattn.so"))
     finally:
         capi._lib = saved
+
+
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    """include/entattn.h is plain C99: a C program using every entry point compiles,
+    links against libentattn.so and gets the argument errors without a GPU."""
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(capi.LIB_PATH)
+    exe = tmp_path / "abi_from_c"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic",
+                    "-I", os.path.join(root, "include"),
+                    os.path.join(root, "tests", "c", "abi_from_c.c"),
+                    "-L", libdir, "-lentattn", "-Wl,-rpath," + libdir, "-o", str(exe)],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert "abi from C ok" in r.stdout
+
+
+@pytest.mark.parametrize("which", ["fwd", "bwd"])
+def test_otilde_argument_errors(lib, which):
+    if which == "fwd":
+        args = dict(q=FAKE, k=FAKE, v=FAKE, B=1, H=1, N=128, d=64, dtype=capi.ENT_BF16,
+                    alpha=1.5, causal=1, o=FAKE, tau=FAKE, block_mask=FAKE, iters=None,
+                    otilde=None, ws=FAKE, ws_bytes=256, stream=None)
+        call = capi.ent_attn_fwd_otilde
+    else:
+        args = dict(q=FAKE, k=FAKE, v=FAKE, otilde=None, dout=FAKE, tau=FAKE, block_mask=FAKE,
+                    B=1, H=1, N=128, d=64, dtype=capi.ENT_BF16, alpha=1.5, causal=1, dq=FAKE,
+                    dk=FAKE, dv=FAKE, ws=FAKE, ws_bytes=1 << 30, stream=None)
+        call = capi.ent_attn_bwd_otilde
+    assert call(**args) == capi.ENT_EINVAL                 # null otilde
+    assert "otilde" in capi.ent_attn_last_error()
+    assert call(**dict(args, otilde=FAKE + 4)) == capi.ENT_EINVAL   # misaligned
+    assert call(**dict(args, d=32, otilde=FAKE)) == capi.ENT_EUNSUPPORTED

@@ -79,9 +79,15 @@ size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype);
  * Forward.  Inputs q, k, v [B,H,N,d].  Outputs: o [B,H,N,d] (same dtype),
  * tau float [B,H,N], block_mask uint8 [B,H,T,T] (all required) and iters
  * uint8 [B,H,N] (nullable): the number of tau-solver passes each row took
- * after the histogram pass.  Per 128-row query tile the kernel runs one
- * statistics pass (row max and score histogram), solver passes until every
- * row of the tile has converged, and one P.V pass over the live key blocks.
+ * after the statistics pass.  Per 128-row query tile the kernel runs one
+ * statistics pass (row max, per-block maxima, and the score histogram when
+ * the histogram start is selected), solver passes until every row of the
+ * tile has converged, and one P.V pass over the live key blocks.  A row stops
+ * when |f(tau)| <= 1e-5 (bf16; 1e-6 float32), when its next step is below
+ * 1e-6 (4e-7) * max(1, |tau|), or after 24 passes; the bf16 path also stops on
+ * an upward Halley step of at most 5e-4, taking that step unverified (the
+ * support only shrinks, so the block mask still covers every p > 0 and may
+ * differ from the exact one only on blocks with max(x - tau) > -5e-4).
  * bf16 inputs start every row's solver from the plain bracket [m-1, m - n^(1-alpha)]
  * (measured faster on B200 than the histogram start, whose inserts cost more than
  * the passes they save).  The environment variable ENTATTN_HIST_BUDGET, read at each

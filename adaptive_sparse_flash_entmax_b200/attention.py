@@ -123,9 +123,11 @@ def read_status(ws: torch.Tensor) -> list[int]:
 class EntmaxAttention(torch.autograd.Function):
     """Autograd wrapper: O = entmax_alpha(Q K^T / sqrt(d)) V.
 
-    With ``delta="otilde"`` the forward also returns otilde (float32, shaped like q) and
-    saves it, and the backward takes delta = dO . otilde instead of a delta pass over the
-    keys; ``delta="recompute"`` saves nothing extra and recomputes delta from the scores."""
+    With ``delta="otilde"`` the forward also computes otilde (float32, shaped like q:
+    B*H*N*d*4 bytes kept for the backward) and the backward takes delta = dO . otilde
+    instead of a delta pass over the keys (faster where most blocks are live);
+    ``delta="recompute"`` keeps nothing extra and recomputes delta from the scores
+    (faster at high block sparsity, and the choice when activation memory is tight)."""
 
     @staticmethod
     def forward(ctx, q, k, v, alpha, causal, delta):

@@ -17,6 +17,11 @@ def _stream_handle(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+# The library launches on the calling thread's current CUDA device; every call below
+# runs with the tensors' device made current, so tensors on another GPU than the
+# current one are handled on theirs.
+
+
 def _check(*ts):
     t0 = ts[0]
     if t0.dim() != 4:
@@ -67,11 +72,13 @@ def entmax_attn_fwd(q, k, v, alpha: float = 1.5, causal: bool = False, *, with_i
             tau.data_ptr(), mask.data_ptr(), iters.data_ptr() if iters is not None else None)
     tail = (ws.data_ptr(), ws.numel(), _stream_handle(q.device))
     if otilde is None:
-        st = capi.ent_attn_fwd(*args, *tail)
+        with torch.cuda.device(q.device):
+            st = capi.ent_attn_fwd(*args, *tail)
         _raise(st, "ent_attn_fwd")
     else:
         _check_otilde(otilde, q)
-        st = capi.ent_attn_fwd_otilde(*args, otilde.data_ptr(), *tail)
+        with torch.cuda.device(q.device):
+            st = capi.ent_attn_fwd_otilde(*args, otilde.data_ptr(), *tail)
         _raise(st, "ent_attn_fwd_otilde")
     return o, tau, mask, iters
 
@@ -102,20 +109,23 @@ def entmax_attn_bwd(q, k, v, o, dout, tau, block_mask, alpha: float = 1.5, causa
             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(),
             _stream_handle(q.device))
     if otilde is None:
-        st = capi.ent_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                               o.data_ptr() if o is not None else None, *tail)
+        with torch.cuda.device(q.device):
+            st = capi.ent_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                   o.data_ptr() if o is not None else None, *tail)
         _raise(st, "ent_attn_bwd")
     else:
         _check_otilde(otilde, q)
-        st = capi.ent_attn_bwd_otilde(q.data_ptr(), k.data_ptr(), v.data_ptr(), otilde.data_ptr(),
-                                      *tail)
+        with torch.cuda.device(q.device):
+            st = capi.ent_attn_bwd_otilde(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                          otilde.data_ptr(), *tail)
         _raise(st, "ent_attn_bwd_otilde")
     return dq, dk, dv
 
 
 def read_status(ws: torch.Tensor) -> list[int]:
     """Counters of the last call that used ``ws`` (synchronises); raises on a timeout flag."""
-    st, ctr = capi.ent_attn_read_status(ws.data_ptr(), _stream_handle(ws.device))
+    with torch.cuda.device(ws.device):
+        st, ctr = capi.ent_attn_read_status(ws.data_ptr(), _stream_handle(ws.device))
     _raise(st, "ent_attn_read_status")
     return ctr
 
@@ -183,10 +193,11 @@ def entmax_rows_fwd(z, alpha: float = 1.5, solver: str = "hist", *, out=None):
         iters = torch.empty(rows, dtype=torch.uint8, device=z.device)
     else:
         p, tau, iters = out
-    st = capi.ent_entmax_rows_fwd(z.data_ptr(), rows, n, _DTYPES[z.dtype], alpha, SOLVERS[solver],
-                                  p.data_ptr(), tau.data_ptr(),
-                                  iters.data_ptr() if iters is not None else None,
-                                  _stream_handle(z.device))
+    with torch.cuda.device(z.device):
+        st = capi.ent_entmax_rows_fwd(z.data_ptr(), rows, n, _DTYPES[z.dtype], alpha,
+                                      SOLVERS[solver], p.data_ptr(), tau.data_ptr(),
+                                      iters.data_ptr() if iters is not None else None,
+                                      _stream_handle(z.device))
     _raise(st, "ent_entmax_rows_fwd")
     return p, tau, iters
 
@@ -196,7 +207,9 @@ def entmax_rows_bwd(z, tau, dp, alpha: float = 1.5, *, out=None):
     _check_rows(z, dp)
     rows, n = z.shape
     dz = torch.empty_like(z) if out is None else out
-    st = capi.ent_entmax_rows_bwd(z.data_ptr(), tau.data_ptr(), dp.data_ptr(), rows, n,
-                                  _DTYPES[z.dtype], alpha, dz.data_ptr(), _stream_handle(z.device))
+    with torch.cuda.device(z.device):
+        st = capi.ent_entmax_rows_bwd(z.data_ptr(), tau.data_ptr(), dp.data_ptr(), rows, n,
+                                      _DTYPES[z.dtype], alpha, dz.data_ptr(),
+                                      _stream_handle(z.device))
     _raise(st, "ent_entmax_rows_bwd")
     return dz

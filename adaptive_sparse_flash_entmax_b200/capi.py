@@ -59,6 +59,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ent_attn_bwd_otilde.restype = ci
     lib.ent_attn_read_status.argtypes = [vp, ctypes.POINTER(ctypes.c_longlong), vp]
     lib.ent_attn_read_status.restype = ci
+    lib.ent_attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci,
+                                         vp, vp, vp, vp]
+    lib.ent_attn_bwd_noalloc.restype = ci
+    lib.ent_attn_noalloc_read_status.argtypes = [ctypes.POINTER(ctypes.c_longlong), vp]
+    lib.ent_attn_noalloc_read_status.restype = ci
     lib.ent_attn_last_error.argtypes = []
     lib.ent_attn_last_error.restype = ctypes.c_char_p
     lib.ent_entmax_rows_max_n.argtypes = []
@@ -135,4 +140,17 @@ def ent_attn_read_status(ws, stream) -> tuple[int, list[int]]:
     """(status, counters[8]) of a workspace; synchronises the stream."""
     arr = (ctypes.c_longlong * 8)()
     st = load().ent_attn_read_status(ws, arr, stream)
+    return st, list(arr)
+
+
+def ent_attn_bwd_noalloc(q, k, v, o, dout, tau, block_mask, B, H, N, d, dtype, alpha, causal,
+                         dq, dk, dv, stream) -> int:
+    return load().ent_attn_bwd_noalloc(q, k, v, o, dout, tau, block_mask, B, H, N, d, dtype,
+                                       float(alpha), int(causal), dq, dk, dv, stream)
+
+
+def ent_attn_noalloc_read_status(stream) -> tuple[int, list[int]]:
+    """(status, counters[8]) of the last ent_attn_bwd_noalloc call on the current device."""
+    arr = (ctypes.c_longlong * 8)()
+    st = load().ent_attn_noalloc_read_status(arr, stream)
     return st, list(arr)

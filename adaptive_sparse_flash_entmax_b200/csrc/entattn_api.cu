@@ -62,18 +62,16 @@ int hist_budget() {
     return 0;
 }
 
-// Backward workspace layout (after the 256-byte header).
+// Backward workspace layout: the 256-byte header, then delta (one float per query row).
 struct BwdLayout {
-    size_t delta, dq_acc, lists, total;
+    size_t delta, total;
 };
 
-BwdLayout bwd_layout(int B, int H, int N, int d) {
-    const size_t BH = (size_t)B * H, T = (size_t)n_tiles(N);
+BwdLayout bwd_layout(int B, int H, int N) {
+    const size_t BH = (size_t)B * H;
     BwdLayout L;
     L.delta = kHdr;
-    L.dq_acc = L.delta + round_up(BH * N * sizeof(float), 256);
-    L.lists = L.dq_acc + round_up(BH * N * d * sizeof(float), 256);
-    L.total = L.lists + round_up(BH * 2 * T * (T + 1) * sizeof(int), 256);
+    L.total = L.delta + round_up(BH * N * sizeof(float), 256);
     return L;
 }
 
@@ -85,6 +83,21 @@ ent_status check_common(int B, int H, int N, int d, int dtype, float alpha, int 
     if (d != 64 && d != 128) return fail(ENT_EUNSUPPORTED, "head dim d=%d (supported: 64, 128)", d);
     if ((long long)B * H > 65535) return fail(ENT_EUNSUPPORTED, "B*H=%lld exceeds 65535", (long long)B * H);
     if (N > 130944) return fail(ENT_EUNSUPPORTED, "N=%d exceeds 130944", N);
+    return ENT_OK;
+}
+
+// Copies a workspace header (status word and counters) to the host after the
+// work queued on `stream` is done.
+ent_status read_header(const void* ws, long long* counters, void* stream) {
+    ent::WsHeader h;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the workspace header");
+    if (counters)
+        for (int i = 0; i < 8; ++i) counters[i] = (long long)h.counters[i];
+    if (h.status != 0)
+        return fail(ENT_ETIMEOUT, "a bounded device wait gave up (site %u)", h.timeout_site);
     return ENT_OK;
 }
 
@@ -102,7 +115,7 @@ size_t ent_attn_fwd_workspace_size(int B, int H, int N, int d, int dtype) {
 size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype) {
     (void)dtype;
     if (B < 0 || H < 0 || N < 0 || d < 0) return 0;
-    return bwd_layout(B, H, N, d).total;
+    return bwd_layout(B, H, N).total;
 }
 
 const char* ent_attn_last_error(void) { return g_err.c_str(); }
@@ -169,7 +182,7 @@ ent_status bwd_impl(const void* q, const void* k, const void* v, const float* ot
     ent_status st = check_common(B, H, N, d, dtype, alpha, causal);
     if (st != ENT_OK) return st;
     if (!ws) return fail(ENT_EINVAL, "null workspace");
-    const BwdLayout L = bwd_layout(B, H, N, d);
+    const BwdLayout L = bwd_layout(B, H, N);
     if (ws_bytes < L.total)
         return fail(ENT_EINVAL, "workspace of %zu bytes is below the required %zu", ws_bytes, L.total);
     if (!aligned16(ws)) return fail(ENT_EINVAL, "workspace pointer not 16-byte aligned");
@@ -193,8 +206,6 @@ ent_status bwd_impl(const void* q, const void* k, const void* v, const float* ot
     char* base = static_cast<char*>(ws);
     a.hdr = reinterpret_cast<ent::WsHeader*>(base);
     a.delta = reinterpret_cast<float*>(base + L.delta);
-    a.dq_acc = reinterpret_cast<float*>(base + L.dq_acc);
-    a.lists = reinterpret_cast<int*>(base + L.lists);
     a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal;
     a.alpha = alpha;
     const int gm = gamma_mode(alpha, &a.gamma);
@@ -313,16 +324,7 @@ ent_status ent_entmax_rows_bwd(const void* z, const float* tau, const void* dp, 
 
 ent_status ent_attn_read_status(const void* ws, long long* counters, void* stream) {
     if (!ws) return fail(ENT_EINVAL, "null workspace");
-    ent::WsHeader h;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-    if (e != cudaSuccess) return cuda_fail(e, "reading the workspace header");
-    if (counters)
-        for (int i = 0; i < 8; ++i) counters[i] = (long long)h.counters[i];
-    if (h.status != 0)
-        return fail(ENT_ETIMEOUT, "a bounded device wait gave up (site %u)", h.timeout_site);
-    return ENT_OK;
+    return read_header(ws, counters, stream);
 }
 
 }  // extern "C"
@@ -406,8 +408,6 @@ extern "C" ent_status ent_attn_bwd_noalloc(const void* q, const void* k, const v
     char* b = static_cast<char*>(base);
     a.hdr = reinterpret_cast<ent::WsHeader*>(b);
     a.delta = reinterpret_cast<float*>(b + kHdr);
-    a.dq_acc = nullptr;
-    a.lists = nullptr;
     a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal;
     a.alpha = alpha;
     const int gm = gamma_mode(alpha, &a.gamma);
@@ -422,4 +422,19 @@ extern "C" ent_status ent_attn_bwd_noalloc(const void* q, const void* k, const v
     }
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return ENT_OK;
+}
+
+extern "C" ent_status ent_attn_noalloc_read_status(long long* counters, void* stream) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    void* base = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_fixed_scratch_mu);
+        if (dev >= 0 && dev < kMaxScratchDevices) base = g_fixed_scratch_addr[dev];
+    }
+    if (!base)
+        return fail(ENT_EINVAL,
+                    "ent_attn_noalloc_read_status: no ent_attn_bwd_noalloc call on device %d yet", dev);
+    return read_header(base, counters, stream);
 }

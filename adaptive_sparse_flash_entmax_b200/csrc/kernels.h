@@ -39,8 +39,6 @@ struct BwdArgs {
     const float* otilde;   // nullable: the forward's otilde; then delta_i = dO_i . otilde_i
                            // and the delta pass over the keys is skipped
     float* delta;          // workspace [BH*N]
-    float* dq_acc;         // workspace [BH*N*d] fp32 (tensor-core path)
-    int* lists;            // workspace: per-tile / per-block live lists (tensor-core path)
     WsHeader* hdr;
     int BH, N, T, causal;
     float alpha, gamma, cx, scale;

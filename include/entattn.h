@@ -71,7 +71,11 @@ typedef enum { ENT_F32 = 0, ENT_BF16 = 1 } ent_dtype;
 /* Query/key tile edge of the block mask (128). */
 int ent_attn_block_size(void);
 
-/* Bytes of device workspace the forward / backward need for this shape. */
+/*
+ * Bytes of device workspace the forward / backward need for this shape.
+ * The backward's is the 256-byte header plus delta, one float per query row:
+ * 256 + round_up(B*H*N*4, 256).  A negative size gives 0.
+ */
 size_t ent_attn_fwd_workspace_size(int B, int H, int N, int d, int dtype);
 size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype);
 
@@ -168,15 +172,26 @@ ent_status ent_attn_bwd_otilde(const void *q, const void *k, const void *v, cons
  *    (the call clears the header itself): calls whose work overlaps on the GPU
  *    (concurrent streams, or other host threads) race and must be ordered by
  *    the caller.
- *  - A bounded device wait that gives up is not reported (there is no
- *    workspace to pass to ent_attn_read_status); use ent_attn_bwd when the
- *    timeout status is needed.
+ *  - A bounded device wait that gives up sets the status word in the array's
+ *    header; ent_attn_noalloc_read_status reads it (and the counters) back.
  * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  */
 ent_status ent_attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
                                 const void *dout, const float *tau, const uint8_t *block_mask,
                                 int B, int H, int N, int d, int dtype, float alpha, int causal,
                                 void *dq, void *dk, void *dv, void *stream);
+
+/*
+ * Status of the last ent_attn_bwd_noalloc call on the current device: the
+ * same as ent_attn_read_status on a workspace (synchronises `stream`, copies
+ * the header to the host, fills counters when non-null, returns ENT_ETIMEOUT
+ * if a bounded wait gave up), read from the library's fixed array.  The array
+ * is shared, so the answer belongs to whichever ent_attn_bwd_noalloc call
+ * last wrote it; order the calls.  Returns ENT_EINVAL if no
+ * ent_attn_bwd_noalloc call has looked up the array on this device yet.
+ * Allocates nothing.
+ */
+ent_status ent_attn_noalloc_read_status(long long *counters, void *stream);
 
 /*
  * Synchronises `stream` and reads the status word and the work counters of a

@@ -42,6 +42,8 @@ int main(void) {
     CHECK(ent_entmax_rows_bwd(fake, ffake, fake, 2, 99999, ENT_F32, 1.5f, fake, NULL) ==
           ENT_EUNSUPPORTED);
     CHECK(ent_attn_read_status(NULL, NULL, NULL) == ENT_EINVAL);
+    /* no device here: the no-alloc status reader reports an error, never OK */
+    CHECK(ent_attn_noalloc_read_status(NULL, NULL) != ENT_OK);
     printf("abi from C ok\n");
     return 0;
 }

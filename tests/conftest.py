@@ -17,3 +17,18 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With ENT_PARITY_REPORT=<path>, write the worst |dO| beyond bf16 storage
+    rounding seen per workload (tests/parity.py O_REPORT) as JSON."""
+    path = os.environ.get("ENT_PARITY_REPORT")
+    if not path:
+        return
+    try:
+        from parity import O_REPORT
+    except ImportError:
+        return
+    import json
+    with open(path, "w") as f:
+        json.dump(dict(sorted(O_REPORT.items())), f, indent=1)

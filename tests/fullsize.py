@@ -28,9 +28,7 @@ BLK = 128
 BAND = 1e-3
 
 
-def _half_ulp_bf16(x):
-    ax = torch.clamp(x.abs(), min=torch.finfo(torch.float32).tiny)
-    return torch.exp2(torch.floor(torch.log2(ax)) - 8)
+from parity import O_TOL, o_excess
 
 
 def check_forward(q, k, v, tau, mask, o, alpha, causal, otilde=None, chunk=512):
@@ -95,10 +93,10 @@ def _check(q, k, v, tau, mask, o, alpha, causal, otilde, chunk):
                 bm[r0 // BLK: r0 // BLK + tmax.shape[0]] = tmax
                 # O = P V with exact p
                 o_ref = torch.pow(up, gamma) @ V
-                err = (o[b, h, r0:r1].float() - o_ref).abs() - _half_ulp_bf16(o_ref) * (o.dtype == torch.bfloat16)
+                odt = "bf16" if o.dtype == torch.bfloat16 else "f32"
+                err = o_excess(o[b, h, r0:r1].float(), o_ref, odt)
                 worst["o"] = max(worst["o"], err.max().item())
-                assert err.max().item() <= (1e-2 if o.dtype == torch.bfloat16 else 1e-4), \
-                    f"O off (head {b},{h}): {err.max().item()}"
+                assert err.max().item() <= O_TOL[odt], f"O off (head {b},{h}): {err.max().item()}"
                 if otilde is not None:
                     ot_ref = (g @ V) / sg[:, None]
                     ot = otilde[b, h, r0:r1]

@@ -30,8 +30,11 @@ def test_sizes(lib):
     assert capi.ent_attn_block_size() == 128
     assert capi.ent_attn_fwd_workspace_size(4, 16, 4096, 128, capi.ENT_BF16) >= 256
     B, H, N, d = 4, 16, 4096, 128
-    ws = capi.ent_attn_bwd_workspace_size(B, H, N, d, capi.ENT_BF16)
-    assert ws >= 256 + B * H * N * 4 + B * H * N * d * 4
+    # the backward's workspace is its header plus delta (one float per query row), no more
+    for (B, H, N, d) in ((4, 16, 4096, 128), (1, 1, 1, 64), (3, 5, 300, 64), (0, 4, 128, 128)):
+        rows = B * H * N * 4
+        assert capi.ent_attn_bwd_workspace_size(B, H, N, d, capi.ENT_BF16) == 256 + -(-rows // 256) * 256
+    assert capi.ent_attn_bwd_workspace_size(-1, 1, 128, 64, capi.ENT_BF16) == 0
 
 
 FAKE = 1 << 20   # a 16-byte-aligned non-null value; never dereferenced on argument errors
@@ -77,7 +80,7 @@ def test_fwd_argument_errors(lib, kw, code):
     (dict(d=32), capi.ENT_EUNSUPPORTED),
     (dict(tau=None), capi.ENT_EINVAL),
     (dict(dq=FAKE + 8), capi.ENT_EINVAL),
-    (dict(ws_bytes=1024), capi.ENT_EINVAL),
+    (dict(ws_bytes=512), capi.ENT_EINVAL),   # needs 256 + 128 * 4
 ])
 def test_bwd_argument_errors(lib, kw, code):
     assert bwd(**kw) == code

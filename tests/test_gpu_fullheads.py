@@ -38,7 +38,7 @@ def _run(w, heads):
     qs, ks, vs, dos = (sel(a) for a in (q, k, v, do))
     o_ref, tau_ref, marg = oracle.attn_fwd(qs, ks, vs, w.alpha, w.causal)
     check_tau(gpu["tau"], tau_ref)
-    check_o(gpu["o"], o_ref, w.dtype)
+    check_o(gpu["o"], o_ref, w.dtype, label=f"{w.name} alpha {w.alpha} beta {w.beta} (whole heads)")
     check_mask(gpu["mask"], marg)
     ref = oracle.attn_bwd(qs, ks, vs, dos, w.alpha, w.causal)[:3]
     for g in (grads, grads_ot):

@@ -29,7 +29,7 @@ def full_parity(q, k, v, do, alpha, causal, dtype, bwd=True):
     gpu = run_gpu(q, k, v, do, alpha, causal, dtype, with_bwd=bwd)
     o_ref, tau_ref, marg = oracle.attn_fwd(q, k, v, alpha, causal)
     check_tau(gpu["tau"], tau_ref)
-    check_o(gpu["o"], o_ref, dtype)
+    check_o(gpu["o"], o_ref, dtype, label=f"small cases {dtype} (whole oracle)")
     check_mask(gpu["mask"], marg)
     B, H, N, d = q.shape
     rows = np.unique(np.r_[0, N - 1, np.arange(0, B * H * N, max(1, B * H * N // 64))])
@@ -179,7 +179,8 @@ def _sampled_parity(w, seed=0, n_rows=48, tiles=(0, -1), late_keys=64, early_key
     rows = np.array(sorted(set(rows)))
     o_r, tau_r, bmax = oracle.attn_fwd_rows(q, k, v, w.alpha, w.causal, rows)
     check_tau(gpu["tau"].reshape(-1)[rows], tau_r)
-    check_o(gpu["o"].reshape(-1, d)[rows], o_r, w.dtype)
+    check_o(gpu["o"].reshape(-1, d)[rows], o_r, w.dtype,
+            label=f"{w.name} alpha {w.alpha} beta {w.beta} (sampled rows)")
     check_support(q, k, gpu["tau"].reshape(-1)[rows], tau_r, w.alpha, w.causal, rows)
     # whole tiles: the mask row needs every row of the tile
     for b, h in heads:

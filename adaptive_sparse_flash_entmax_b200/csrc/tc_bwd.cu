@@ -14,8 +14,9 @@
 // there as its A operand:
 //   dq kernel   one CTA per 128-row query tile, one live 128-key block per job.
 //               Phase A: S = Q K^T, dP = dO V^T -> delta per row (also written
-//               to the workspace).  Phase B: again S and dP, dS as a pair of
-//               bf16 parts (hi + lo) and dQ += dS K (K read MN-major).  Given
+//               to the workspace).  Phase B: again S and dP, dS rounded to
+//               bf16 and dQ += dS K (K read MN-major), then a rank-1 correction
+//               for the rounding residual of dS's rows (which sum to 0).  Given
 //               the forward's otilde = sum_j g_ij v_j / sum_j g_ij, delta_i =
 //               dO_i . otilde_i (since dP = dO V^T) and phase A is skipped.
 //   dkv kernel  one CTA per 128-key block, Q/dO in 64-row sub-tiles of the
@@ -84,8 +85,7 @@ __device__ __forceinline__ void store_out_row(void* out, size_t off, const float
 // dq kernel: delta and dQ for one 128-row query tile, one 128-key live block
 // per job (128-wide MMAs run at the tensor rate; 64-wide ones do not).
 // TMEM: phase A keeps two S/dP pairs (S at 256p, dP at 256p + 128); phase B
-// one pair at 0, dQ at 256 and dS (bf16 hi at 384, lo at 448, two keys per
-// column).  K blocks stay three jobs in shared memory (S, then dQ reads them
+// one pair at 0, dQ at 256 and dS (bf16 at 384, two keys per column).  K blocks stay three jobs in shared memory (S, then dQ reads them
 // MN-major one job later); V blocks feed dP only.
 // =========================================================================
 template <int D>
@@ -97,8 +97,8 @@ struct DqLayout {
     static constexpr int kDO = kQ + kTile;
     static constexpr int kK0 = kDO + kTile;
     static constexpr int kV0 = kK0 + kKSlots * kTile;
-    static constexpr int kXch = kV0 + kVSlots * kTile;  // [2][2][128] f32
-    static constexpr int kBars = kXch + 2 * 2 * 128 * 4;
+    static constexpr int kXch = kV0 + kVSlots * kTile;  // [5][2][128] f32
+    static constexpr int kBars = kXch + 5 * 2 * 128 * 4;
     static constexpr int kMisc = kBars + 8 * 24;        // up to 24 mbarriers
     static constexpr int kList = kMisc + 16;            // live key blocks, uint16 [T]
     static size_t bytes(int T) { return (size_t)kList + 2 * (size_t)T + 16 + 1024; }
@@ -242,8 +242,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 umma_commit(&s_full[p]);
                 return true;
             };
-            // dQ += (dS_hi + dS_lo) K for phase B job i: the two bf16 parts carry dS to
-            // ~16 bits, which the cancellation in sum_j dS_ij k_j (rows of dS sum to 0) needs
+            // dQ += bf16(dS) K for phase B job i (the rounding residual of dS, whose rows
+            // sum to 0, is corrected in the epilogue)
             auto issue_dq = [&](int i) -> bool {
                 const int ks = (nA + i) % KS;
                 if (!mbar_wait(ds_full, i & 1, ab, 25)) return false;
@@ -253,7 +253,6 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int kk = 0; kk < kBlk / 16; ++kk) {
                     const uint64_t bdesc = bk + ((kk * 16 * 128) >> 4);
                     umma_bf16_ts(tmem + 256, tmem + 384 + kk * 8, bdesc, idesc_dq, (i > 0 || kk > 0) ? 1u : 0u);
-                    umma_bf16_ts(tmem + 256, tmem + 448 + kk * 8, bdesc, idesc_dq, 1u);
                 }
                 umma_commit(ds_free);
                 umma_commit(&kempty[ks]);
@@ -285,7 +284,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const uint32_t lane_base = lane0 + half * 64;
         const float gamma = a.gamma, cx = a.cx;
         const float tau = row_valid ? a.tau[(size_t)bh * N + i] : 0.f;
-        float* xch = reinterpret_cast<float*>(smem + L::kXch);   // [2][2][128]
+        float* xch = reinterpret_cast<float*>(smem + L::kXch);   // [5][2][128]
         const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-tau, -tau);
         bool ok = true;
         // S and dP of job j, columns [32r, 32r + 32) of this thread's 64 keys; the pair is
@@ -363,31 +362,47 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             delta = (SG > 0.f) ? SGDP / SG : 0.f;
         }
         if (row_valid && half == 0) a.delta[(size_t)bh * N + i] = delta;
-        // phase B: dS = g (dP - delta) as bf16 hi + lo into TMEM
+        // phase B: dS = g (dP - delta) rounded to bf16 into TMEM.  With dS rounded once,
+        // the rows' residuals eps_i = sum_j (bf16(dS_ij) - dS_ij) would reach dQ as
+        // eps_i times the common part of the support's keys (large on clustered keys,
+        // where sum_j dS_ij k_j cancels); the epilogue subtracts eps_i k_{j*}, j* the
+        // row's arg-max key, which leaves only eps-sized errors times k_j - k_{j*}.
         const float2 nd2 = make_float2(-delta, -delta), m1 = make_float2(-1.f, -1.f);
+        float best = -INFINITY;   // this thread's largest score and its key
+        int jbest = 0;
+        float2 eps2 = make_float2(0.f, 0.f);
         for (int ib = 0; ib < nB && ok; ++ib) {
             const int j = nA + ib;
             if (!(ok = mbar_wait(&s_full[0], use_of(j) & 1, ab, 26))) break;
             tc_fence_after();
-            uint32_t whi[32], wlo[32];
+            const int key0 = list[ib] * kBlk + half * 64;   // key of this thread's first column
+            uint32_t whi[32];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 float s[32], dp[32];
                 load_round(j, r, s, dp);
+                float rmax = s[0];
+#pragma unroll
+                for (int c = 1; c < 32; ++c) rmax = fmaxf(rmax, s[c]);
+                if (rmax > best) {   // rare after the first blocks: find the column
+                    best = rmax;
+                    int cc = 0;
+#pragma unroll
+                    for (int c = 31; c >= 0; --c) cc = (s[c] == rmax) ? c : cc;
+                    jbest = key0 + r * 32 + cc;
+                }
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const float2 g = entmax_g_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma);
                     const float2 d = __fmul2_rn(g, __fadd2_rn(make_float2(dp[c], dp[c + 1]), nd2));
                     const __nv_bfloat162 h = __floats2bfloat162_rn(d.x, d.y);
-                    const float2 lo = __ffma2_rn(__bfloat1622float2(h), m1, d);   // d - bf16(d), exact
+                    eps2 = __fadd2_rn(eps2, __ffma2_rn(d, m1, __bfloat1622float2(h)));   // bf16(d) - d
                     whi[r * 16 + (c >> 1)] = *reinterpret_cast<const uint32_t*>(&h);
-                    wlo[r * 16 + (c >> 1)] = pack_bf16(lo.x, lo.y);
                 }
             }
             // the dS region is free once dQ of the previous job has read it
             if (!(ok = mbar_wait(ds_free, (ib & 1) ^ 1, ab, 27))) break;
             tmem_st32(lane0 + 384 + half * 32, whi);
-            tmem_st32(lane0 + 448 + half * 32, wlo);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -406,9 +421,34 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int c = 0; c < DH; ++c) acc[c] = 0.f;
         }
+        // the row's arg-max key and residual: the halves meet in shared memory (slots of
+        // their own, so no reader of the delta exchange is overtaken; every elementwise
+        // thread reaches this barrier once, also after an abort)
+        xch[(2 * 2 + half) * 128 + row] = best;
+        xch[(3 * 2 + half) * 128 + row] = __int_as_float(jbest);
+        xch[(4 * 2 + half) * 128 + row] = eps2.x + eps2.y;
+        named_bar(1, kEw);
+        const float obest = xch[(2 * 2 + (half ^ 1)) * 128 + row];
+        const int ojbest = __float_as_int(xch[(3 * 2 + (half ^ 1)) * 128 + row]);
+        const float eps = eps2.x + eps2.y + xch[(4 * 2 + (half ^ 1)) * 128 + row];
+        const int js = (obest > best || (obest == best && ojbest < jbest)) ? ojbest : jbest;
+        if (row_valid && ok && nB > 0 && fmaxf(best, obest) > -INFINITY) {
+            const __nv_bfloat16* kr = static_cast<const __nv_bfloat16*>(a.k) + ((size_t)bh * N + js) * D + half * DH;
+#pragma unroll
+            for (int c = 0; c < DH; c += 8) {
+                const uint4 k8 = *reinterpret_cast<const uint4*>(kr + c);
+                const uint32_t w[4] = {k8.x, k8.y, k8.z, k8.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                    acc[c + 2 * e] = fmaf(-eps, kv.x, acc[c + 2 * e]);
+                    acc[c + 2 * e + 1] = fmaf(-eps, kv.y, acc[c + 2 * e + 1]);
+                }
+            }
+        }
         if (row_valid) store_out_row(a.dq, ((size_t)bh * N + i) * D + half * DH, acc, DH, a.scale);
-        if (threadIdx.x == 64)   // block products: phase A S, dP (2) + phase B S, dP, dQ hi, lo (4)
-            atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(2 * nA + 4 * nB));
+        if (threadIdx.x == 64)   // block products: phase A S, dP (2) + phase B S, dP, dQ (3)
+            atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(2 * nA + 3 * nB));
     }
 
     tc_fence_before();

@@ -62,6 +62,33 @@ int hist_budget() {
     return 0;
 }
 
+// Forward workspace layout: the 256-byte header, then (bf16 path) the key-block bounds
+// of the statistics pass: per head max |c| and min R (float bits), per 64-key
+// half-block {R, L} and the bf16 centroid.
+struct FwdLayout {
+    size_t maxc, minr, stats, cent, total;
+};
+
+FwdLayout fwd_layout(int B, int H, int N, int d) {
+    const size_t BH = (size_t)B * H, T2 = 2 * (size_t)n_tiles(N);
+    FwdLayout L;
+    L.maxc = kHdr;                       // [BH] words, then min R [BH] right after them
+    L.minr = L.maxc + BH * 4;
+    L.stats = L.maxc + round_up(BH * 8, 256);
+    L.cent = L.stats + round_up(BH * T2 * 8, 256);
+    L.total = L.cent + round_up(BH * T2 * (size_t)d * 2, 256);
+    return L;
+}
+
+// Statistics-pass skipping by key-block bounds (bf16 path), on by default.
+// ENTATTN_BOUND=0 (environment, read per call) turns it off, for ablations; the
+// outputs are the same either way (a block it rules out holds no u > 0 and no row
+// maximum, so every later pass sees the same blocks and sums).
+bool bound_enabled() {
+    const char* v = getenv("ENTATTN_BOUND");
+    return !(v && *v && atoi(v) == 0);
+}
+
 // Backward workspace layout: the 256-byte header, then delta (one float per query row).
 struct BwdLayout {
     size_t delta, total;
@@ -108,8 +135,9 @@ extern "C" {
 int ent_attn_block_size(void) { return ent::kBlk; }
 
 size_t ent_attn_fwd_workspace_size(int B, int H, int N, int d, int dtype) {
-    (void)B; (void)H; (void)N; (void)d; (void)dtype;
-    return kHdr;
+    (void)dtype;
+    if (B < 0 || H < 0 || N < 0 || d < 0) return 0;
+    return fwd_layout(B, H, N, d).total;
 }
 
 size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype) {
@@ -144,7 +172,11 @@ ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, i
     if (!empty && want_otilde && (!otilde || !aligned16(otilde)))
         return fail(ENT_EINVAL, "otilde must be a non-null 16-byte aligned pointer");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
+    const FwdLayout FL = fwd_layout(B, H, N, d);
+    const bool bound = dtype == ENT_BF16 && hist_budget() == 0 && bound_enabled() && !empty;
+    // header and the per-head max |c| start at 0, the per-head min R at all ones
+    cudaError_t e = cudaMemsetAsync(ws, 0, bound ? FL.minr : kHdr, s);
+    if (e == cudaSuccess && bound) e = cudaMemsetAsync(static_cast<char*>(ws) + FL.minr, 0xFF, (size_t)B * H * 4, s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace header");
     if (empty) return ENT_OK;
 
@@ -162,6 +194,14 @@ ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, i
     a.ftol = dtype == ENT_F32 ? 1e-6f : 1e-5f;
     a.stol = dtype == ENT_F32 ? 4e-7f : 1e-6f;
     a.hist_budget = hist_budget();
+    if (bound) {
+        // statistics-pass skipping by key-block bounds; off with the histogram start, whose
+        // windows must count every score down to their lowest bin
+        char* base = static_cast<char*>(ws);
+        a.head_words = reinterpret_cast<unsigned int*>(base + FL.maxc);
+        a.bstats = reinterpret_cast<float2*>(base + FL.stats);
+        a.cent = base + FL.cent;
+    }
     if (dtype == ENT_F32) {
         e = ent::simt_fwd_f32(a, d, gm, s);
     } else {

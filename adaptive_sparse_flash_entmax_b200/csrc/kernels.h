@@ -24,6 +24,18 @@ struct FwdArgs {
     int hist_budget;       // tensor-core path: histogram inserts a tile may make after its
                            // first block (0: no histogram, < 0: no limit)
     float* otilde;         // nullable [BH][N][d] fp32: sum_j g_ij v_j / sum_j g_ij
+    // Key-block bounds for skipping statistics-pass blocks (tensor-core path; all null:
+    // no bound pass).  Per 64-key half-block hb of head bh (T2 = 2T of them):
+    //   cent[bh][hb][d]  bf16 centroid c (mean of its valid keys, rounded),
+    //   bstats[bh][hb]   {R, L}: every computed score q.k_j of the half-block is
+    //                    <= q.c + |q| R, and the largest is >= q.c - |q| L (R < 0: no
+    //                    valid key),
+    //   head_words       [BH] max |c| then [BH] min R, as float bits (a bound can rule out
+    //                    a block only where R < 2 max |c|, so heads without such a block
+    //                    skip the pass).
+    void* cent;
+    float2* bstats;
+    unsigned int* head_words;
 };
 
 struct BwdArgs {

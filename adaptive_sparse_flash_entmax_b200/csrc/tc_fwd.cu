@@ -26,6 +26,13 @@
 // maximum of x, and a block is streamed again only if some warp's maximum
 // exceeds that warp's smallest current tau (otherwise no row of the tile has
 // u > 0 there, so the skipped block adds nothing to the sums or the mask).
+// Before pass 0 a bound pass may rule out whole key blocks (Exploiting
+// Sparsity, applied to the statistics pass itself): S_c = Q C^T against the
+// centroids of the 64-key half-blocks gives, per row and half-block, an upper
+// bound q.c + |q| R of every score and a lower bound q.c - |q| L of the
+// largest one.  A block whose upper bound lies at or below (largest lower
+// bound) - 1 <= m - 1 <= tau for every row of the tile has p = 0 throughout,
+// cannot hold a row maximum, and is left out of pass 0 and of everything after.
 // After each score pass the elementwise group publishes a decision (another
 // solver pass, or the P.V pass with its live-block list) that the producer and
 // the MMA issuer wait on.  Every wait is bounded (2 s); a wait that gives up
@@ -71,7 +78,8 @@ struct Layout {
     static constexpr int kNumBars = 40;
     static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, decision, njobs, abort
     static constexpr int kPtab = kMisc + 32;              // 68 floats
-    static constexpr int kLive = kPtab + 68 * 4;          // live[T], cand[T] (bytes), list[T] (int),
+    static constexpr int kMw = kPtab + 68 * 4;            // 8 floats: per-warp bound thresholds
+    static constexpr int kLive = kMw + 8 * 4;             // live[T], cand[T] (bytes), list[T] (int),
                                                           // per-warp block maxima [T][8] (bf16)
     __host__ __device__ static size_t r16(int T) { return (size_t)((T + 15) / 16) * 16; }
     static size_t bytes(int T) { return (size_t)kLive + 2 * r16(T) + 4 * (size_t)T + 16 * (size_t)T + 1024; }
@@ -90,6 +98,24 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// Column maxima over the 32 lanes of a warp for 32 values per lane: after five
+// exchange steps lane l holds the maximum of column l in v[0].  Each step keeps
+// half of the columns (the lane bit picks which half) and combines them with the
+// partner lane's copy of the same columns.
+__device__ __forceinline__ void warp_colmax_32(float* v, int lane) {
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        const int w = 16 >> step, bit = 16 >> step;
+        const bool up = (lane & bit) != 0;
+#pragma unroll
+        for (int c = 0; c < w; ++c) {
+            const float send = up ? v[c] : v[c + w];
+            const float keep = up ? v[c + w] : v[c];
+            v[c] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, bit));
+        }
+    }
+}
+
 // Bounded wait that ignores the abort flag (used to drain in-flight copies).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = globaltimer_ns();
@@ -105,7 +131,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 template <int D, int GM, bool OT>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_c,
+              const FwdArgs a) {
     using L = Layout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -138,6 +165,16 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int nblk = a.causal ? t + 1 : T;
     const Abort ab{&misc->abort, a.hdr};
     constexpr int SB = (OT && D == 128) ? 2 : kSbuf;   // S buffers of the P.V pass
+    // Bound pass for this tile: only where a centroid bound can rule a block out at all
+    // (some half-block of the head has R < 2 max |c|: a bound q.c_b + |q| R_b below
+    // q.c_b' - |q| L_b' - 1/cx needs R_b < |c_b' - c_b| <= 2 max |c|)
+    bool use_bound = false;
+    if (a.bstats != nullptr) {
+        const float maxc = __uint_as_float(a.head_words[bh]);
+        const float minr = __uint_as_float(a.head_words[a.BH + bh]);
+        use_bound = minr < 2.f * maxc;
+    }
+    const int nbj = use_bound ? (2 * nblk + 127) >> 7 : 0;   // 128-centroid jobs of the bound pass
     constexpr uint32_t kOtCol = 256 + D;                // G.V accumulator (OT)
 
     if (threadIdx.x == 0) {
@@ -161,6 +198,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         fence_barrier_init();
         // the Q tile goes first, before the block-wide setup
         prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
+        if (use_bound) prefetch_tmap(&tm_c);
         mbar_arrive_expect_tx(q_full, L::kTile);
         for (int at = 0; at < D / 64; ++at)
             tma_load_3d(smem + L::kQ + at * kAtom, &tm_q, at * 64, t * kBlk, bh, q_full);
@@ -180,18 +218,19 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (lane == 0) {
             int sj = 0, dj = 0, kind = kDecSolve;   // P.V-pass tiles, score-pass double slots loaded
             uint32_t dec_phase = 0;
-            bool ok = true, first = true;
+            bool ok = true, first = !use_bound, bound = use_bound;
             // a score-pass job: K blocks b0 and b1 (b1 < 0: none) stacked in one double slot,
-            // block h at rows 128h of each [256 rows x 64] atom
-            auto load_pair = [&](int b0, int b1) -> bool {
+            // block h at rows 128h of each [256 rows x 64] atom (the bound pass loads blocks
+            // of 128 centroids from `map` the same way)
+            auto load_pair = [&](const CUtensorMap* map, int b0, int b1) -> bool {
                 const int ds = dj % kDSlots;
                 if (!mbar_wait(&kempty2[ds], ((dj / kDSlots) & 1) ^ 1, ab, 1)) return false;
                 mbar_arrive_expect_tx(&kfull2[ds], (b1 >= 0 ? 2 : 1) * L::kTile);
                 uint8_t* base = smem + L::kRing + ds * 2 * L::kTile;
                 for (int at = 0; at < D / 64; ++at) {
-                    tma_load_3d(base + at * 2 * kAtom, &tm_k, at * 64, b0 * kBlk, bh, &kfull2[ds]);
+                    tma_load_3d(base + at * 2 * kAtom, map, at * 64, b0 * kBlk, bh, &kfull2[ds]);
                     if (b1 >= 0)
-                        tma_load_3d(base + at * 2 * kAtom + kAtom, &tm_k, at * 64, b1 * kBlk, bh, &kfull2[ds]);
+                        tma_load_3d(base + at * 2 * kAtom + kAtom, map, at * 64, b1 * kBlk, bh, &kfull2[ds]);
                 }
                 ++dj;
                 return true;
@@ -208,12 +247,15 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             };
             while (ok) {
                 const bool pv = kind == kDecPv;
-                const int njobs = first ? nblk : misc->njobs;
-                if (!pv) {
+                const int njobs = bound ? nbj : first ? nblk : misc->njobs;
+                if (bound) {
+                    for (int i = 0; i < njobs && ok; i += 2)
+                        ok = load_pair(&tm_c, i, (i + 1 < njobs) ? i + 1 : -1);
+                } else if (!pv) {
                     for (int i = 0; i < njobs && ok; i += 2) {
                         const int b0 = first ? i : job_list[i];
                         const int b1 = (i + 1 < njobs) ? (first ? i + 1 : job_list[i + 1]) : -1;
-                        ok = load_pair(b0, b1);
+                        ok = load_pair(&tm_k, b0, b1);
                     }
                 } else {
                     for (int i = 0; i < njobs && ok; ++i) {
@@ -222,7 +264,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         if (ok) ok = load_tile(&tm_v, b);
                     }
                 }
-                first = false;
+                first = bound = false;
                 if (!ok || pv) break;
                 if (!(ok = mbar_wait(dec_bar, dec_phase, ab, 2))) break;
                 dec_phase ^= 1;
@@ -248,7 +290,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tc_fence_after();
             int sjob = 0, kind = kDecSolve;   // score-pass jobs issued (= double slots consumed)
             uint32_t dec_phase = 0;
-            bool first = true;
+            bool first = !use_bound, bound = use_bound;
             auto wait_tile = [&](int tt) { return mbar_wait(&kfull[tt % kSlots], (tt / kSlots) & 1, ab, 4); };
             auto issue_s = [&](int sb, int tt) {
                 const uint64_t dk = dring + ((uint32_t)((tt % kSlots) * L::kTile) >> 4);
@@ -263,8 +305,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             };
             while (ok) {
                 const bool pv = kind == kDecPv;
-                const int njobs = first ? nblk : misc->njobs;
-                first = false;
+                const int njobs = bound ? nbj : first ? nblk : misc->njobs;
+                first = bound = false;
                 if (!pv) {
                     for (int i = 0; i < njobs && ok; i += 2, ++sjob) {
                         const int sb = sjob & 1, ds = sjob % kDSlots;
@@ -405,16 +447,126 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         sv.iters = 0;
         const int wi = warp - 2;                  // elementwise warp index 0..7
         int sjob = 0, pass = 0, nlive = 0;
-        long long qk_blocks = nblk;
+        long long qk_blocks = use_bound ? nbj : nblk, skipped = 0;
         bool ok = true;
+        if (use_bound) {
+            // ---- bound pass: S_c = Q C^T over the tile's half-block centroids
+            // |q| of this row from the swizzled Q tile (a sum of squares does not depend on
+            // the order of the 16-byte chunks; lanes start at different chunks so that a
+            // warp's loads spread over the banks)
+            ok = mbar_wait(q_full, 0, ab, 12);
+            float qq = 0.f;
+            if (ok) {
+                constexpr int kCh = (D == 128) ? 8 : 4;
+                const uint8_t* qrow = smem + L::kQ + (D == 128 ? half * kAtom : half * 64) + row * 128;
+#pragma unroll
+                for (int cc = 0; cc < kCh; ++cc) {
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(qrow + ((cc + lane) & (kCh - 1)) * 16);
+                    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+                        qq = fmaf(f2.x, f2.x, fmaf(f2.y, f2.y, qq));
+                    }
+                }
+            }
+            X(1, half) = qq;
+            named_bar(1, kEw);
+            // rounding of the 2 x 64 squares and the square root: far below 1e-5 relative
+            const float qn = sqrtf(qq + X(1, half ^ 1)) * 1.00001f;
+            float mlb = -INFINITY;                      // largest lower bound of this half-row
+            const float2* bst = a.bstats + (size_t)bh * 2 * T;
+            const int wq = (quarter - 2) & 3;           // warp slot of this quarter, key half 0 (+4: 1)
+            for (int jj = 0; jj < nbj && ok; jj += 2, ++sjob) {
+                const int sb = sjob & 1;
+                if (!(ok = mbar_wait(&s_full2[sb], (sjob >> 1) & 1, ab, 13))) break;
+                tc_fence_after();
+                const int nb2 = (jj + 1 < nbj) ? 2 : 1;
+#pragma unroll 1
+                for (int h = 0; h < nb2; ++h) {
+#pragma unroll 1
+                    for (int r = 0; r < 2; ++r) {
+                        float s[32];
+                        tmem_ld32(lane_base + sb * 256 + h * 128 + c0 + 32 * r, s);
+                        tmem_wait_ld();
+                        reg_fence<32>(s);
+                        if (h == nb2 - 1 && r == 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&s_empty2[sb]);
+                        }
+                        const int cbase = (jj + h) * kBlk + c0 + 32 * r;   // centroid of column 0
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const int cent = cbase + c;       // half-block: keys 64 cent .. 64 cent + 63
+                            const float2 st = (cent < 2 * nblk) ? __ldg(bst + cent) : make_float2(-1.f, 0.f);
+                            const bool has = row_valid && st.x >= 0.f;
+                            const bool some = !a.causal || cent * 64 <= i;        // a key of it is admissible
+                            const bool every = !a.causal || cent * 64 + 63 <= i;  // all of its keys are
+                            const float ub = cx * fmaf(qn, st.x, s[c]);
+                            const float lb = cx * fmaf(-qn, st.y, s[c]);
+                            if (has && every) mlb = fmaxf(mlb, lb);
+                            s[c] = (has && some) ? ub : -INFINITY;
+                        }
+                        warp_colmax_32(s, lane);
+                        const int cent = cbase + lane;    // lane l: the warp's maximum of column l
+                        if ((cent >> 1) < nblk) bmw[(cent >> 1) * 8 + wq + 4 * (cent & 1)] = __float2bfloat16_ru(s[0]);
+                    }
+                }
+            }
+            ok = named_bar_and(1, kEw, ok);
+            if (ok) {
+                X(0, half) = mlb;
+                named_bar(1, kEw);
+                mlb = fmaxf(mlb, X(0, half ^ 1));
+                // a block is ruled out for this warp's rows when its upper bound lies at or
+                // below the smallest (lower bound of the row max) - 1 <= m - 1 <= tau
+                float th = row_valid ? mlb - 1.f : INFINITY;
+#pragma unroll
+                for (int o2 = 16; o2 > 0; o2 >>= 1) th = fminf(th, __shfl_xor_sync(0xffffffffu, th, o2));
+                float* mw = reinterpret_cast<float*>(smem + L::kMw);
+                if (lane == 0) mw[wi] = th;
+                named_bar(1, kEw);   // every warp's bounds and threshold are in
+                for (int b = ew; b < nblk; b += kEw) {
+                    bool need = false;
+#pragma unroll
+                    for (int w8 = 0; w8 < 8; ++w8) {
+                        const float thw = mw[w8];
+                        need |= __bfloat162float(bmw[b * 8 + w8]) > thw - 1e-4f * fmaxf(1.f, fabsf(thw));
+                    }
+                    // a block left out holds no u > 0 for any tau the solver visits (tau >= m - 1)
+                    if (!need)
+                        for (int w8 = 0; w8 < 8; ++w8) bmw[b * 8 + w8] = __float2bfloat16(-INFINITY);
+                    live[b] = need ? 1 : 0;
+                }
+                named_bar(1, kEw);
+                if (warp == 2) {
+                    int n = 0;
+                    for (int base = 0; base < nblk; base += 32) {
+                        const int bb = base + lane;
+                        const bool f = bb < nblk && live[bb] != 0;
+                        const unsigned int msk = __ballot_sync(0xffffffffu, f);
+                        if (f) job_list[n + __popc(msk & ((1u << lane) - 1u))] = bb;
+                        n += __popc(msk);
+                    }
+                    if (lane == 0) {
+                        misc->njobs = n;
+                        misc->decision = kDecSolve;
+                        mbar_arrive(dec_bar);
+                    }
+                }
+            }
+        }
         for (;; ++pass) {
             float F0 = 0.f, F1 = 0.f, F2 = 0.f;
             int npj = nblk;
-            if (pass > 0) {
-                for (int bb = ew; bb < nblk; bb += kEw) live[bb] = 0;
+            if (pass > 0 || use_bound) {
+                if (pass > 0)
+                    for (int bb = ew; bb < nblk; bb += kEw) live[bb] = 0;
                 named_bar(1, kEw);   // also publishes job_list / njobs of this pass
                 npj = misc->njobs;
                 qk_blocks += npj;
+                if (pass == 0) skipped = nblk - npj;
             }
             // jobs of two blocks (one 256-column S buffer); the buffer is released after
             // the second block's load
@@ -426,7 +578,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll 1
                 for (int h = 0; h < nb2; ++h) {
                     const int bi = jj + h;      // block index within this pass
-                    const int b = (pass == 0) ? bi : job_list[bi];
+                    const int b = (pass == 0 && !use_bound) ? bi : job_list[bi];
                     float s[64];
                     tmem_ld32(lane_base + sb * 256 + h * 128 + c0, &s[0]);
                     tmem_ld32(lane_base + sb * 256 + h * 128 + c0 + 32, &s[32]);
@@ -711,6 +863,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             atomicAdd(&a.hdr->counters[kCtrPasses], (unsigned long long)npass);
             atomicAdd(&a.hdr->counters[kCtrTiles], 1ull);
             if (OT) atomicAdd(&a.hdr->counters[kCtrGvBlocks], (unsigned long long)nlive);
+            if (skipped) atomicAdd(&a.hdr->counters[kCtrSkipped], (unsigned long long)skipped);
         }
     }
 
@@ -759,36 +912,141 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int N, int D) {
     return make_tmap_bf16_rows(map, base, BH, N, D, 128);
 }
 
+// ------------------------------------------------------------------ key-block bounds
+// One warp per 64-key half-block hb of head bh (keys 64 hb .. 64 hb + 63 below N):
+//   c   = the mean of its keys, rounded to bf16 (stored: the bound pass multiplies it
+//         with Q on the tensor cores),
+//   r   = max_j |k_j - c|, so q.k_j <= q.c + |q| r (Cauchy-Schwarz),
+//   dc  = |mean - c|, so max_j q.k_j >= q.mean >= q.c - |q| dc.
+// The computed scores differ from the exact ones by the fp32 accumulation of the
+// tensor-core products, at most d 2^-23 |q| |k| each; with e = 2 d 2^-23 (twice that
+// bound) and |k_j| <= |c| + r the stored terms R = r + e (2|c| + r) and
+// L = dc + e (2|c| + r) + 1e-4 (|c| + r) (the last term for the fp32 mean) cover both
+// the score and the centroid product.  R < 0 marks a half-block with no key.  The
+// head's max |c| and min R go to head_words by atomic max / min on the float bits
+// (non-negative floats order like their bit patterns): head_words[bh] and
+// head_words[BH + bh], BH = gridDim.y.
+template <int D>
+__global__ void __launch_bounds__(128) block_stats_kernel(const __nv_bfloat16* __restrict__ k, int N, int T2,
+                                                          __nv_bfloat16* __restrict__ cent,
+                                                          float2* __restrict__ bstats,
+                                                          unsigned int* __restrict__ head_words) {
+    constexpr int PL = D / 32;                 // dimensions per lane
+    const int lane = threadIdx.x & 31;
+    const int hb = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int bh = blockIdx.y;
+    if (hb >= T2) return;
+    const int j0 = hb * 64;
+    const int nk = min(64, N - j0);
+    const __nv_bfloat16* kr = k + ((size_t)bh * N + max(j0, 0)) * D + lane * PL;
+    __nv_bfloat16* cr = cent + ((size_t)bh * T2 + hb) * D + lane * PL;
+    auto load = [&](int j, float* x) {
+        if (PL == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(kr + (size_t)j * D);
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+            const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+            x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+        } else {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(kr + (size_t)j * D);
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+            x[0] = a.x; x[1] = a.y;
+        }
+    };
+    auto wsum = [](float x) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        return x;
+    };
+    if (nk <= 0) {
+#pragma unroll
+        for (int e = 0; e < PL; ++e) cr[e] = __float2bfloat16(0.f);
+        if (lane == 0) bstats[(size_t)bh * T2 + hb] = make_float2(-1.f, 0.f);
+        return;
+    }
+    float sum[PL];
+#pragma unroll
+    for (int e = 0; e < PL; ++e) sum[e] = 0.f;
+    for (int j = 0; j < nk; ++j) {
+        float x[PL];
+        load(j, x);
+#pragma unroll
+        for (int e = 0; e < PL; ++e) sum[e] += x[e];
+    }
+    float c[PL], dc2 = 0.f, c2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < PL; ++e) {
+        const float mean = sum[e] / (float)nk;
+        const __nv_bfloat16 cb = __float2bfloat16_rn(mean);
+        cr[e] = cb;
+        c[e] = __bfloat162float(cb);
+        dc2 = fmaf(mean - c[e], mean - c[e], dc2);
+        c2 = fmaf(c[e], c[e], c2);
+    }
+    dc2 = wsum(dc2);
+    c2 = wsum(c2);
+    float r2 = 0.f;
+    for (int j = 0; j < nk; ++j) {
+        float x[PL], d2 = 0.f;
+        load(j, x);
+#pragma unroll
+        for (int e = 0; e < PL; ++e) d2 = fmaf(x[e] - c[e], x[e] - c[e], d2);
+        r2 = fmaxf(r2, wsum(d2));
+    }
+    // fp32 sums of at most d squares: relative error below d 2^-24, halved by the root
+    const float slack = 1.f + 4e-5f;
+    const float r = sqrtf(r2) * slack, nc = sqrtf(c2) * slack, dc = sqrtf(dc2) * slack;
+    const float e = 2.f * (float)D * 1.1920929e-7f;   // 2 d 2^-23
+    const float R = (r + e * (2.f * nc + r)) * slack;
+    const float Lm = (dc + e * (2.f * nc + r) + 1e-4f * (nc + r)) * slack;
+    if (lane == 0) {
+        bstats[(size_t)bh * T2 + hb] = make_float2(R, Lm);
+        atomicMax(&head_words[bh], __float_as_uint(nc));
+        atomicMin(&head_words[gridDim.y + bh], __float_as_uint(R));
+    }
+}
+
 template <int D, int GM>
 static cudaError_t launch_tc_fwd(const CUtensorMap& mq, const CUtensorMap& mk,
-                                 const CUtensorMap& mv, const FwdArgs& a, cudaStream_t s) {
+                                 const CUtensorMap& mv, const CUtensorMap& mc, const FwdArgs& a,
+                                 cudaStream_t s) {
+    if (a.bstats) {
+        const int T2 = 2 * a.T;
+        block_stats_kernel<D><<<dim3((T2 + 3) / 4, a.BH), 128, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(a.k), a.N, T2, static_cast<__nv_bfloat16*>(a.cent),
+            a.bstats, a.head_words);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     const size_t sm = Layout<D>::bytes(a.T);
     auto kern = a.otilde ? tc_fwd_kernel<D, GM, true> : tc_fwd_kernel<D, GM, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(mq, mk, mv, a);
+    kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(mq, mk, mv, mc, a);
     return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t tc_fwd_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                            const FwdArgs& a, int gm, cudaStream_t s) {
+                            const CUtensorMap& mc, const FwdArgs& a, int gm, cudaStream_t s) {
     switch (gm) {
-        case 1: return launch_tc_fwd<D, 1>(mq, mk, mv, a, s);
-        case 2: return launch_tc_fwd<D, 2>(mq, mk, mv, a, s);
-        case 4: return launch_tc_fwd<D, 4>(mq, mk, mv, a, s);
-        default: return launch_tc_fwd<D, 0>(mq, mk, mv, a, s);
+        case 1: return launch_tc_fwd<D, 1>(mq, mk, mv, mc, a, s);
+        case 2: return launch_tc_fwd<D, 2>(mq, mk, mv, mc, a, s);
+        case 4: return launch_tc_fwd<D, 4>(mq, mk, mv, mc, a, s);
+        default: return launch_tc_fwd<D, 0>(mq, mk, mv, mc, a, s);
     }
 }
 
 cudaError_t tc_fwd(const FwdArgs& a, int d, int gm, cudaStream_t s, const char** why) {
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mc;
+    // the centroids [BH][2T][d] load like K blocks (128 of them per box); without the
+    // bound pass the map is never used and points at K
+    const bool okc = a.cent ? make_tmap_bf16(&mc, a.cent, a.BH, 2 * a.T, d) : make_tmap_bf16(&mc, a.k, a.BH, a.N, d);
     if (!make_tmap_bf16(&mq, a.q, a.BH, a.N, d) || !make_tmap_bf16(&mk, a.k, a.BH, a.N, d) ||
-        !make_tmap_bf16(&mv, a.v, a.BH, a.N, d)) {
+        !make_tmap_bf16(&mv, a.v, a.BH, a.N, d) || !okc) {
         *why = "cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
-    return d == 64 ? tc_fwd_d<64>(mq, mk, mv, a, gm, s) : tc_fwd_d<128>(mq, mk, mv, a, gm, s);
+    return d == 64 ? tc_fwd_d<64>(mq, mk, mv, mc, a, gm, s) : tc_fwd_d<128>(mq, mk, mv, mc, a, gm, s);
 }
 
 }  // namespace ent

@@ -42,7 +42,7 @@ FAKE = 1 << 20   # a 16-byte-aligned non-null value; never dereferenced on argum
 
 def fwd(**kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, B=1, H=1, N=128, d=64, dtype=capi.ENT_BF16, alpha=1.5,
-             causal=1, o=FAKE, tau=FAKE, block_mask=FAKE, iters=None, ws=FAKE, ws_bytes=256,
+             causal=1, o=FAKE, tau=FAKE, block_mask=FAKE, iters=None, ws=FAKE, ws_bytes=1 << 30,
              stream=None)
     a.update(kw)
     return capi.ent_attn_fwd(**a)
@@ -121,7 +121,7 @@ def test_otilde_argument_errors(lib, which):
     if which == "fwd":
         args = dict(q=FAKE, k=FAKE, v=FAKE, B=1, H=1, N=128, d=64, dtype=capi.ENT_BF16,
                     alpha=1.5, causal=1, o=FAKE, tau=FAKE, block_mask=FAKE, iters=None,
-                    otilde=None, ws=FAKE, ws_bytes=256, stream=None)
+                    otilde=None, ws=FAKE, ws_bytes=1 << 30, stream=None)
         call = capi.ent_attn_fwd_otilde
     else:
         args = dict(q=FAKE, k=FAKE, v=FAKE, otilde=None, dout=FAKE, tau=FAKE, block_mask=FAKE,

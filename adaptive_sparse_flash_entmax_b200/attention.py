@@ -47,13 +47,24 @@ def workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
+def alloc_lists(q):
+    """Support-list buffers for ``entmax_attn_fwd(..., lists=)``: (key int32, u float32
+    [B, H, N, cap], n uint8 [B, H, N])."""
+    B, H, N, _ = q.shape
+    cap = capi.ent_attn_list_cap()
+    return (torch.empty((B, H, N, cap), dtype=torch.int32, device=q.device),
+            torch.empty((B, H, N, cap), dtype=torch.float32, device=q.device),
+            torch.empty((B, H, N), dtype=torch.uint8, device=q.device))
+
+
 def entmax_attn_fwd(q, k, v, alpha: float = 1.5, causal: bool = False, *, with_iters=False,
-                    ws: torch.Tensor | None = None, out=None, otilde=None):
+                    ws: torch.Tensor | None = None, out=None, otilde=None, lists=None):
     """Forward: returns (o, tau, block_mask, iters_or_None).
 
     ``otilde``: a float32 tensor shaped like q to call ``ent_attn_fwd_otilde`` instead,
     which also fills it with sum_j g_ij v_j / sum_j g_ij (the backward's delta is then
-    dO . otilde, see ``entmax_attn_bwd``)."""
+    dO . otilde, see ``entmax_attn_bwd``).  ``lists``: the buffers of ``alloc_lists`` to
+    call ``ent_attn_fwd_lists``, which also records every row's (key, u) support list."""
     _check(q, k, v)
     B, H, N, d = q.shape
     dt = _DTYPES[q.dtype]
@@ -71,7 +82,14 @@ def entmax_attn_fwd(q, k, v, alpha: float = 1.5, causal: bool = False, *, with_i
     args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, N, d, dt, alpha, causal, o.data_ptr(),
             tau.data_ptr(), mask.data_ptr(), iters.data_ptr() if iters is not None else None)
     tail = (ws.data_ptr(), ws.numel(), _stream_handle(q.device))
-    if otilde is None:
+    if lists is not None:
+        if otilde is not None:
+            raise ValueError("otilde and lists are separate forward variants")
+        lk, lu, ln = lists
+        with torch.cuda.device(q.device):
+            st = capi.ent_attn_fwd_lists(*args, lk.data_ptr(), lu.data_ptr(), ln.data_ptr(), *tail)
+        _raise(st, "ent_attn_fwd_lists")
+    elif otilde is None:
         with torch.cuda.device(q.device):
             st = capi.ent_attn_fwd(*args, *tail)
         _raise(st, "ent_attn_fwd")
@@ -90,11 +108,13 @@ def _check_otilde(otilde, q):
 
 
 def entmax_attn_bwd(q, k, v, o, dout, tau, block_mask, alpha: float = 1.5, causal: bool = False,
-                    *, ws: torch.Tensor | None = None, out=None, otilde=None):
+                    *, ws: torch.Tensor | None = None, out=None, otilde=None, lists=None):
     """Backward: returns (dq, dk, dv).
 
     ``otilde``: the tensor a forward with ``otilde=`` filled; the call then goes to
-    ``ent_attn_bwd_otilde`` (delta = dO . otilde, no delta pass over the keys)."""
+    ``ent_attn_bwd_otilde`` (delta = dO . otilde, no delta pass over the keys).
+    ``lists``: the support lists a forward with ``lists=`` filled; the call then goes to
+    ``ent_attn_bwd_lists`` (query tiles whose rows all have lists are done from them)."""
     _check(q, k, v, dout)
     B, H, N, d = q.shape
     dt = _DTYPES[q.dtype]
@@ -102,13 +122,22 @@ def entmax_attn_bwd(q, k, v, o, dout, tau, block_mask, alpha: float = 1.5, causa
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     else:
         dq, dk, dv = out
-    need = capi.ent_attn_bwd_workspace_size(B, H, N, d, dt)
+    need = (capi.ent_attn_bwd_lists_workspace_size if lists is not None
+            else capi.ent_attn_bwd_workspace_size)(B, H, N, d, dt)
     if ws is None or ws.numel() < need:
         ws = workspace(need, q.device)
     tail = (dout.data_ptr(), tau.data_ptr(), block_mask.data_ptr(), B, H, N, d, dt, alpha, causal,
             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(),
             _stream_handle(q.device))
-    if otilde is None:
+    if lists is not None:
+        if otilde is not None:
+            raise ValueError("otilde and lists are separate backward variants")
+        lk, lu, ln = lists
+        with torch.cuda.device(q.device):
+            st = capi.ent_attn_bwd_lists(q.data_ptr(), k.data_ptr(), v.data_ptr(), lk.data_ptr(),
+                                         lu.data_ptr(), ln.data_ptr(), *tail)
+        _raise(st, "ent_attn_bwd_lists")
+    elif otilde is None:
         with torch.cuda.device(q.device):
             st = capi.ent_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                    o.data_ptr() if o is not None else None, *tail)

@@ -64,6 +64,16 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.ent_attn_bwd_noalloc.restype = ci
     lib.ent_attn_noalloc_read_status.argtypes = [ctypes.POINTER(ctypes.c_longlong), vp]
     lib.ent_attn_noalloc_read_status.restype = ci
+    lib.ent_attn_list_cap.argtypes = []
+    lib.ent_attn_list_cap.restype = ci
+    lib.ent_attn_bwd_lists_workspace_size.argtypes = [ci, ci, ci, ci, ci]
+    lib.ent_attn_bwd_lists_workspace_size.restype = sz
+    lib.ent_attn_fwd_lists.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp, vp, vp, vp, vp,
+                                       vp, vp, vp, sz, vp]
+    lib.ent_attn_fwd_lists.restype = ci
+    lib.ent_attn_bwd_lists.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf,
+                                       ci, vp, vp, vp, vp, sz, vp]
+    lib.ent_attn_bwd_lists.restype = ci
     lib.ent_attn_last_error.argtypes = []
     lib.ent_attn_last_error.restype = ctypes.c_char_p
     lib.ent_entmax_rows_max_n.argtypes = []
@@ -154,3 +164,25 @@ def ent_attn_noalloc_read_status(stream) -> tuple[int, list[int]]:
     arr = (ctypes.c_longlong * 8)()
     st = load().ent_attn_noalloc_read_status(arr, stream)
     return st, list(arr)
+
+
+def ent_attn_list_cap() -> int:
+    return load().ent_attn_list_cap()
+
+
+def ent_attn_bwd_lists_workspace_size(B, H, N, d, dtype) -> int:
+    return load().ent_attn_bwd_lists_workspace_size(B, H, N, d, dtype)
+
+
+def ent_attn_fwd_lists(q, k, v, B, H, N, d, dtype, alpha, causal, o, tau, block_mask, iters,
+                       list_key, list_u, list_n, ws, ws_bytes, stream) -> int:
+    return load().ent_attn_fwd_lists(q, k, v, B, H, N, d, dtype, float(alpha), int(causal), o,
+                                     tau, block_mask, iters, list_key, list_u, list_n, ws,
+                                     ws_bytes, stream)
+
+
+def ent_attn_bwd_lists(q, k, v, list_key, list_u, list_n, dout, tau, block_mask, B, H, N, d,
+                       dtype, alpha, causal, dq, dk, dv, ws, ws_bytes, stream) -> int:
+    return load().ent_attn_bwd_lists(q, k, v, list_key, list_u, list_n, dout, tau, block_mask, B,
+                                     H, N, d, dtype, float(alpha), int(causal), dq, dk, dv, ws,
+                                     ws_bytes, stream)

@@ -35,7 +35,7 @@ struct WsHeader {
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
 enum Counter { kCtrQkBlocks = 0, kCtrPvBlocks = 1, kCtrPasses = 2, kCtrTiles = 3,
-               kCtrBwdBlocks = 4, kCtrGvBlocks = 5, kCtrSkipped = 6 };
+               kCtrBwdBlocks = 4, kCtrGvBlocks = 5, kCtrSkipped = 6, kCtrListEntries = 7 };
 
 __device__ __forceinline__ float load_f(const float* p, size_t i) { return p[i]; }
 __device__ __forceinline__ float load_f(const __nv_bfloat16* p, size_t i) {

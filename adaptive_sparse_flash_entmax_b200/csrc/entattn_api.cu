@@ -107,7 +107,8 @@ ent_status check_common(int B, int H, int N, int d, int dtype, float alpha, int 
     if (dtype != ENT_F32 && dtype != ENT_BF16) return fail(ENT_EINVAL, "unknown dtype %d", dtype);
     if (!(alpha > 1.f && alpha <= 2.f)) return fail(ENT_EINVAL, "alpha=%g outside (1, 2]", (double)alpha);
     if (causal != 0 && causal != 1) return fail(ENT_EINVAL, "causal must be 0 or 1 (got %d)", causal);
-    if (d != 64 && d != 128) return fail(ENT_EUNSUPPORTED, "head dim d=%d (supported: 64, 128)", d);
+    if (d != 32 && d != 64 && d != 128)
+        return fail(ENT_EUNSUPPORTED, "head dim d=%d (supported: 32, 64, 128)", d);
     if ((long long)B * H > 65535) return fail(ENT_EUNSUPPORTED, "B*H=%lld exceeds 65535", (long long)B * H);
     if (N > 130944) return fail(ENT_EUNSUPPORTED, "N=%d exceeds 130944", N);
     return ENT_OK;
@@ -152,13 +153,39 @@ const char* ent_attn_last_error(void) { return g_err.c_str(); }
 
 namespace {
 
+// Support lists of ent_attn_fwd_lists / ent_attn_bwd_lists (all null otherwise).
+struct Lists {
+    int32_t* key = nullptr;
+    float* u = nullptr;
+    uint8_t* n = nullptr;
+    bool want = false;
+};
+
+// Backward workspace of ent_attn_bwd_lists: the plain layout, then the per-tile flags
+// and the fp32 dK, dV accumulators of the list kernel.
+struct ListLayout {
+    size_t tiles, dk, dv, total;
+};
+
+ListLayout list_layout(int B, int H, int N, int d) {
+    const size_t BH = (size_t)B * H;
+    ListLayout L;
+    L.tiles = bwd_layout(B, H, N).total;
+    L.dk = L.tiles + round_up(BH * (size_t)n_tiles(N), 256);
+    L.dv = L.dk + round_up(BH * N * (size_t)d * 4, 256);
+    L.total = L.dv + round_up(BH * N * (size_t)d * 4, 256);
+    return L;
+}
+
 // Forward of ent_attn_fwd and, with a non-null otilde, of ent_attn_fwd_otilde.
 ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                     int dtype, float alpha, int causal, void* o, float* tau, uint8_t* block_mask,
                     uint8_t* iters, float* otilde, bool want_otilde, void* ws, size_t ws_bytes,
-                    void* stream) {
+                    void* stream, const Lists& lists = Lists()) {
     ent_status st = check_common(B, H, N, d, dtype, alpha, causal);
     if (st != ENT_OK) return st;
+    if (lists.want && dtype != ENT_BF16)
+        return fail(ENT_EUNSUPPORTED, "support lists are built by the bf16 forward only");
     if (!ws) return fail(ENT_EINVAL, "null workspace");
     if (ws_bytes < ent_attn_fwd_workspace_size(B, H, N, d, dtype))
         return fail(ENT_EINVAL, "workspace of %zu bytes is below the required %zu", ws_bytes,
@@ -171,6 +198,8 @@ ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, i
         return fail(ENT_EINVAL, "q/k/v/o must be 16-byte aligned");
     if (!empty && want_otilde && (!otilde || !aligned16(otilde)))
         return fail(ENT_EINVAL, "otilde must be a non-null 16-byte aligned pointer");
+    if (!empty && lists.want && (!lists.key || !lists.u || !lists.n))
+        return fail(ENT_EINVAL, "null list_key/list_u/list_n pointer");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const FwdLayout FL = fwd_layout(B, H, N, d);
     const bool bound = dtype == ENT_BF16 && hist_budget() == 0 && bound_enabled() && !empty;
@@ -183,8 +212,9 @@ ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, i
     ent::FwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.o = o; a.tau = tau; a.mask = block_mask; a.iters = iters;
     a.otilde = want_otilde ? otilde : nullptr;
+    a.list_key = lists.key; a.list_u = lists.u; a.list_n = lists.n;
     a.hdr = static_cast<ent::WsHeader*>(ws);
-    a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal;
+    a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal; a.dr = d;
     a.alpha = alpha;
     const int gm = gamma_mode(alpha, &a.gamma);
     a.scale = 1.f / sqrtf((float)d);
@@ -218,13 +248,17 @@ ent_status bwd_impl(const void* q, const void* k, const void* v, const float* ot
                     bool want_otilde, const void* dout, const float* tau,
                     const uint8_t* block_mask, int B, int H, int N, int d, int dtype, float alpha,
                     int causal, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
-                    void* stream) {
+                    void* stream, const Lists& lists = Lists()) {
     ent_status st = check_common(B, H, N, d, dtype, alpha, causal);
     if (st != ENT_OK) return st;
+    if (lists.want && dtype != ENT_BF16)
+        return fail(ENT_EUNSUPPORTED, "support lists are built by the bf16 forward only");
     if (!ws) return fail(ENT_EINVAL, "null workspace");
     const BwdLayout L = bwd_layout(B, H, N);
-    if (ws_bytes < L.total)
-        return fail(ENT_EINVAL, "workspace of %zu bytes is below the required %zu", ws_bytes, L.total);
+    const ListLayout LL = list_layout(B, H, N, d);
+    const size_t need = lists.want ? LL.total : L.total;
+    if (ws_bytes < need)
+        return fail(ENT_EINVAL, "workspace of %zu bytes is below the required %zu", ws_bytes, need);
     if (!aligned16(ws)) return fail(ENT_EINVAL, "workspace pointer not 16-byte aligned");
     const bool empty = (long long)B * H == 0 || N == 0;
     if (!empty && (!q || !k || !v || !dout || !tau || !block_mask || !dq || !dk || !dv))
@@ -234,10 +268,16 @@ ent_status bwd_impl(const void* q, const void* k, const void* v, const float* ot
         return fail(ENT_EINVAL, "q/k/v/dout/dq/dk/dv must be 16-byte aligned");
     if (!empty && want_otilde && (!otilde || !aligned16(otilde)))
         return fail(ENT_EINVAL, "otilde must be a non-null 16-byte aligned pointer");
+    if (!empty && lists.want && (!lists.key || !lists.u || !lists.n))
+        return fail(ENT_EINVAL, "null list_key/list_u/list_n pointer");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace header");
     if (empty) return ENT_OK;
+    if (lists.want) {   // the list kernel's dK, dV accumulators start at zero
+        e = cudaMemsetAsync(static_cast<char*>(ws) + LL.dk, 0, LL.total - LL.dk, s);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the list accumulators");
+    }
 
     ent::BwdArgs a{};
     a.q = q; a.k = k; a.v = v; a.dout = dout; a.tau = tau; a.mask = block_mask;
@@ -246,16 +286,24 @@ ent_status bwd_impl(const void* q, const void* k, const void* v, const float* ot
     char* base = static_cast<char*>(ws);
     a.hdr = reinterpret_cast<ent::WsHeader*>(base);
     a.delta = reinterpret_cast<float*>(base + L.delta);
-    a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal;
+    a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal; a.dr = d;
     a.alpha = alpha;
     const int gm = gamma_mode(alpha, &a.gamma);
     a.scale = 1.f / sqrtf((float)d);
     a.cx = (alpha - 1.f) * a.scale;
+    if (lists.want) {
+        a.list_key = lists.key; a.list_u = lists.u; a.list_n = lists.n;
+        a.tile_list = reinterpret_cast<uint8_t*>(base + LL.tiles);
+        a.dk_acc = reinterpret_cast<float*>(base + LL.dk);
+        a.dv_acc = reinterpret_cast<float*>(base + LL.dv);
+    }
     if (dtype == ENT_F32) {
         e = ent::simt_bwd_f32(a, d, gm, s);
     } else {
         const char* why = nullptr;
-        e = ent::tc_bwd(a, d, gm, s, &why);
+        // the list kernel first: it decides which query tiles it covers
+        if (lists.want) e = ent::list_bwd(a, d, gm, s);
+        if (e == cudaSuccess) e = ent::tc_bwd(a, d, gm, s, &why);
         if (e != cudaSuccess && why) return fail(ENT_ECUDA, "backward launch: %s", why);
     }
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
@@ -298,6 +346,37 @@ ent_status ent_attn_bwd_otilde(const void* q, const void* k, const void* v, cons
                                void* stream) {
     return bwd_impl(q, k, v, otilde, true, dout, tau, block_mask, B, H, N, d, dtype, alpha, causal,
                     dq, dk, dv, ws, ws_bytes, stream);
+}
+
+int ent_attn_list_cap(void) { return ent::kListCap; }
+
+size_t ent_attn_bwd_lists_workspace_size(int B, int H, int N, int d, int dtype) {
+    (void)dtype;
+    if (B < 0 || H < 0 || N < 0 || d < 0) return 0;
+    return list_layout(B, H, N, d).total;
+}
+
+ent_status ent_attn_fwd_lists(const void* q, const void* k, const void* v, int B, int H, int N,
+                              int d, int dtype, float alpha, int causal, void* o, float* tau,
+                              uint8_t* block_mask, uint8_t* iters, int32_t* list_key,
+                              float* list_u, uint8_t* list_n, void* ws, size_t ws_bytes,
+                              void* stream) {
+    Lists l;
+    l.key = list_key; l.u = list_u; l.n = list_n; l.want = true;
+    return fwd_impl(q, k, v, B, H, N, d, dtype, alpha, causal, o, tau, block_mask, iters, nullptr,
+                    false, ws, ws_bytes, stream, l);
+}
+
+ent_status ent_attn_bwd_lists(const void* q, const void* k, const void* v, const int32_t* list_key,
+                              const float* list_u, const uint8_t* list_n, const void* dout,
+                              const float* tau, const uint8_t* block_mask, int B, int H, int N,
+                              int d, int dtype, float alpha, int causal, void* dq, void* dk,
+                              void* dv, void* ws, size_t ws_bytes, void* stream) {
+    Lists l;
+    l.key = const_cast<int32_t*>(list_key); l.u = const_cast<float*>(list_u);
+    l.n = const_cast<uint8_t*>(list_n); l.want = true;
+    return bwd_impl(q, k, v, nullptr, false, dout, tau, block_mask, B, H, N, d, dtype, alpha,
+                    causal, dq, dk, dv, ws, ws_bytes, stream, l);
 }
 
 int ent_entmax_rows_max_n(void) { return 16384; }
@@ -448,7 +527,7 @@ extern "C" ent_status ent_attn_bwd_noalloc(const void* q, const void* k, const v
     char* b = static_cast<char*>(base);
     a.hdr = reinterpret_cast<ent::WsHeader*>(b);
     a.delta = reinterpret_cast<float*>(b + kHdr);
-    a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal;
+    a.BH = B * H; a.N = N; a.T = n_tiles(N); a.causal = causal; a.dr = d;
     a.alpha = alpha;
     const int gm = gamma_mode(alpha, &a.gamma);
     a.scale = 1.f / sqrtf((float)d);

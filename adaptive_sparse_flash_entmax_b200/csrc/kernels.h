@@ -7,6 +7,9 @@
 
 namespace ent {
 
+constexpr int kListCap = 16;        // entries per row in the support lists
+constexpr uint8_t kListOver = 255;  // list_n of a row with more than kListCap nonzeros
+
 struct FwdArgs {
     const void* q;
     const void* k;
@@ -17,6 +20,8 @@ struct FwdArgs {
     uint8_t* iters;        // nullable
     WsHeader* hdr;         // workspace header (status, counters)
     int BH, N, T, causal;
+    int dr;                // head dimension of the tensors (row stride); the tensor-core
+                           // kernels run d = 32 as d = 64 with zero-filled upper columns
     float alpha, gamma;    // gamma = 1/(alpha-1)
     float cx;              // (alpha-1)/sqrt(d): x = cx * (q . k)
     float scale;           // 1/sqrt(d)
@@ -36,6 +41,12 @@ struct FwdArgs {
     void* cent;
     float2* bstats;
     unsigned int* head_words;
+    // Per-row support lists (nullable; tensor-core path): for each query row the keys j
+    // with p_ij > 0 and their u_ij = x_ij - tau_i, up to kListCap of them, in list_key /
+    // list_u [BH][N][kListCap]; list_n [BH][N] the count, kListOver when the row has more.
+    int* list_key;
+    float* list_u;
+    uint8_t* list_n;
 };
 
 struct BwdArgs {
@@ -51,8 +62,19 @@ struct BwdArgs {
     const float* otilde;   // nullable: the forward's otilde; then delta_i = dO_i . otilde_i
                            // and the delta pass over the keys is skipped
     float* delta;          // workspace [BH*N]
+    // Support-list backward (nullable): the forward's lists, a per-tile flag (1: every row
+    // of the query tile has a list, so the list kernel covers the tile and the block
+    // kernels skip it) and fp32 accumulators of the list kernel's dK, dV contributions
+    // that the dkv kernel adds before it stores.
+    const int* list_key;
+    const float* list_u;
+    const uint8_t* list_n;
+    uint8_t* tile_list;    // workspace [BH][T]
+    float* dk_acc;         // workspace [BH][N][d]
+    float* dv_acc;         // workspace [BH][N][d]
     WsHeader* hdr;
     int BH, N, T, causal;
+    int dr;                // head dimension of the tensors, as in FwdArgs
     float alpha, gamma, cx, scale;
 };
 
@@ -82,5 +104,9 @@ cudaError_t simt_bwd_f32(const BwdArgs& a, int d, int gm, cudaStream_t s);
 // bf16 tensor-core path (tcgen05 + TMEM + TMA).  `why` names a host-side failure.
 cudaError_t tc_fwd(const FwdArgs& a, int d, int gm, cudaStream_t s, const char** why);
 cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char** why);
+
+// Support-list backward of the query tiles whose rows all have lists (tc_lists.cu): dQ of
+// those rows, their dK / dV contributions added into dk_acc / dv_acc, and tile_list.
+cudaError_t list_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s);
 
 }  // namespace ent

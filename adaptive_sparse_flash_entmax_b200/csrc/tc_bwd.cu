@@ -79,6 +79,22 @@ __device__ __forceinline__ void store_out_row(void* out, size_t off, const float
     }
 }
 
+// The same with an fp32 row added after scaling: out = v * sc + add (the support-list
+// kernel's dK / dV contributions).
+__device__ __forceinline__ void store_out_row_add(void* out, size_t off, const float* v, int D, float sc,
+                                                  const float* add) {
+    __nv_bfloat16* p = static_cast<__nv_bfloat16*>(out) + off;
+    for (int c = 0; c < D; c += 8) {
+        const float4 a0 = *reinterpret_cast<const float4*>(add + off + c);
+        const float4 a1 = *reinterpret_cast<const float4*>(add + off + c + 4);
+        uint4 val = make_uint4(pack_bf16(fmaf(v[c], sc, a0.x), fmaf(v[c + 1], sc, a0.y)),
+                               pack_bf16(fmaf(v[c + 2], sc, a0.z), fmaf(v[c + 3], sc, a0.w)),
+                               pack_bf16(fmaf(v[c + 4], sc, a1.x), fmaf(v[c + 5], sc, a1.y)),
+                               pack_bf16(fmaf(v[c + 6], sc, a1.z), fmaf(v[c + 7], sc, a1.w)));
+        *reinterpret_cast<uint4*>(p + c) = val;
+    }
+}
+
 }  // namespace
 
 // =========================================================================
@@ -134,6 +150,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int bh = blockIdx.y;
     const int nblk = a.causal ? t + 1 : T;
     const Abort ab{&misc->abort, a.hdr};
+    // a tile the support-list kernel covered (its dQ is written) is done
+    if (a.tile_list && a.tile_list[(size_t)bh * T + t]) return;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < KS; ++i) { mbar_init(&kfull[i], 1); mbar_init(&kempty[i], 1); }
@@ -331,9 +349,12 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         constexpr int DH = D / 2;
         float dpart = 0.f;   // with otilde: this half's share of dO_i . otilde_i
-        if (a.otilde && row_valid) {
-            const __nv_bfloat16* dor = static_cast<const __nv_bfloat16*>(a.dout) + ((size_t)bh * N + i) * D + half * DH;
-            const float* otr = a.otilde + ((size_t)bh * N + i) * D + half * DH;
+        // d = 32 runs as D = 64 (zero upper columns): the half holding columns 32..63 reads
+        // and stores nothing
+        const bool own_half = half * DH < a.dr;
+        if (a.otilde && row_valid && own_half) {
+            const __nv_bfloat16* dor = static_cast<const __nv_bfloat16*>(a.dout) + ((size_t)bh * N + i) * a.dr + half * DH;
+            const float* otr = a.otilde + ((size_t)bh * N + i) * a.dr + half * DH;
             float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll 4
             for (int c = 0; c < DH; c += 8) {
@@ -432,8 +453,8 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int ojbest = __float_as_int(xch[(3 * 2 + (half ^ 1)) * 128 + row]);
         const float eps = eps2.x + eps2.y + xch[(4 * 2 + (half ^ 1)) * 128 + row];
         const int js = (obest > best || (obest == best && ojbest < jbest)) ? ojbest : jbest;
-        if (row_valid && ok && nB > 0 && fmaxf(best, obest) > -INFINITY) {
-            const __nv_bfloat16* kr = static_cast<const __nv_bfloat16*>(a.k) + ((size_t)bh * N + js) * D + half * DH;
+        if (row_valid && own_half && ok && nB > 0 && fmaxf(best, obest) > -INFINITY) {
+            const __nv_bfloat16* kr = static_cast<const __nv_bfloat16*>(a.k) + ((size_t)bh * N + js) * a.dr + half * DH;
 #pragma unroll
             for (int c = 0; c < DH; c += 8) {
                 const uint4 k8 = *reinterpret_cast<const uint4*>(kr + c);
@@ -446,7 +467,7 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             }
         }
-        if (row_valid) store_out_row(a.dq, ((size_t)bh * N + i) * D + half * DH, acc, DH, a.scale);
+        if (row_valid && own_half) store_out_row(a.dq, ((size_t)bh * N + i) * a.dr + half * DH, acc, DH, a.scale);
         if (threadIdx.x == 64)   // block products: phase A S, dP (2) + phase B S, dP, dQ (3)
             atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(2 * nA + 3 * nB));
     }
@@ -533,7 +554,9 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         for (int base = a.causal ? b : 0; base < T; base += 32) {
             const int t = base + lane;
             int c = 0, i0a = 0, i0b = 0;
-            if (t < T && a.mask[((size_t)bh * T + t) * T + b]) {
+            // live query tiles of this key block, except those the support-list kernel covered
+            if (t < T && a.mask[((size_t)bh * T + t) * T + b] &&
+                !(a.tile_list && a.tile_list[(size_t)bh * T + t])) {
                 for (int h = 0; h < 2; ++h) {
                     const int i0 = t * kBlk + h * kSub;
                     if (i0 >= N || (a.causal && i0 + kSub - 1 < b * kBlk)) continue;
@@ -728,14 +751,22 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 #pragma unroll
             for (int c = 0; c < DH; ++c) acc[c] = 0.f;
         }
-        if (key_valid) store_out_row(a.dv, ((size_t)bh * N + jkey) * D + half * DH, acc, DH, 1.f);
+        const bool own_half = half * DH < a.dr;   // d = 32 as D = 64: columns 32..63 are not stored
+        const size_t orow = ((size_t)bh * N + jkey) * a.dr + half * DH;
+        if (key_valid && own_half) {
+            if (a.dv_acc) store_out_row_add(a.dv, orow, acc, DH, 1.f, a.dv_acc);
+            else store_out_row(a.dv, orow, acc, DH, 1.f);
+        }
         if (ok && njobs > 0) {
 #pragma unroll
             for (int c = 0; c < DH / 32; ++c) tmem_ld32(tm_dk + qoff + c * 32, &acc[c * 32]);
             tmem_wait_ld();
             reg_fence<DH>(acc);
         }
-        if (key_valid) store_out_row(a.dk, ((size_t)bh * N + jkey) * D + half * DH, acc, DH, a.scale);
+        if (key_valid && own_half) {
+            if (a.dk_acc) store_out_row_add(a.dk, orow, acc, DH, a.scale, a.dk_acc);
+            else store_out_row(a.dk, orow, acc, DH, a.scale);
+        }
         if (ew == 0)   // block products: S^T, dP^T, dV, dK (4) per 64-row half
             atomicAdd(&a.hdr->counters[kCtrBwdBlocks], (unsigned long long)(2 * njobs));
     }
@@ -791,7 +822,8 @@ cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char**
         *why = "cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
-    return d == 64 ? tc_bwd_d<64>(a, gm, s, m) : tc_bwd_d<128>(a, gm, s, m);
+    // d = 32 runs on the d = 64 kernels (zero-filled upper columns, see tc_fwd)
+    return d == 128 ? tc_bwd_d<128>(a, gm, s, m) : tc_bwd_d<64>(a, gm, s, m);
 }
 
 }  // namespace ent

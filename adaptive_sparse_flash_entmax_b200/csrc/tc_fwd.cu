@@ -79,7 +79,8 @@ struct Layout {
     static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, decision, njobs, abort
     static constexpr int kPtab = kMisc + 32;              // 68 floats
     static constexpr int kMw = kPtab + 68 * 4;            // 8 floats: per-warp bound thresholds
-    static constexpr int kLive = kMw + 8 * 4;             // live[T], cand[T] (bytes), list[T] (int),
+    static constexpr int kCnt = kMw + 8 * 4;              // 128 ints: support-list counts per row
+    static constexpr int kLive = kCnt + 128 * 4;          // live[T], cand[T] (bytes), list[T] (int),
                                                           // per-warp block maxima [T][8] (bf16)
     __host__ __device__ static size_t r16(int T) { return (size_t)((T + 15) / 16) * 16; }
     static size_t bytes(int T) { return (size_t)kLive + 2 * r16(T) + 4 * (size_t)T + 16 * (size_t)T + 1024; }
@@ -208,6 +209,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tmem_relinquish();
     }
     for (int b = threadIdx.x; b < T; b += kThreads) { live[b] = 0; cand[b] = 0; }
+    int* lcnt = reinterpret_cast<int*>(smem + L::kCnt);    // support-list entries per row
+    if (threadIdx.x < kBlk) lcnt[threadIdx.x] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -788,6 +791,27 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
                     }
                 }
+                if (a.list_n) {
+                    // support list of the row: (key, u) for every p > 0 (a bf16 p is nonzero
+                    // exactly when its bits are; most threads see none in a block)
+                    uint32_t nzw = 0u;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) nzw |= pk[c];
+                    if (nzw != 0u) {
+                        const size_t lbase = ((size_t)bh * N + i) * kListCap;
+#pragma unroll
+                        for (int c = 0; c < 64; ++c) {
+                            const float u = __fmaf_rn(s[c], cx, -sv.tau);
+                            if (u > 0.f) {
+                                const int slot = atomicAdd(&lcnt[row], 1);
+                                if (slot < kListCap) {
+                                    a.list_key[lbase + slot] = b * kBlk + c0 + c;
+                                    a.list_u[lbase + slot] = u;
+                                }
+                            }
+                        }
+                    }
+                }
                 // P over this thread's own S columns: keys c0 .. c0+63 -> columns c0 .. c0+31
                 // (and G, with otilde, -> columns c0+32 .. c0+63)
                 tmem_st32(lane_base + sbuf_col(sb) + c0, pk);
@@ -813,8 +837,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
             for (int c = 0; c < DH; ++c) o[c] = 0.f;
         }
-        if (row_valid) {
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + ((size_t)bh * N + i) * D + half * DH;
+        // d = 32 runs as D = 64 (zero upper columns): the half holding columns 32..63 stores nothing
+        const bool store_half = half * DH < a.dr;
+        if (row_valid && store_half) {
+            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.o) + ((size_t)bh * N + i) * a.dr + half * DH;
 #pragma unroll
             for (int c = 0; c < DH; c += 8) {
                 uint4 val;
@@ -825,6 +851,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 h = __floats2bfloat162_rn(o[c + 6], o[c + 7]); val.w = *reinterpret_cast<uint32_t*>(&h);
                 *reinterpret_cast<uint4*>(orow + c) = val;
             }
+        }
+        if (row_valid) {
             if (half == 0) {
                 a.tau[(size_t)bh * N + i] = sv.tau;
                 if (a.iters) a.iters[(size_t)bh * N + i] = (uint8_t)sv.iters;
@@ -847,12 +875,19 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 for (int c = 0; c < DH; ++c) o[c] = 0.f;
             }
             const float rs = sg > 0.f ? 1.f / sg : 0.f;
-            if (row_valid) {
-                float* orow = a.otilde + ((size_t)bh * N + i) * D + half * DH;
+            if (row_valid && store_half) {
+                float* orow = a.otilde + ((size_t)bh * N + i) * a.dr + half * DH;
 #pragma unroll
                 for (int c = 0; c < DH; c += 4)
                     *reinterpret_cast<float4*>(orow + c) =
                         make_float4(o[c] * rs, o[c + 1] * rs, o[c + 2] * rs, o[c + 3] * rs);
+            }
+        }
+        if (a.list_n) {
+            named_bar(1, kEw);   // every half-row's entries are counted
+            if (row_valid && half == 0) {
+                const int n = lcnt[row];
+                a.list_n[(size_t)bh * N + i] = (ok && n <= kListCap) ? (uint8_t)n : kListOver;
             }
         }
         uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
@@ -894,7 +929,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-// [BH][N][D] bf16 tensor, box {64, box_rows, 1}, 128-byte swizzle, zero fill out of bounds.
+// [BH][N][D] bf16 tensor, box {64, box_rows, 1}, 128-byte swizzle, zero fill out of bounds
+// (D = 32: the box's columns 32..63 lie outside the tensor and arrive as zeros).
 bool make_tmap_bf16_rows(CUtensorMap* map, const void* base, int BH, int N, int D, int box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -941,15 +977,17 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const __nv_bfloat16* _
     const __nv_bfloat16* kr = k + ((size_t)bh * N + max(j0, 0)) * D + lane * PL;
     __nv_bfloat16* cr = cent + ((size_t)bh * T2 + hb) * D + lane * PL;
     auto load = [&](int j, float* x) {
-        if (PL == 4) {
+        if (PL == 1) {
+            x[0] = __bfloat162float(kr[(size_t)j * D]);
+        } else if (PL == 4) {
             const uint2 w = *reinterpret_cast<const uint2*>(kr + (size_t)j * D);
-            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
-            const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
-            x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+            const float2 a2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+            const float2 b2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+            x[0] = a2.x; x[1] = a2.y; x[2] = b2.x; x[3] = b2.y;
         } else {
             const uint32_t w = *reinterpret_cast<const uint32_t*>(kr + (size_t)j * D);
-            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
-            x[0] = a.x; x[1] = a.y;
+            const float2 a2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+            x[0] = a2.x; x[1] = a2.y;
         }
     };
     auto wsum = [](float x) {
@@ -1011,9 +1049,13 @@ static cudaError_t launch_tc_fwd(const CUtensorMap& mq, const CUtensorMap& mk,
                                  cudaStream_t s) {
     if (a.bstats) {
         const int T2 = 2 * a.T;
-        block_stats_kernel<D><<<dim3((T2 + 3) / 4, a.BH), 128, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(a.k), a.N, T2, static_cast<__nv_bfloat16*>(a.cent),
-            a.bstats, a.head_words);
+        const dim3 grid((T2 + 3) / 4, a.BH);
+        const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(a.k);
+        __nv_bfloat16* cc = static_cast<__nv_bfloat16*>(a.cent);
+        if (a.dr == 32)
+            block_stats_kernel<32><<<grid, 128, 0, s>>>(kk, a.N, T2, cc, a.bstats, a.head_words);
+        else
+            block_stats_kernel<D><<<grid, 128, 0, s>>>(kk, a.N, T2, cc, a.bstats, a.head_words);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -1046,7 +1088,9 @@ cudaError_t tc_fwd(const FwdArgs& a, int d, int gm, cudaStream_t s, const char**
         *why = "cuTensorMapEncodeTiled failed";
         return cudaErrorInvalidValue;
     }
-    return d == 64 ? tc_fwd_d<64>(mq, mk, mv, mc, a, gm, s) : tc_fwd_d<128>(mq, mk, mv, mc, a, gm, s);
+    // d = 32 runs on the d = 64 kernel: its tiles hold zeros in columns 32..63, which add
+    // nothing to q.k, make O's upper columns 0 and are not stored
+    return d == 128 ? tc_fwd_d<128>(mq, mk, mv, mc, a, gm, s) : tc_fwd_d<64>(mq, mk, mv, mc, a, gm, s);
 }
 
 }  // namespace ent

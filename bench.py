@@ -51,10 +51,12 @@ def parse():
     p.add_argument("--hist-budget", type=int, default=None,
                    help="ablation: histogram insert budget per forward tile (0: no histogram, "
                         "i.e. every row from the plain bracket; -1: no limit)")
-    p.add_argument("--delta", choices=["auto", "otilde", "recompute"], default="auto",
-                   help="backward delta: from the forward's otilde (ent_attn_fwd_otilde + "
-                        "ent_attn_bwd_otilde), recomputed by a pass over the keys, or auto: "
-                        "otilde unless an untimed forward finds >= 50%% of the blocks empty")
+    p.add_argument("--delta", choices=["auto", "otilde", "recompute", "lists"], default="auto",
+                   help="backward path: delta from the forward's otilde (ent_attn_fwd_otilde + "
+                        "ent_attn_bwd_otilde), recomputed by a pass over the keys, the support "
+                        "lists (ent_attn_fwd_lists + ent_attn_bwd_lists), or auto: lists when an "
+                        "untimed forward leaves >= 90%% of the query rows with a list, else "
+                        "otilde below 50%% empty blocks, else recompute")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--B", type=int, default=None, help="override the batch (profiling cases)")
     p.add_argument("--H", type=int, default=None, help="override the head count")
@@ -430,30 +432,42 @@ class Case:
             # Measured on B200: delta from otilde makes the dense-block workloads 2-4 %
             # faster per step (the backward drops S and dP of every live block, the
             # forward adds one G V product per live block); at 95 % block sparsity the
-            # saving no longer pays for the forward's extra work.  One untimed forward
-            # measures the sparsity.
+            # saving no longer pays for the forward's extra work.  Where nearly every row
+            # has at most 16 nonzeros the support lists replace the block backward.  One
+            # untimed forward of each kind measures the sparsity and the list coverage.
             A.entmax_attn_fwd(self.qd, self.kd, self.vd, w.alpha, w.causal, ws=self.wsf,
                               out=(self.o, self.tau, self.mask, None))
             sp0 = 1.0 - int(self.mask.sum().item()) / self.admissible
-            delta = "otilde" if sp0 < 0.5 else "recompute"
-            self.delta_why = f"auto: block sparsity {sp0:.3f} of an untimed forward (otilde below 0.5)"
+            cover = 0.0
+            if w.dtype == "bf16":
+                lists = A.alloc_lists(self.qd)
+                A.entmax_attn_fwd(self.qd, self.kd, self.vd, w.alpha, w.causal, ws=self.wsf,
+                                  out=(self.o, self.tau, self.mask, None), lists=lists)
+                cover = (lists[2] != 255).float().mean().item()
+                del lists
+            delta = "lists" if cover >= 0.9 else "otilde" if sp0 < 0.5 else "recompute"
+            self.delta_why = (f"auto: block sparsity {sp0:.3f}, rows with a support list "
+                              f"{cover:.3f} of an untimed forward")
         self.delta = delta
         # otilde = G V / sum g (float32, like q) when the backward takes delta from it
         self.ot = (torch.empty(self.qd.shape, dtype=torch.float32, device=dev)
                    if delta == "otilde" else None)
+        self.lists = A.alloc_lists(self.qd) if delta == "lists" else None
+        if delta == "lists":
+            self.wsb = A.workspace(capi.ent_attn_bwd_lists_workspace_size(B, H, N, d, dt_code), dev)
 
     def fwd(self, iters=None):
         from adaptive_sparse_flash_entmax_b200 import attention as A
         w = self.w
         A.entmax_attn_fwd(self.qd, self.kd, self.vd, w.alpha, w.causal, ws=self.wsf,
-                          out=(self.o, self.tau, self.mask, iters), otilde=self.ot)
+                          out=(self.o, self.tau, self.mask, iters), otilde=self.ot, lists=self.lists)
 
     def bwd(self):
         from adaptive_sparse_flash_entmax_b200 import attention as A
         w = self.w
         A.entmax_attn_bwd(self.qd, self.kd, self.vd, self.o, self.dod, self.tau, self.mask,
                           w.alpha, w.causal, ws=self.wsb, out=(self.dq, self.dk, self.dv),
-                          otilde=self.ot)
+                          otilde=self.ot, lists=self.lists)
 
     def step(self):
         self.fwd()
@@ -472,7 +486,9 @@ class Case:
         cb = A.read_status(self.wsb)
         blk = 2.0 * 128 * 128 * d
         fwd_flops = blk * (cf[0] + 2 * cf[1] + cf[5])
-        bwd_flops = blk * cb[4]
+        # block products of the backward kernels, plus 8 d flops per support-list entry
+        # (dP, dQ, dK and dV terms of one nonzero)
+        bwd_flops = blk * cb[4] + 8.0 * d * cb[7]
         live = int(self.mask.sum().item())
         itf = it.float()
         hist = torch.bincount(it.reshape(-1).long(), minlength=1).tolist()
@@ -631,9 +647,9 @@ def run_ours(args):
                 qq, kk, vv, dd = din[bset]
                 oo, tt, mm, g1, g2, g3 = dout[bset]
                 A.entmax_attn_fwd(qq, kk, vv, w.alpha, w.causal, ws=c.wsf, out=(oo, tt, mm, None),
-                                  otilde=ot)
+                                  otilde=ot, lists=c.lists)
                 A.entmax_attn_bwd(qq, kk, vv, oo, dd, tt, mm, w.alpha, w.causal, ws=c.wsb, otilde=ot,
-                                  out=(g1, g2, g3))
+                                  lists=c.lists, out=(g1, g2, g3))
                 done_cmp.append(torch.cuda.Event())
                 done_cmp[-1].record(s_cmp)
             with torch.cuda.stream(s_out):

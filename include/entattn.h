@@ -36,7 +36,7 @@
  *    the 128x128 block of P for query tile t and key block b holds a nonzero
  *    (blocks above the diagonal are 0 when causal).  The forward writes it;
  *    the backward reads it and skips exactly the 0 blocks.
- *  - Supported: 1 < alpha <= 2, d in {64, 128}, 1 <= N <= 130944 (any N; the
+ *  - Supported: 1 < alpha <= 2, d in {32, 64, 128}, 1 <= N <= 130944 (any N; the
  *    last tile may be ragged), B, H >= 0, B*H <= 65535.  B*H == 0 or N == 0 is a no-op returning ENT_OK.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
  *    legacy default stream).  Argument errors return synchronously before any
@@ -154,6 +154,46 @@ ent_status ent_attn_bwd_otilde(const void *q, const void *k, const void *v, cons
                                void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Support lists: the forward pair for rows with few nonzeros ("AdaSplash: Adaptive
+ * Sparse Flash Attention", Technical Deep Dive / Exploiting Sparsity -- skipping the
+ * zeros of P, here at the grain of single keys instead of 128x128 blocks).
+ *
+ * ent_attn_fwd_lists is ent_attn_fwd (same outputs, workspace, limits) that also
+ * records, for every query row, the keys j with p_ij > 0 and u_ij = x_ij - tau_i:
+ *   list_key int32 [B,H,N,cap], list_u float [B,H,N,cap] (cap = ent_attn_list_cap(),
+ *   16): entries 0 .. list_n-1 of the row, in no particular order (the rest of the
+ *   row is not written);
+ *   list_n uint8 [B,H,N]: the number of entries, or 255 when the row has more than
+ *   cap nonzeros (its list is then incomplete and must not be used).
+ * All three are caller-owned device buffers, required (NULL is ENT_EINVAL).  bf16
+ * inputs only (float32: ENT_EUNSUPPORTED).
+ *
+ * ent_attn_bwd_lists is ent_attn_bwd given those lists (and the tau and block_mask of
+ * the same forward): every query tile whose rows all have lists (list_n != 255) is
+ * done from its lists alone -- per listed key, dP = dO_i . v_j, then delta, dS and
+ * the dQ, dK, dV contributions, with no score recomputation -- and the remaining
+ * tiles by the block kernels of ent_attn_bwd.  Same outputs as ent_attn_bwd (up to
+ * fp32 summation order: dK and dV collect the list contributions by atomic adds).
+ * Its workspace: ent_attn_bwd_lists_workspace_size (ent_attn_bwd's plus one byte per
+ * query tile and two float [B,H,N,d] accumulators).
+ */
+int ent_attn_list_cap(void);
+size_t ent_attn_bwd_lists_workspace_size(int B, int H, int N, int d, int dtype);
+ent_status ent_attn_fwd_lists(const void *q, const void *k, const void *v,
+                              int B, int H, int N, int d, int dtype,
+                              float alpha, int causal,
+                              void *o, float *tau, uint8_t *block_mask, uint8_t *iters,
+                              int32_t *list_key, float *list_u, uint8_t *list_n,
+                              void *ws, size_t ws_bytes, void *stream);
+ent_status ent_attn_bwd_lists(const void *q, const void *k, const void *v,
+                              const int32_t *list_key, const float *list_u,
+                              const uint8_t *list_n, const void *dout, const float *tau,
+                              const uint8_t *block_mask,
+                              int B, int H, int N, int d, int dtype, float alpha, int causal,
+                              void *dq, void *dk, void *dv,
+                              void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Backward without a workspace argument.  The pages have no counterpart: this
  * is a library convenience.  It computes exactly what ent_attn_bwd computes
  * (same kernels, same arguments minus ws / ws_bytes) for callers that cannot
@@ -203,8 +243,12 @@ ent_status ent_attn_noalloc_read_status(long long *counters, void *stream);
  *   [3] query tiles processed,
  *   [4] block products issued by the backward kernels (all of them),
  *   [5] G.V block products of ent_attn_fwd_otilde (one per live block),
- *   [6]..[7] reserved (0).
- * Executed flops of a call = 2*128*128*d * ([0] + 2*[1] + [4] + [5]).
+ *   [6] key blocks a forward left out of its statistics pass because a centroid
+ *       bound rules them out for every row of the query tile (bf16 path; the
+ *       bound's own products, one per 128 centroids, are counted in [0]),
+ *   [7] support-list entries the backward of ent_attn_bwd_lists handled (8*d flops
+ *       each: the dP, dQ, dK and dV terms of one nonzero).
+ * Executed flops of a call = 2*128*128*d * ([0] + 2*[1] + [4] + [5]) + 8*d*[7].
  * Returns ENT_OK, ENT_ETIMEOUT if a bounded wait gave up, ENT_ECUDA on a
  * CUDA error.
  */

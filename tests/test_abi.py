@@ -77,7 +77,7 @@ def test_fwd_argument_errors(lib, kw, code):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(alpha=0.5), capi.ENT_EINVAL),
-    (dict(d=32), capi.ENT_EUNSUPPORTED),
+    (dict(d=256), capi.ENT_EUNSUPPORTED),
     (dict(tau=None), capi.ENT_EINVAL),
     (dict(dq=FAKE + 8), capi.ENT_EINVAL),
     (dict(ws_bytes=512), capi.ENT_EINVAL),   # needs 256 + 128 * 4
@@ -131,4 +131,4 @@ def test_otilde_argument_errors(lib, which):
     assert call(**args) == capi.ENT_EINVAL                 # null otilde
     assert "otilde" in capi.ent_attn_last_error()
     assert call(**dict(args, otilde=FAKE + 4)) == capi.ENT_EINVAL   # misaligned
-    assert call(**dict(args, d=32, otilde=FAKE)) == capi.ENT_EUNSUPPORTED
+    assert call(**dict(args, d=48, otilde=FAKE)) == capi.ENT_EUNSUPPORTED

@@ -27,6 +27,7 @@ CASES = [
     ("clustered4k", {"span": 128, "B": 1, "H": 4}, True),
     ("clustered4k", {"span": 128, "B": 1, "H": 2, "d": 64, "N": 1000}, True),      # ragged tail, d 64
     ("clustered4k", {"span": 64, "B": 1, "H": 2, "causal": False, "N": 2000}, True),  # non-causal
+    ("clustered4k", {"span": 128, "B": 1, "H": 2, "d": 32, "N": 900}, True),        # d 32
     ("long", {"H": 2}, True),
     ("iid", {"B": 1, "H": 4}, False),
 ]

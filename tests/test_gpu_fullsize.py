@@ -22,7 +22,8 @@ def _cuda():
 
 CASES = [("iid", {}, True), ("iid", {"beta": 8.0}, False), ("alpha", {"alpha": 1.25}, False),
          ("alpha", {"alpha": 2.0}, True), ("alpha", {}, True), ("long", {}, False),
-         ("long", {}, True), ("lm", {}, True), ("clustered4k", {"span": 128}, False)]
+         ("long", {}, True), ("lm", {}, True), ("clustered4k", {"span": 128}, False),
+         ("iid", {"d": 32}, True), ("clustered4k", {"span": 128, "d": 32}, False)]
 
 
 @pytest.mark.parametrize("name,change,with_otilde", CASES,

@@ -48,13 +48,20 @@ def test_tiny_fp32_workload():
 
 
 @pytest.mark.parametrize("N", [128, 300, 384])
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [32, 64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("alpha", [1.25, 1.5, 1.7, 2.0])
 def test_small_bf16(N, d, causal, alpha):
     w, (q, k, v, do) = inputs.small_case(B=1, H=2, N=N, d=d, causal=causal, alpha=alpha,
                                          beta=2.0, seed=N + d)
     full_parity(q, k, v, do, alpha, causal, "bf16")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_small_f32_d32(causal):
+    w, (q, k, v, do) = inputs.small_case(B=1, H=2, N=200, d=32, dtype="f32", causal=causal,
+                                         alpha=1.5, beta=2.0, seed=32)
+    full_parity(q, k, v, do, 1.5, causal, "f32")
 
 
 @pytest.mark.parametrize("alpha", [1.5, 2.0])
@@ -231,6 +238,12 @@ def test_workload_long_clustered():
 
 def test_workload_lm():
     _sampled_parity(inputs.WORKLOADS["lm"], early_keys=16)
+
+
+def test_workload_head_dim_32():
+    # the iid shape at d = 32 (run by the d = 64 kernels on zero-filled upper columns)
+    _sampled_parity(inputs.WORKLOADS["iid"].replace(d=32, beta=2.0), early_keys=16)
+    _sampled_parity(inputs.WORKLOADS["clustered4k"].replace(d=32, span=128), n_rows=32, early_keys=8)
 
 
 def test_workload_clustered4k_span_sweep():

@@ -85,11 +85,23 @@ __device__ __forceinline__ float entmax_g(float u, float gamma) {
     return exp2f((gamma - 1.f) * __log2f(u));
 }
 
-// Per-row solver state.
+// Per-row solver state.  `unv`: the row stopped on a Halley step it did not
+// evaluate (the forward verifies it afterwards); `down`: that step went down, so the
+// support may have grown past the blocks live in the last pass.
 struct RowSolver {
     float tau, lo, hi;
     int done;
     int iters;
+    int unv = 0;
+    int down = 0;
+};
+
+// Unverified-step rules of solver_update (all 0: every stop is at an evaluated tau).
+struct AcceptRule {
+    float up = 0.f;        // upward steps up to this size
+    float up_far = 0.f;    // upward steps up to this size when `cert` certifies them
+    float cert = 0.f;      // bound on what the support's leaving elements can change in f
+    float down = 0.f;      // downward steps up to this size
 };
 
 // One Halley-bisection update after a pass evaluated F0 = sum u^gamma,
@@ -99,16 +111,19 @@ struct RowSolver {
 // within the closed bracket [lo, hi] (a point that rounding put a few ulps
 // outside is clamped onto it: a root on a bracket end, such as tau = m - 1 for
 // a one-element support, must stay reachable); otherwise the bracket is bisected.
-// `accept` > 0 also stops on an upward Halley step of at most `accept` (absolute, in
-// x units), taking the new point without evaluating it: the root is then within the
-// step of it (Halley's error is cubic in the step between support changes), and since
-// tau only grew the support only shrank, so the live blocks marked in this pass still
-// cover every block with p > 0.  A block marked live whose elements all lie in
-// (tau_old, tau_new] has max(x - tau) > -accept, so with accept below the 1e-3 band of
-// the mask contract the mask stays exact outside that band at any |tau|.
+// The rule `acc` may also stop a row on a Halley step it takes without evaluating
+// it (near the root Halley's error is cubic in the step while the support stays
+// the same):
+//   upward by at most acc.up, or by at most acc.up_far when the elements that can
+//   leave the support (u <= step) change f by at most acc.cert: each adds at most
+//   step^gamma, so their total is below step^2 F2 (gamma >= 2) or step F1 (gamma < 2);
+//   downward by at most acc.down (elements may enter the support; the caller adds
+//   the blocks they can lie in).
+// Either way the caller checks f at the new tau afterwards.
 __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1, float F2,
                                               float gamma, bool gamma_is_one, int pass,
-                                              float ftol, float stol, float accept = 0.f) {
+                                              float ftol, float stol,
+                                              const AcceptRule& acc = AcceptRule()) {
     if (st.done) return;
     const float f = F0 - 1.f;
     if (fabsf(f) <= ftol || pass >= kMaxPass) { st.done = 1; st.iters = pass; return; }
@@ -120,9 +135,16 @@ __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1,
     const float tol = stol * scale;
     const bool halley = isfinite(h) && h >= st.lo - tol && h <= st.hi + tol;
     const float next = halley ? fminf(fmaxf(h, st.lo), st.hi) : 0.5f * (st.lo + st.hi);
-    if (fabsf(next - st.tau) <= tol) { st.done = 1; st.iters = pass; return; }
-    if (halley && next > st.tau && next - st.tau <= accept) {
-        st.tau = next; st.done = 1; st.iters = pass; return;
+    const float dl = next - st.tau;
+    if (fabsf(dl) <= tol) { st.done = 1; st.iters = pass; return; }
+    if (halley && dl > 0.f) {
+        const float leave = (gamma >= 2.f) ? F2 * dl * dl : F1 * dl;
+        if (dl <= acc.up || (dl <= acc.up_far && leave <= acc.cert)) {
+            st.tau = next; st.done = 1; st.unv = 1; st.iters = pass; return;
+        }
+    }
+    if (halley && dl < 0.f && -dl <= acc.down) {
+        st.tau = next; st.done = 1; st.unv = 1; st.down = 1; st.iters = pass; return;
     }
     st.tau = next;
 }

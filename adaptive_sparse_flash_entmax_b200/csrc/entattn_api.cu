@@ -66,7 +66,7 @@ int hist_budget() {
 // of the statistics pass: per head max |c| and min R (float bits), per 64-key
 // half-block {R, L} and the bf16 centroid.
 struct FwdLayout {
-    size_t maxc, minr, stats, cent, total;
+    size_t maxc, minr, stats, cent, fix, total;
 };
 
 FwdLayout fwd_layout(int B, int H, int N, int d) {
@@ -76,7 +76,8 @@ FwdLayout fwd_layout(int B, int H, int N, int d) {
     L.minr = L.maxc + BH * 4;
     L.stats = L.maxc + round_up(BH * 8, 256);
     L.cent = L.stats + round_up(BH * T2 * 8, 256);
-    L.total = L.cent + round_up(BH * T2 * (size_t)d * 2, 256);
+    L.fix = L.cent + round_up(BH * T2 * (size_t)d * 2, 256);   // [BH][T] flags of the second launch
+    L.total = L.fix + round_up(BH * T2 / 2, 256);
     return L;
 }
 
@@ -87,6 +88,29 @@ FwdLayout fwd_layout(int B, int H, int N, int d) {
 bool bound_enabled() {
     const char* v = getenv("ENTATTN_BOUND");
     return !(v && *v && atoi(v) == 0);
+}
+
+// Unverified Halley steps of the bf16 forward (each checked in the P.V pass, see
+// solver_update): upward up to 5e-4, or up to 1e-2 when the elements that can leave
+// the support change f by at most 2e-5; downward up to 1e-2.  ENTATTN_ACCEPT=0
+// (environment, read per call) stops every row at an evaluated tau instead, for
+// ablations.  ENTATTN_VERIFY_TOL sets the check's tolerance on |sum_j p - 1|
+// (default 1e-4; a negative value sends every tile with such a row through the
+// second launch, which tests that path).
+ent::AcceptRule accept_rule() {
+    ent::AcceptRule r;
+    const char* v = getenv("ENTATTN_ACCEPT");
+    if (v && *v && atoi(v) == 0) return r;
+    r.up = 5e-4f;
+    r.up_far = 1e-2f;
+    r.cert = 2e-5f;
+    r.down = 1e-2f;
+    return r;
+}
+
+float verify_tol() {
+    const char* v = getenv("ENTATTN_VERIFY_TOL");
+    return (v && *v) ? (float)atof(v) : 1e-4f;
 }
 
 // Backward workspace layout: the 256-byte header, then delta (one float per query row).
@@ -224,6 +248,11 @@ ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, i
     a.ftol = dtype == ENT_F32 ? 1e-6f : 1e-5f;
     a.stol = dtype == ENT_F32 ? 4e-7f : 1e-6f;
     a.hist_budget = hist_budget();
+    if (dtype == ENT_BF16) {
+        a.acc = accept_rule();
+        a.verify_tol = verify_tol();
+        a.fix_flags = reinterpret_cast<uint8_t*>(static_cast<char*>(ws) + FL.fix);
+    }
     if (bound) {
         // statistics-pass skipping by key-block bounds; off with the histogram start, whose
         // windows must count every score down to their lowest bin

@@ -28,6 +28,15 @@ struct FwdArgs {
     float ftol, stol;      // solver stop rule: |f| <= ftol, or a step <= stol*max(1,|tau|)
     int hist_budget;       // tensor-core path: histogram inserts a tile may make after its
                            // first block (0: no histogram, < 0: no limit)
+    // Unverified Halley steps (tensor-core path): the rule, and the check in the P.V pass
+    // (|sum_j p_ij - 1| <= verify_tol for every row that stopped on one).  A tile that
+    // fails it is flagged in fix_flags [BH][T] and solved again by a second launch with
+    // fix_mode = 1 (tiles not flagged return at once; that launch takes no unverified
+    // step).
+    AcceptRule acc;
+    float verify_tol;
+    uint8_t* fix_flags;
+    int fix_mode;
     float* otilde;         // nullable [BH][N][d] fp32: sum_j g_ij v_j / sum_j g_ij
     // Key-block bounds for skipping statistics-pass blocks (tensor-core path; all null:
     // no bound pass).  Per 64-key half-block hb of head bh (T2 = 2T of them):

@@ -60,9 +60,7 @@ constexpr int kTmemCols = 512;     // score passes: S [0,256), [256,512); P.V pa
                                    // S1 [128,256), O [256, 256+D), then either S2 [384, 512)
                                    // or, with otilde, G.V [256+D, 256+2D) (and S2 when D = 64)
 constexpr int kDecSolve = 1, kDecPv = 2;
-// Largest upward Halley step taken without a verifying pass (x units; below the 1e-3
-// band within which the block mask may differ from the exact one).
-constexpr float kAcceptStep = 5e-4f;
+constexpr uint8_t kPvLive = 255;   // cand[] of a block with a nonzero p in the P.V pass
 
 __host__ __device__ constexpr uint32_t sbuf_col(int sb) { return sb < 2 ? sb * 128 : 384; }
 
@@ -163,6 +161,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int T = a.T, N = a.N;
     const int t = a.causal ? (T - 1 - (int)blockIdx.x) : (int)blockIdx.x;   // long tiles first
     const int bh = blockIdx.y;
+    // the second launch solves again only the tiles the first one flagged
+    if (a.fix_mode && !a.fix_flags[(size_t)bh * T + t]) return;
     const int nblk = a.causal ? t + 1 : T;
     const Abort ab{&misc->abort, a.hdr};
     constexpr int SB = (OT && D == 128) ? 2 : kSbuf;   // S buffers of the P.V pass
@@ -716,11 +716,15 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 X(0, half) = F0; X(1, half) = F1; X(2, half) = F2;
                 named_bar(1, kEw);
                 const float G0 = F0 + X(0, half ^ 1), G1 = F1 + X(1, half ^ 1), G2 = F2 + X(2, half ^ 1);
-                solver_update(sv, G0, G1, G2, gamma, gamma == 1.f, pass, a.ftol, a.stol, kAcceptStep);
+                solver_update(sv, G0, G1, G2, gamma, gamma == 1.f, pass, a.ftol, a.stol, a.acc);
             }
             const int all = named_bar_and(1, kEw, sv.done) && pass > 0;
+            // after an unverified downward step the support may reach blocks that were not
+            // live in this pass: the P.V pass then also visits the candidates at the final
+            // tau (a uniform barrier, since `all` is)
+            const bool any_down = all && !named_bar_and(1, kEw, !(row_valid && sv.down));
             const uint8_t tag = (uint8_t)(pass + 2);
-            if (!all) {
+            if (!all || any_down) {
                 // Candidates for the next pass: a block can hold u > 0 for a row of this
                 // warp only if the warp's block maximum exceeds the warp's smallest tau.
                 float th = row_valid ? sv.tau : INFINITY;
@@ -736,7 +740,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 int n = 0;
                 for (int base = 0; base < nblk; base += 32) {
                     const int bb = base + lane;
-                    const bool f = bb < nblk && (all ? live[bb] != 0 : cand[bb] == tag);
+                    const bool f = bb < nblk && (all ? (live[bb] != 0 || (any_down && cand[bb] == tag))
+                                                     : cand[bb] == tag);
                     const unsigned int msk = __ballot_sync(0xffffffffu, f);
                     if (f) job_list[n + __popc(msk & ((1u << lane) - 1u))] = bb;
                     n += __popc(msk);
@@ -751,6 +756,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         const int npass = pass;
         [[maybe_unused]] float2 sg2 = make_float2(0.f, 0.f);   // sum_j g of this half-row (OT)
+        float2 fsum2 = make_float2(0.f, 0.f);                   // sum_j p of this half-row
         if (ok) {
             named_bar(1, kEw);   // job_list / njobs of the P.V pass visible to the group
             nlive = misc->njobs;
@@ -769,38 +775,46 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                     for (int c = 0; c < 64; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
                 }
-                uint32_t pk[32];
-                [[maybe_unused]] uint32_t gk[32];
                 const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-sv.tau, -sv.tau);
+                uint32_t nzb = 0u;   // OR of this thread's bf16 p bits: nonzero iff some p > 0
+                // two rounds of 32 keys; P of keys c0 + 32 hc .. + 31 goes over this thread's
+                // own S columns c0 + 16 hc .. + 15 (G, with otilde, 32 columns further on)
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const float2 u2 = __ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2);
-                    if constexpr (OT) {
-                        float2 p2, g2;
-                        entmax_pg_x2<GM>(u2, gamma, p2, g2);
-                        const __nv_bfloat162 hp = __floats2bfloat162_rn(p2.x, p2.y);
-                        const __nv_bfloat162 hg = __floats2bfloat162_rn(g2.x, g2.y);
-                        pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
-                        gk[c >> 1] = *reinterpret_cast<const uint32_t*>(&hg);
-                        // sum the rounded weights the G.V product uses: otilde is then
-                        // a weighted mean whose weights sum to one
-                        sg2 = __fadd2_rn(sg2, __bfloat1622float2(hg));
-                    } else {
-                        const float2 p2 = entmax_p_x2<GM>(u2, gamma);
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p2.x, p2.y);
-                        pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+                for (int hc = 0; hc < 2; ++hc) {
+                    uint32_t pk[16];
+                    [[maybe_unused]] uint32_t gk[16];
+#pragma unroll
+                    for (int c2 = 0; c2 < 32; c2 += 2) {
+                        const int c = 32 * hc + c2;
+                        const float2 u2 = __ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2);
+                        if constexpr (OT) {
+                            float2 p2, g2;
+                            entmax_pg_x2<GM>(u2, gamma, p2, g2);
+                            fsum2 = __fadd2_rn(fsum2, p2);
+                            const __nv_bfloat162 hp = __floats2bfloat162_rn(p2.x, p2.y);
+                            const __nv_bfloat162 hg = __floats2bfloat162_rn(g2.x, g2.y);
+                            pk[c2 >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
+                            gk[c2 >> 1] = *reinterpret_cast<const uint32_t*>(&hg);
+                            // sum the rounded weights the G.V product uses: otilde is then
+                            // a weighted mean whose weights sum to one
+                            sg2 = __fadd2_rn(sg2, __bfloat1622float2(hg));
+                        } else {
+                            const float2 p2 = entmax_p_x2<GM>(u2, gamma);
+                            fsum2 = __fadd2_rn(fsum2, p2);
+                            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p2.x, p2.y);
+                            pk[c2 >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+                        }
                     }
-                }
-                if (a.list_n) {
-                    // support list of the row: (key, u) for every p > 0 (a bf16 p is nonzero
-                    // exactly when its bits are; most threads see none in a block)
                     uint32_t nzw = 0u;
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) nzw |= pk[c];
-                    if (nzw != 0u) {
+                    for (int c = 0; c < 16; ++c) nzw |= pk[c];
+                    nzb |= nzw;
+                    if (a.list_n && nzw != 0u) {
+                        // support list of the row: (key, u) for every p > 0 of these keys
                         const size_t lbase = ((size_t)bh * N + i) * kListCap;
 #pragma unroll
-                        for (int c = 0; c < 64; ++c) {
+                        for (int c2 = 0; c2 < 32; ++c2) {
+                            const int c = 32 * hc + c2;
                             const float u = __fmaf_rn(s[c], cx, -sv.tau);
                             if (u > 0.f) {
                                 const int slot = atomicAdd(&lcnt[row], 1);
@@ -811,11 +825,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             }
                         }
                     }
+                    tmem_st16(lane_base + sbuf_col(sb) + c0 + 16 * hc, pk);
+                    if constexpr (OT) tmem_st16(lane_base + sbuf_col(sb) + c0 + 32 + 16 * hc, gk);
                 }
-                // P over this thread's own S columns: keys c0 .. c0+63 -> columns c0 .. c0+31
-                // (and G, with otilde, -> columns c0+32 .. c0+63)
-                tmem_st32(lane_base + sbuf_col(sb) + c0, pk);
-                if constexpr (OT) tmem_st32(lane_base + sbuf_col(sb) + c0 + 32, gk);
+                // the block mask: some p > 0 in the block at the final tau (a bf16 p is
+                // nonzero exactly when its bits are)
+                if (__any_sync(0xffffffffu, nzb != 0u) && lane == 0) cand[b] = kPvLive;
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -890,8 +905,17 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 a.list_n[(size_t)bh * N + i] = (ok && n <= kListCap) ? (uint8_t)n : kListOver;
             }
         }
+        // verification of the rows that stopped on an unevaluated step: f at the final tau
+        // is sum_j p_ij - 1, summed above over a superset of the support; a tile where one
+        // such row misses the tolerance is solved again by the second launch
+        X(3, half) = fsum2.x + fsum2.y;
+        named_bar(1, kEw);   // also: every warp's P.V-pass mask flags are in
+        const float f_end = X(3, 0) + X(3, 1) - 1.f;
+        const bool bad = ok && row_valid && sv.unv && !(fabsf(f_end) <= a.verify_tol);
+        const bool tile_bad = !named_bar_and(1, kEw, !bad);
+        if (!a.fix_mode && ew == 0) a.fix_flags[(size_t)bh * T + t] = tile_bad ? 1 : 0;
         uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
-        for (int bb = ew; bb < T; bb += kEw) mrow[bb] = (bb < nblk) ? live[bb] : 0;
+        for (int bb = ew; bb < T; bb += kEw) mrow[bb] = (bb < nblk && cand[bb] == kPvLive) ? 1 : 0;
         if (ew == 0) {
             atomicAdd(&a.hdr->counters[kCtrQkBlocks], (unsigned long long)qk_blocks);
             atomicAdd(&a.hdr->counters[kCtrPvBlocks], (unsigned long long)nlive);
@@ -1064,6 +1088,12 @@ static cudaError_t launch_tc_fwd(const CUtensorMap& mq, const CUtensorMap& mk,
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(mq, mk, mv, mc, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // tiles whose verification failed, solved again with evaluated stops only
+    FwdArgs f = a;
+    f.fix_mode = 1;
+    f.acc = AcceptRule();
+    kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(mq, mk, mv, mc, f);
     return cudaGetLastError();
 }
 

@@ -392,8 +392,17 @@ def combine_ranks(ms: float, units: float, world: int, device) -> tuple:
     return t.item(), u.item()
 
 
-# GPU kernels launched per step (forward: one; backward: dq and dkv)
-LAUNCHES_PER_STEP = {"bf16": 3, "f32": 4}
+def launches_per_step(dtype, delta):
+    """Kernels of this library launched per step.  bf16: the key-block statistics (unless
+    ENTATTN_BOUND=0 or the histogram start is selected), the forward and its second
+    launch for tiles that failed verification (it returns at once for the others), the
+    support-list backward (lists only), dq and dkv.  float32: the forward and three
+    backward kernels."""
+    if dtype != "bf16":
+        return 4
+    hb = os.environ.get("ENTATTN_HIST_BUDGET")
+    bound = os.environ.get("ENTATTN_BOUND", "1") != "0" and (not hb or int(hb) == 0)
+    return int(bound) + 2 + (1 if delta == "lists" else 0) + 2
 
 SWEEP = ([("iid", {"beta": b}) for b in (1.0, 2.0, 4.0, 8.0)]
          + [("alpha", {"alpha": a}) for a in (1.25, 1.5, 2.0)]
@@ -710,7 +719,7 @@ def run_ours(args):
     roof["traffic"] = profiled_traffic(w, roof["kernel"].split(":")[0],
                                        "otilde" if ot is not None else "plain")
     value = flops_all / (ms_step * 1e-3) / 1e12
-    c_why = c.delta_why
+    c_why, c_delta = c.delta_why, c.delta
     del c
     torch.cuda.empty_cache()
     sweep = None
@@ -756,7 +765,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": {"value": flops_all / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-            "gpu_launches": LAUNCHES_PER_STEP[w.dtype] * args.steps,
+            "gpu_launches": launches_per_step(w.dtype, c_delta) * args.steps,
             "clocks": clocks,
             "timed_region_s": timed_region_s,
             "peaks": {"source": peak_kind, "bf16_tflops": peaks["bf16_tflops"],

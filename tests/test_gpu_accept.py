@@ -1,0 +1,75 @@
+"""Unevaluated Halley stops of the bf16 forward and their check.
+
+A row may stop on a Halley step it does not evaluate (upward up to 5e-4, or up to 1e-2
+when the elements that can leave the support change f by at most 2e-5; downward up to
+1e-2); the P.V pass then sums p at the final tau, and a tile where such a row misses
+|sum p - 1| <= 1e-4 is solved again by a second launch that stops only at evaluated
+points.  Checked here: the oracle parity of the default rule (small cases, every
+alpha), fewer solver passes than with evaluated stops only, and the second launch: with
+a negative tolerance every such tile goes through it, and the outputs are then
+bit-identical to those of evaluated stops only (ENTATTN_ACCEPT=0)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from adaptive_sparse_flash_entmax_b200 import attention as A
+from adaptive_sparse_flash_entmax_b200 import capi, inputs
+
+from parity import check_mask, check_o, check_tau, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    capi.load()
+
+
+def _fwd(w, qd, kd, vd, otilde=False):
+    B, H, N, d = w.shape
+    ws = A.workspace(capi.ent_attn_fwd_workspace_size(B, H, N, d, capi.ENT_BF16), qd.device)
+    ot = torch.empty(qd.shape, dtype=torch.float32, device=qd.device) if otilde else None
+    o, tau, mask, it = A.entmax_attn_fwd(qd, kd, vd, w.alpha, w.causal, ws=ws, with_iters=True,
+                                         otilde=ot)
+    return (o, tau, mask, it, ot), A.read_status(ws)
+
+
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0])
+@pytest.mark.parametrize("name", ["iid", "lm"])
+def test_fewer_passes_same_contract(name, alpha, monkeypatch):
+    w = inputs.WORKLOADS[name].replace(B=1, alpha=alpha, **({"H": 4} if name == "iid" else {}))
+    q, k, v, _ = inputs.make_inputs(w, seed=8)
+    qd, kd, vd = (to_dev(a, "bf16") for a in (q, k, v))
+    monkeypatch.delenv("ENTATTN_ACCEPT", raising=False)
+    (o, tau, mask, it, _), c1 = _fwd(w, qd, kd, vd)
+    monkeypatch.setenv("ENTATTN_ACCEPT", "0")
+    _, c0 = _fwd(w, qd, kd, vd)
+    assert c1[2] <= c0[2]                       # solver passes summed over tiles
+    assert c1[3] == c0[3]                       # no tile needed the second launch
+    # the first head against the oracle: tau, O and the block mask, every row
+    sel = lambda a: np.ascontiguousarray(a[:1, :1])
+    o_ref, tau_ref, marg = oracle.attn_fwd(sel(q), sel(k), sel(v), w.alpha, w.causal)
+    check_tau(sel(to_np(tau)), tau_ref)
+    check_o(sel(to_np(o)), o_ref, "bf16")
+    check_mask(sel(to_np(mask)), marg)
+
+
+@pytest.mark.parametrize("otilde", [False, True])
+@pytest.mark.parametrize("name,change", [("iid", {"B": 1, "H": 4}), ("long", {"H": 2}),
+                                         ("alpha", {"B": 1, "H": 2, "alpha": 1.25})])
+def test_second_launch_matches_evaluated_stops(name, change, otilde, monkeypatch):
+    w = inputs.WORKLOADS[name].replace(**change)
+    q, k, v, _ = inputs.make_inputs(w, seed=9)
+    qd, kd, vd = (to_dev(a, "bf16") for a in (q, k, v))
+    monkeypatch.setenv("ENTATTN_VERIFY_TOL", "-1")
+    forced, cf = _fwd(w, qd, kd, vd, otilde)
+    monkeypatch.delenv("ENTATTN_VERIFY_TOL")
+    monkeypatch.setenv("ENTATTN_ACCEPT", "0")
+    plain, c0 = _fwd(w, qd, kd, vd, otilde)
+    for a, b in zip(forced, plain):
+        if a is not None:
+            assert torch.equal(a, b)
+    assert cf[3] > c0[3]                        # tiles went through the second launch

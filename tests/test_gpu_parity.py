@@ -154,7 +154,8 @@ def test_counters_and_status():
     o, tau, mask, _ = A.entmax_attn_fwd(qd, kd, vd, 1.5, True, ws=ws)
     ctr = A.read_status(ws)
     assert ctr[3] == 2 * 2 * 4                           # query tiles
-    assert ctr[1] == int(mask.sum())                     # P.V blocks == live blocks
+    assert ctr[1] >= int(mask.sum())                     # P.V blocks: the live ones and, after
+                                                         # an unevaluated downward stop, candidates
     causal_blocks = 2 * 2 * (1 + 2 + 3 + 4)
     assert ctr[0] >= 2 * causal_blocks                   # stats pass + at least one solver pass
     assert ctr[2] >= ctr[3]                              # every tile ran >= 1 solver pass

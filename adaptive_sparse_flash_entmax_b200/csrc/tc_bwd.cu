@@ -65,6 +65,16 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// 4-byte asynchronous copy global -> shared, and an arrive on `bar` once every earlier
+// cp.async of this thread has landed (the arrival counts toward the barrier's expected
+// count, which includes it).
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<const uint32_t*>(&h);
@@ -492,8 +502,8 @@ struct DkvLayout {
     static constexpr int kV = kK + kTile;
     static constexpr int kStage0 = kV + kTile;
     static constexpr int kStageBytes = 2 * kSubT;       // Q_sub, dO_sub
-    static constexpr int kTauDelta = kStage0 + kNst * kStageBytes;   // [2][2][64] floats
-    static constexpr int kBars = kTauDelta + 4 * 64 * 4;
+    static constexpr int kTauDelta = kStage0 + kNst * kStageBytes;   // [kNst][tau|delta][64] floats
+    static constexpr int kBars = kTauDelta + kNst * 2 * 64 * 4;
     static constexpr int kMisc = kBars + 8 * 24;   // up to 24 mbarriers
     static constexpr int kList = kMisc + 16;
     static size_t bytes(int T) { return (size_t)kList + 8 * (size_t)T + 1024; }
@@ -518,7 +528,7 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint64_t* mma_done = in_full + 1;
     Misc* misc = reinterpret_cast<Misc*>(smem + L::kMisc);
     int* jobs = reinterpret_cast<int*>(smem + L::kList);   // row offsets of the 64-row sub-tiles
-    float* td = reinterpret_cast<float*>(smem + L::kTauDelta);   // [buf][tau|delta][64]
+    float* td = reinterpret_cast<float*>(smem + L::kTauDelta);   // [stage][tau|delta][64]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, N = a.N;
@@ -527,7 +537,9 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const Abort ab{&misc->abort, a.hdr};
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kNst; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        // a stage is full once its Q/dO tiles (TMA, one arrival with the byte count) and
+        // its tau/delta (cp.async by the 32 producer lanes, one arrival each) have landed
+        for (int s = 0; s < kNst; ++s) { mbar_init(&full[s], 1 + 32); mbar_init(&empty[s], 1); }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&s_free[s], 1);
@@ -589,13 +601,17 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const uint32_t tm_dv = tmem + 256, tm_dk = tmem + 256 + D;
 
     if (warp == 0) {
-        if (lane == 0) {
-            int job = 0;
-            bool ok = true;
-            for (; job < njobs && ok; ++job) {
-                const int i0 = jobs[job];
-                const int st = job % kNst;
-                if (!(ok = mbar_wait(&empty[st], ((job / kNst) & 1) ^ 1, ab, 31))) break;
+        // the whole warp: lane 0 waits for the stage and issues the Q/dO tiles, every lane
+        // copies two of the sub-tile's 64 tau and delta values
+        int job = 0;
+        bool ok = true;
+        for (; job < njobs && ok; ++job) {
+            const int i0 = jobs[job];
+            const int st = job % kNst;
+            if (lane == 0) ok = mbar_wait(&empty[st], ((job / kNst) & 1) ^ 1, ab, 31);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane == 0) {
                 uint8_t* sb = smem + L::kStage0 + st * L::kStageBytes;
                 mbar_arrive_expect_tx(&full[st], 2 * L::kSubT);
                 for (int at = 0; at < D / 64; ++at) {
@@ -603,6 +619,17 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     tma_load_3d(sb + L::kSubT + at * kAtom64, &tm_do64, at * 64, i0, bh, &full[st]);
                 }
             }
+            // rows past N copy row N-1 (finite values for columns the elementwise warps mask)
+            float* tds = td + st * 128;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int ii = min(i0 + lane + 32 * r, N - 1);
+                cp_async_4(tds + lane + 32 * r, a.tau + (size_t)bh * N + ii);
+                cp_async_4(tds + 64 + lane + 32 * r, a.delta + (size_t)bh * N + ii);
+            }
+            cp_async_arrive_noinc(&full[st]);
+        }
+        if (lane == 0) {
             drain_wait(in_full, 0);
             for (int j = job - 1; j >= 0 && j >= job - kNst; --j) drain_wait(&full[j % kNst], (j / kNst) & 1);
         }
@@ -671,28 +698,14 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + half * 32;
         const float gamma = a.gamma, cx = a.cx;
         bool ok = true;
-        // -tau, -delta of the sub-tile's 64 query rows, loaded one job ahead
-        float ntau_n = 0.f, ndel_n = 0.f;
-        auto load_td = [&](int jj) {
-            const int ii = jobs[jj] + ew;
-            ntau_n = ii < N ? -a.tau[(size_t)bh * N + ii] : 0.f;
-            ndel_n = ii < N ? -a.delta[(size_t)bh * N + ii] : 0.f;
-        };
-        if (ew < 64 && njobs > 0) load_td(0);
         for (int j = 0; j < njobs; ++j) {
             const int i0 = jobs[j];
-            float* tdb = td + (j & 1) * 128;
-            if (ew < 64) {
-                tdb[ew] = ntau_n;
-                tdb[64 + ew] = ndel_n;
-                if (j + 1 < njobs) load_td(j + 1);
-            }
-            // the group agrees on `ok` at its barrier: a wait that gave up in the previous
-            // job makes every thread leave here together
-            ok = named_bar_and(1, kEw, ok);
-            if (!ok) break;
+            const int st = j % kNst;
             const int sbuf = j & 1;
-            if (!(ok = mbar_wait(&s_full[sbuf], (j >> 1) & 1, ab, 36))) continue;
+            // tau and delta of the sub-tile arrive with its stage (the MMA waited for the
+            // same phase before S^T); this wait makes the copies visible here
+            if (!(ok = mbar_wait(&full[st], (j / kNst) & 1, ab, 37))) break;
+            if (!(ok = mbar_wait(&s_full[sbuf], (j >> 1) & 1, ab, 36))) break;
             tc_fence_after();
             float s[32], dp[32];
             tmem_ld32(lane_base + sbuf * 128, &s[0]);
@@ -704,7 +717,7 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             const int ib = i0 + half * 32;
             const int cmin = a.causal ? jkey - ib : 0;       // c >= cmin
             const int cmax = min(32, N - ib);                // c < cmax
-            const float* tcol = tdb + half * 32;
+            const float* tcol = td + st * 128 + half * 32;   // tau, then delta 64 floats on
             if (!__all_sync(0xffffffffu, key_valid && cmin <= 0 && cmax >= 32)) {
                 // diagonal or ragged sub-tile: inadmissible columns get s = -inf (u < 0)
 #pragma unroll
@@ -715,8 +728,10 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             const float2 cx2 = make_float2(cx, cx);
 #pragma unroll
             for (int c = 0; c < 32; c += 4) {
-                const float4 ntq = *reinterpret_cast<const float4*>(tcol + c);        // -tau
-                const float4 ndl = *reinterpret_cast<const float4*>(tcol + 64 + c);   // -delta
+                const float4 tq = *reinterpret_cast<const float4*>(tcol + c);
+                const float4 dl = *reinterpret_cast<const float4*>(tcol + 64 + c);
+                const float4 ntq = make_float4(-tq.x, -tq.y, -tq.z, -tq.w);
+                const float4 ndl = make_float4(-dl.x, -dl.y, -dl.z, -dl.w);
                 float2 p0, g0, p1, g1;
                 entmax_pg_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, make_float2(ntq.x, ntq.y)),
                                  gamma, p0, g0);

@@ -810,17 +810,22 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int c = 0; c < 16; ++c) nzw |= pk[c];
                     nzb |= nzw;
                     if (a.list_n && nzw != 0u) {
-                        // support list of the row: (key, u) for every p > 0 of these keys
+                        // support list of the row: (key, u) for every p > 0 of these keys,
+                        // found word by word (a packed pair is nonzero iff one of its p is)
                         const size_t lbase = ((size_t)bh * N + i) * kListCap;
 #pragma unroll
-                        for (int c2 = 0; c2 < 32; ++c2) {
-                            const int c = 32 * hc + c2;
-                            const float u = __fmaf_rn(s[c], cx, -sv.tau);
-                            if (u > 0.f) {
-                                const int slot = atomicAdd(&lcnt[row], 1);
-                                if (slot < kListCap) {
-                                    a.list_key[lbase + slot] = b * kBlk + c0 + c;
-                                    a.list_u[lbase + slot] = u;
+                        for (int w = 0; w < 16; ++w) {
+                            if (pk[w] == 0u) continue;
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int c = 32 * hc + 2 * w + e;
+                                const float u = __fmaf_rn(s[c], cx, -sv.tau);
+                                if (u > 0.f) {
+                                    const int slot = atomicAdd(&lcnt[row], 1);
+                                    if (slot < kListCap) {
+                                        a.list_key[lbase + slot] = b * kBlk + c0 + c;
+                                        a.list_u[lbase + slot] = u;
+                                    }
                                 }
                             }
                         }

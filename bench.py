@@ -55,8 +55,8 @@ def parse():
                    help="backward path: delta from the forward's otilde (ent_attn_fwd_otilde + "
                         "ent_attn_bwd_otilde), recomputed by a pass over the keys, the support "
                         "lists (ent_attn_fwd_lists + ent_attn_bwd_lists), or auto: lists when an "
-                        "untimed forward leaves >= 90%% of the query rows with a list, else "
-                        "otilde below 50%% empty blocks, else recompute")
+                        "untimed forward gives >= 90%% of the query tiles a list for every row, "
+                        "else otilde below 50%% empty blocks, else recompute")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--B", type=int, default=None, help="override the batch (profiling cases)")
     p.add_argument("--H", type=int, default=None, help="override the head count")
@@ -452,11 +452,16 @@ class Case:
                 lists = A.alloc_lists(self.qd)
                 A.entmax_attn_fwd(self.qd, self.kd, self.vd, w.alpha, w.causal, ws=self.wsf,
                                   out=(self.o, self.tau, self.mask, None), lists=lists)
-                cover = (lists[2] != 255).float().mean().item()
+                # fraction of query tiles whose rows all have lists (the list kernel's tiles)
+                ln = lists[2]
+                T_ = -(-N // 128)
+                pad = torch.full((B, H, T_ * 128), 0, dtype=torch.uint8, device=dev)
+                pad[:, :, :N] = ln
+                cover = (pad.view(B, H, T_, 128) != 255).all(dim=3).float().mean().item()
                 del lists
             delta = "lists" if cover >= 0.9 else "otilde" if sp0 < 0.5 else "recompute"
-            self.delta_why = (f"auto: block sparsity {sp0:.3f}, rows with a support list "
-                              f"{cover:.3f} of an untimed forward")
+            self.delta_why = (f"auto: block sparsity {sp0:.3f}, query tiles with every row's "
+                              f"support list {cover:.3f}, of untimed forwards")
         self.delta = delta
         # otilde = G V / sum g (float32, like q) when the backward takes delta from it
         self.ot = (torch.empty(self.qd.shape, dtype=torch.float32, device=dev)

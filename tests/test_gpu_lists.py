@@ -83,7 +83,8 @@ def test_small_all_list_tiles(d, causal, alpha):
     check_tau(gpu["tau"], tau_ref)
     check_o(gpu["o"], o_ref, "bf16")
     assert check_lists(q, k, gpu["tau"], lists, alpha, causal) > 0
-    if alpha != 2.0:
+    assert tiles.any()
+    if alpha >= 1.5:       # alpha 1.25 keeps more than 16 nonzeros in some rows
         assert tiles.all()
     check_grads(gpu, oracle.attn_bwd(q, k, v, do, alpha, causal)[:3])
 

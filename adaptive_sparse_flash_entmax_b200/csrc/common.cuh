@@ -27,8 +27,8 @@ constexpr int kMaxPass = 24;       // solver pass cap (bisection alone needs ~20
 struct WsHeader {
     unsigned int status;           // 0 = ok, 1 = a bounded wait gave up
     unsigned int timeout_site;     // where it gave up (debug)
-    unsigned int tile_counter;     // persistent-scheduler work counter
-    unsigned int pad0;
+    unsigned int tile_counter;     // forward: CTAs finished (the last one re-solves failed tiles)
+    unsigned int fail_count;       // forward: tiles on the failure list
     unsigned long long counters[8];
     unsigned char pad1[256 - 16 - 64];
 };
@@ -98,10 +98,9 @@ struct RowSolver {
 
 // Unverified-step rules of solver_update (all 0: every stop is at an evaluated tau).
 struct AcceptRule {
-    float up = 0.f;        // upward steps up to this size
-    float up_far = 0.f;    // upward steps up to this size when `cert` certifies them
-    float cert = 0.f;      // bound on what the support's leaving elements can change in f
-    float down = 0.f;      // downward steps up to this size
+    float step = 0.f;      // largest step, either way
+    float cert = 0.f;      // bound on the change in f from elements crossing the support
+                           // boundary within the step
 };
 
 // One Halley-bisection update after a pass evaluated F0 = sum u^gamma,
@@ -112,13 +111,13 @@ struct AcceptRule {
 // outside is clamped onto it: a root on a bracket end, such as tau = m - 1 for
 // a one-element support, must stay reachable); otherwise the bracket is bisected.
 // The rule `acc` may also stop a row on a Halley step it takes without evaluating
-// it (near the root Halley's error is cubic in the step while the support stays
-// the same):
-//   upward by at most acc.up, or by at most acc.up_far when the elements that can
-//   leave the support (u <= step) change f by at most acc.cert: each adds at most
-//   step^gamma, so their total is below step^2 F2 (gamma >= 2) or step F1 (gamma < 2);
-//   downward by at most acc.down (elements may enter the support; the caller adds
-//   the blocks they can lie in).
+// it: near the root Halley's error is cubic in the step while the support stays the
+// same, so what the step can miss is the change of support.  Each element that
+// crosses the boundary within a step h changes f by at most h^gamma.  Upward, only
+// elements of the support (u <= h) can leave: together at most h^2 F2 (gamma >= 2) or
+// h F1 (gamma < 2), from the sums just evaluated.  Downward, the elements that can
+// enter are not counted by the sums; the step is taken when h^min(gamma,2) alone is
+// below the bound (a handful of entering elements stays within the caller's check).
 // Either way the caller checks f at the new tau afterwards.
 __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1, float F2,
                                               float gamma, bool gamma_is_one, int pass,
@@ -137,14 +136,13 @@ __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1,
     const float next = halley ? fminf(fmaxf(h, st.lo), st.hi) : 0.5f * (st.lo + st.hi);
     const float dl = next - st.tau;
     if (fabsf(dl) <= tol) { st.done = 1; st.iters = pass; return; }
-    if (halley && dl > 0.f) {
-        const float leave = (gamma >= 2.f) ? F2 * dl * dl : F1 * dl;
-        if (dl <= acc.up || (dl <= acc.up_far && leave <= acc.cert)) {
-            st.tau = next; st.done = 1; st.unv = 1; st.iters = pass; return;
+    if (halley && fabsf(dl) <= acc.step) {
+        const float h = fabsf(dl);
+        const float cross = (dl > 0.f) ? ((gamma >= 2.f) ? F2 * h * h : F1 * h)
+                                       : ((gamma >= 2.f) ? h * h : exp2f(gamma * __log2f(h)));
+        if (cross <= acc.cert) {
+            st.tau = next; st.done = 1; st.unv = 1; st.down = dl < 0.f; st.iters = pass; return;
         }
-    }
-    if (halley && dl < 0.f && -dl <= acc.down) {
-        st.tau = next; st.done = 1; st.unv = 1; st.down = 1; st.iters = pass; return;
     }
     st.tau = next;
 }

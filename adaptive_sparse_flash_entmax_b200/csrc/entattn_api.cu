@@ -76,8 +76,8 @@ FwdLayout fwd_layout(int B, int H, int N, int d) {
     L.minr = L.maxc + BH * 4;
     L.stats = L.maxc + round_up(BH * 8, 256);
     L.cent = L.stats + round_up(BH * T2 * 8, 256);
-    L.fix = L.cent + round_up(BH * T2 * (size_t)d * 2, 256);   // [BH][T] flags of the second launch
-    L.total = L.fix + round_up(BH * T2 / 2, 256);
+    L.fix = L.cent + round_up(BH * T2 * (size_t)d * 2, 256);   // failure list, one int per tile
+    L.total = L.fix + round_up(BH * T2 / 2 * 4, 256);
     return L;
 }
 
@@ -91,20 +91,18 @@ bool bound_enabled() {
 }
 
 // Unverified Halley steps of the bf16 forward (each checked in the P.V pass, see
-// solver_update): upward up to 5e-4, or up to 1e-2 when the elements that can leave
-// the support change f by at most 2e-5; downward up to 1e-2.  ENTATTN_ACCEPT=0
+// solver_update): steps up to 1e-2 either way whose boundary crossings can change f by
+// at most 1e-5 (upward from the sums, downward per entering element).  ENTATTN_ACCEPT=0
 // (environment, read per call) stops every row at an evaluated tau instead, for
-// ablations.  ENTATTN_VERIFY_TOL sets the check's tolerance on |sum_j p - 1|
-// (default 1e-4; a negative value sends every tile with such a row through the
-// second launch, which tests that path).
+// ablations.  ENTATTN_VERIFY_TOL sets the check's tolerance on |sum_j p - 1| (default
+// 1e-4; a negative value makes every tile with such a row be solved again, which
+// tests that path).
 ent::AcceptRule accept_rule() {
     ent::AcceptRule r;
     const char* v = getenv("ENTATTN_ACCEPT");
     if (v && *v && atoi(v) == 0) return r;
-    r.up = 5e-4f;
-    r.up_far = 1e-2f;
-    r.cert = 2e-5f;
-    r.down = 1e-2f;
+    r.step = 1e-2f;
+    r.cert = 1e-5f;
     return r;
 }
 
@@ -226,7 +224,9 @@ ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, i
         return fail(ENT_EINVAL, "null list_key/list_u/list_n pointer");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const FwdLayout FL = fwd_layout(B, H, N, d);
-    const bool bound = dtype == ENT_BF16 && hist_budget() == 0 && bound_enabled() && !empty;
+    // (no tile of a shorter sequence runs the bound pass, so its statistics are not computed)
+    const bool bound = dtype == ENT_BF16 && hist_budget() == 0 && bound_enabled() && !empty &&
+                       n_tiles(N) >= ent::kBoundMinBlocks;
     // header and the per-head max |c| start at 0, the per-head min R at all ones
     cudaError_t e = cudaMemsetAsync(ws, 0, bound ? FL.minr : kHdr, s);
     if (e == cudaSuccess && bound) e = cudaMemsetAsync(static_cast<char*>(ws) + FL.minr, 0xFF, (size_t)B * H * 4, s);
@@ -251,7 +251,7 @@ ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, i
     if (dtype == ENT_BF16) {
         a.acc = accept_rule();
         a.verify_tol = verify_tol();
-        a.fix_flags = reinterpret_cast<uint8_t*>(static_cast<char*>(ws) + FL.fix);
+        a.fail_list = reinterpret_cast<int*>(static_cast<char*>(ws) + FL.fix);
     }
     if (bound) {
         // statistics-pass skipping by key-block bounds; off with the histogram start, whose

@@ -8,6 +8,7 @@
 namespace ent {
 
 constexpr int kListCap = 16;        // entries per row in the support lists
+constexpr int kBoundMinBlocks = 64; // shortest query tile (key blocks) that runs the bound pass
 constexpr uint8_t kListOver = 255;  // list_n of a row with more than kListCap nonzeros
 
 struct FwdArgs {
@@ -30,13 +31,11 @@ struct FwdArgs {
                            // first block (0: no histogram, < 0: no limit)
     // Unverified Halley steps (tensor-core path): the rule, and the check in the P.V pass
     // (|sum_j p_ij - 1| <= verify_tol for every row that stopped on one).  A tile that
-    // fails it is flagged in fix_flags [BH][T] and solved again by a second launch with
-    // fix_mode = 1 (tiles not flagged return at once; that launch takes no unverified
-    // step).
+    // fails it goes on the failure list fail_list [BH*T] (count in the workspace header);
+    // the last CTA of the grid to finish solves those tiles again with evaluated stops.
     AcceptRule acc;
     float verify_tol;
-    uint8_t* fix_flags;
-    int fix_mode;
+    int* fail_list;
     float* otilde;         // nullable [BH][N][d] fp32: sum_j g_ij v_j / sum_j g_ij
     // Key-block bounds for skipping statistics-pass blocks (tensor-core path; all null:
     // no bound pass).  Per 64-key half-block hb of head bh (T2 = 2T of them):

@@ -90,7 +90,8 @@ struct Misc {
     int njobs;      // blocks in job_list for the next pass
     int abort;
     int inserts;    // histogram inserts of the whole tile so far (pass 0)
-    int pad[3];
+    int next;       // the CTA's next tile (flat bh * T + t), or -1
+    int pad[2];
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -159,26 +160,40 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, N = a.N;
-    const int t = a.causal ? (T - 1 - (int)blockIdx.x) : (int)blockIdx.x;   // long tiles first
-    const int bh = blockIdx.y;
-    // the second launch solves again only the tiles the first one flagged
-    if (a.fix_mode && !a.fix_flags[(size_t)bh * T + t]) return;
+    constexpr int SB = (OT && D == 128) ? 2 : kSbuf;   // S buffers of the P.V pass
+    constexpr uint32_t kOtCol = 256 + D;                // G.V accumulator (OT)
+    if (warp == 1) {   // TMEM for the CTA's whole life (it may solve more than one tile)
+        tmem_alloc(&misc->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    // This CTA's tile, then (last CTA of the grid only) the tiles on the failure list.
+    int cur_t = a.causal ? (T - 1 - (int)blockIdx.x) : (int)blockIdx.x;   // long tiles first
+    int cur_bh = blockIdx.y;
+    bool fixing = false;
+    int fail_cursor = 0;
+    for (int rep = 0;; ++rep) {
+    const int t = cur_t;
+    const int bh = cur_bh;
     const int nblk = a.causal ? t + 1 : T;
     const Abort ab{&misc->abort, a.hdr};
-    constexpr int SB = (OT && D == 128) ? 2 : kSbuf;   // S buffers of the P.V pass
+    // a tile solved again takes evaluated stops only
+    const AcceptRule acc = fixing ? AcceptRule() : a.acc;
     // Bound pass for this tile: only where a centroid bound can rule a block out at all
     // (some half-block of the head has R < 2 max |c|: a bound q.c_b + |q| R_b below
     // q.c_b' - |q| L_b' - 1/cx needs R_b < |c_b' - c_b| <= 2 max |c|)
+    // (and only in tiles of at least kBoundMinBlocks key blocks: the pass and its decision
+    // cost a few microseconds per tile, which a shorter tile does not win back)
     bool use_bound = false;
-    if (a.bstats != nullptr) {
+    if (a.bstats != nullptr && nblk >= kBoundMinBlocks) {
         const float maxc = __uint_as_float(a.head_words[bh]);
         const float minr = __uint_as_float(a.head_words[a.BH + bh]);
         use_bound = minr < 2.f * maxc;
     }
     const int nbj = use_bound ? (2 * nblk + 127) >> 7 : 0;   // 128-centroid jobs of the bound pass
-    constexpr uint32_t kOtCol = 256 + D;                // G.V accumulator (OT)
 
     if (threadIdx.x == 0) {
+        if (rep > 0)   // every phase of the previous tile is complete and nothing is in flight
+            for (uint64_t* bb = bars; bb <= mma_done; ++bb) mbar_inval(bb);
         for (int s = 0; s < kSlots; ++s) { mbar_init(&kfull[s], 1); mbar_init(&kempty[s], 1); }
         for (int s = 0; s < kDSlots; ++s) { mbar_init(&kfull2[s], 1); mbar_init(&kempty2[s], 1); }
         for (int s = 0; s < 2; ++s) { mbar_init(&s_full2[s], 1); mbar_init(&s_empty2[s], kEwWarps); }
@@ -203,10 +218,6 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         mbar_arrive_expect_tx(q_full, L::kTile);
         for (int at = 0; at < D / 64; ++at)
             tma_load_3d(smem + L::kQ + at * kAtom, &tm_q, at * 64, t * kBlk, bh, q_full);
-    }
-    if (warp == 1) {
-        tmem_alloc(&misc->tmem_base, kTmemCols);
-        tmem_relinquish();
     }
     for (int b = threadIdx.x; b < T; b += kThreads) { live[b] = 0; cand[b] = 0; }
     int* lcnt = reinterpret_cast<int*>(smem + L::kCnt);    // support-list entries per row
@@ -716,7 +727,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 X(0, half) = F0; X(1, half) = F1; X(2, half) = F2;
                 named_bar(1, kEw);
                 const float G0 = F0 + X(0, half ^ 1), G1 = F1 + X(1, half ^ 1), G2 = F2 + X(2, half ^ 1);
-                solver_update(sv, G0, G1, G2, gamma, gamma == 1.f, pass, a.ftol, a.stol, a.acc);
+                solver_update(sv, G0, G1, G2, gamma, gamma == 1.f, pass, a.ftol, a.stol, acc);
             }
             const int all = named_bar_and(1, kEw, sv.done) && pass > 0;
             // after an unverified downward step the support may reach blocks that were not
@@ -809,13 +820,14 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                     for (int c = 0; c < 16; ++c) nzw |= pk[c];
                     nzb |= nzw;
-                    if (a.list_n && nzw != 0u) {
+                    if (a.list_n && __any_sync(0xffffffffu, nzw != 0u)) {
                         // support list of the row: (key, u) for every p > 0 of these keys,
-                        // found word by word (a packed pair is nonzero iff one of its p is)
+                        // found word by word (a packed pair is nonzero iff one of its p is);
+                        // the warp skips together every word that is zero in all its rows
                         const size_t lbase = ((size_t)bh * N + i) * kListCap;
 #pragma unroll
                         for (int w = 0; w < 16; ++w) {
-                            if (pk[w] == 0u) continue;
+                            if (!__any_sync(0xffffffffu, pk[w] != 0u)) continue;
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
                                 const int c = 32 * hc + 2 * w + e;
@@ -918,7 +930,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const float f_end = X(3, 0) + X(3, 1) - 1.f;
         const bool bad = ok && row_valid && sv.unv && !(fabsf(f_end) <= a.verify_tol);
         const bool tile_bad = !named_bar_and(1, kEw, !bad);
-        if (!a.fix_mode && ew == 0) a.fix_flags[(size_t)bh * T + t] = tile_bad ? 1 : 0;
+        if (tile_bad && ew == 0) {
+            a.fail_list[atomicAdd(&a.hdr->fail_count, 1u)] = bh * T + t;
+            __threadfence();   // the entry is visible before this CTA counts itself finished
+        }
         uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
         for (int bb = ew; bb < T; bb += kEw) mrow[bb] = (bb < nblk && cand[bb] == kPvLive) ? 1 : 0;
         if (ew == 0) {
@@ -933,10 +948,37 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     tc_fence_before();
     __syncthreads();
+    // next: for the last CTA of the grid to finish, the tiles on the failure list
+    if (threadIdx.x == 0) {
+        int next = -1;
+        if (!misc->abort) {
+            bool last = fixing;
+            if (!fixing) {
+                __threadfence();
+                last = atomicAdd(&a.hdr->tile_counter, 1u) == gridDim.x * gridDim.y - 1;
+                __threadfence();
+            }
+            if (last) {
+                const int nfail = (int)*reinterpret_cast<volatile unsigned int*>(&a.hdr->fail_count);
+                if (fail_cursor < nfail) next = reinterpret_cast<volatile int*>(a.fail_list)[fail_cursor];
+            }
+        }
+        misc->next = next;
+    }
+    __syncthreads();
+    const int next = misc->next;
+    if (next < 0) break;
+    fixing = true;
+    ++fail_cursor;
+    cur_bh = next / T;
+    cur_t = next - cur_bh * T;
+    tc_fence_after();
+    }   // tiles of this CTA
+
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(misc->tmem_base, kTmemCols);
     }
 }
 
@@ -1093,12 +1135,6 @@ static cudaError_t launch_tc_fwd(const CUtensorMap& mq, const CUtensorMap& mk,
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
     kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(mq, mk, mv, mc, a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // tiles whose verification failed, solved again with evaluated stops only
-    FwdArgs f = a;
-    f.fix_mode = 1;
-    f.acc = AcceptRule();
-    kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(mq, mk, mv, mc, f);
     return cudaGetLastError();
 }
 

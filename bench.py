@@ -392,16 +392,17 @@ def combine_ranks(ms: float, units: float, world: int, device) -> tuple:
     return t.item(), u.item()
 
 
-def launches_per_step(dtype, delta):
-    """Kernels of this library launched per step.  bf16: the key-block statistics (unless
-    ENTATTN_BOUND=0 or the histogram start is selected), the forward and its second
-    launch for tiles that failed verification (it returns at once for the others), the
-    support-list backward (lists only), dq and dkv.  float32: the forward and three
-    backward kernels."""
+def launches_per_step(dtype, delta, T):
+    """Kernels of this library launched per step.  bf16: the key-block statistics (at
+    least 64 query tiles, unless ENTATTN_BOUND=0 or the histogram start is selected), the
+    forward and its second launch for tiles that failed verification (it returns at once
+    for the others), the support-list backward (lists only), dq and dkv.  float32: the
+    forward and three backward kernels."""
     if dtype != "bf16":
         return 4
     hb = os.environ.get("ENTATTN_HIST_BUDGET")
-    bound = os.environ.get("ENTATTN_BOUND", "1") != "0" and (not hb or int(hb) == 0)
+    bound = (os.environ.get("ENTATTN_BOUND", "1") != "0" and (not hb or int(hb) == 0)
+             and T >= 64)
     return int(bound) + 2 + (1 if delta == "lists" else 0) + 2
 
 SWEEP = ([("iid", {"beta": b}) for b in (1.0, 2.0, 4.0, 8.0)]
@@ -750,9 +751,13 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32" if w.dtype == "f32" else "bf16 inputs, f32 accumulate",
             "data": "synthetic",
-            "config": config_of(w, world, {"delta": (
-                "from the forward's otilde = G V / sum g (ent_attn_fwd_otilde, ent_attn_bwd_otilde)"
-                if ot is not None else "recomputed by a pass over the live keys") + f" [{c_why}]"}),
+            "config": config_of(w, world, {"delta": {
+                "otilde": "from the forward's otilde = G V / sum g (ent_attn_fwd_otilde, "
+                          "ent_attn_bwd_otilde)",
+                "recompute": "recomputed by a pass over the live keys",
+                "lists": "per row from the support lists (ent_attn_fwd_lists, ent_attn_bwd_lists) "
+                         "where every row of the query tile has one, else block kernels"}[c_delta]
+                + f" [{c_why}]"}),
             "ms_fwd": ms_fwd, "ms_bwd": ms_bwd,
             "executed_tflop_per_step": flops_all / 1e12,
             "effective_dense_tflops": world * dense_flops(w) / (ms_step * 1e-3) / 1e12,
@@ -770,7 +775,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": {"value": flops_all / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-            "gpu_launches": launches_per_step(w.dtype, c_delta) * args.steps,
+            "gpu_launches": launches_per_step(w.dtype, c_delta, -(-N // 128)) * args.steps,
             "clocks": clocks,
             "timed_region_s": timed_region_s,
             "peaks": {"source": peak_kind, "bf16_tflops": peaks["bf16_tflops"],

@@ -1,13 +1,14 @@
 """Unevaluated Halley stops of the bf16 forward and their check.
 
-A row may stop on a Halley step it does not evaluate (upward up to 5e-4, or up to 1e-2
-when the elements that can leave the support change f by at most 2e-5; downward up to
-1e-2); the P.V pass then sums p at the final tau, and a tile where such a row misses
-|sum p - 1| <= 1e-4 is solved again by a second launch that stops only at evaluated
-points.  Checked here: the oracle parity of the default rule (small cases, every
-alpha), fewer solver passes than with evaluated stops only, and the second launch: with
-a negative tolerance every such tile goes through it, and the outputs are then
-bit-identical to those of evaluated stops only (ENTATTN_ACCEPT=0)."""
+A row may stop on a Halley step it does not evaluate (up to 1e-2 either way, when the
+elements that can cross the support boundary within the step change f by at most
+1e-5); the P.V pass then sums p at the final tau, and a tile where such a row misses
+|sum p - 1| <= 1e-4 goes on a failure list that the last CTA of the grid solves again,
+stopping only at evaluated points.  Checked here: the oracle parity of the default rule
+(every row of a head, every alpha), no more solver passes than with evaluated stops
+only, and the re-solve path: with a negative tolerance every such tile goes through
+it, and the outputs are then bit-identical to those of evaluated stops only
+(ENTATTN_ACCEPT=0)."""
 import numpy as np
 import pytest
 import torch
@@ -48,7 +49,7 @@ def test_fewer_passes_same_contract(name, alpha, monkeypatch):
     monkeypatch.setenv("ENTATTN_ACCEPT", "0")
     _, c0 = _fwd(w, qd, kd, vd)
     assert c1[2] <= c0[2]                       # solver passes summed over tiles
-    assert c1[3] == c0[3]                       # no tile needed the second launch
+    assert c1[3] == c0[3]                       # no tile needed solving again
     # the first head against the oracle: tau, O and the block mask, every row
     sel = lambda a: np.ascontiguousarray(a[:1, :1])
     o_ref, tau_ref, marg = oracle.attn_fwd(sel(q), sel(k), sel(v), w.alpha, w.causal)
@@ -60,7 +61,7 @@ def test_fewer_passes_same_contract(name, alpha, monkeypatch):
 @pytest.mark.parametrize("otilde", [False, True])
 @pytest.mark.parametrize("name,change", [("iid", {"B": 1, "H": 4}), ("long", {"H": 2}),
                                          ("alpha", {"B": 1, "H": 2, "alpha": 1.25})])
-def test_second_launch_matches_evaluated_stops(name, change, otilde, monkeypatch):
+def test_resolved_tiles_match_evaluated_stops(name, change, otilde, monkeypatch):
     w = inputs.WORKLOADS[name].replace(**change)
     q, k, v, _ = inputs.make_inputs(w, seed=9)
     qd, kd, vd = (to_dev(a, "bf16") for a in (q, k, v))
@@ -72,4 +73,4 @@ def test_second_launch_matches_evaluated_stops(name, change, otilde, monkeypatch
     for a, b in zip(forced, plain):
         if a is not None:
             assert torch.equal(a, b)
-    assert cf[3] > c0[3]                        # tiles went through the second launch
+    assert cf[3] > c0[3]                        # tiles were solved again

@@ -1,4 +1,5 @@
-"""Statistics-pass skipping by key-block bounds (bf16 forward).
+"""Statistics-pass skipping by key-block bounds (bf16 forward; query tiles of at least
+64 key blocks).
 
 A key block whose centroid bound lies at or below (lower bound of the row maximum) - 1
 for every row of a tile is left out of the statistics pass and of everything after
@@ -23,13 +24,14 @@ def _cuda():
     capi.load()
 
 
+# the bound pass runs in query tiles of at least 64 key blocks, so N >= 8192
 CASES = [
-    ("clustered4k", {"span": 128, "B": 1, "H": 4}, True),
-    ("clustered4k", {"span": 128, "B": 1, "H": 2, "d": 64, "N": 1000}, True),      # ragged tail, d 64
-    ("clustered4k", {"span": 64, "B": 1, "H": 2, "causal": False, "N": 2000}, True),  # non-causal
-    ("clustered4k", {"span": 128, "B": 1, "H": 2, "d": 32, "N": 900}, True),        # d 32
+    ("clustered4k", {"span": 128, "B": 1, "H": 2, "N": 8192}, True),
+    ("clustered4k", {"span": 128, "B": 1, "H": 2, "d": 64, "N": 8492}, True),       # ragged tail, d 64
+    ("clustered4k", {"span": 64, "B": 1, "H": 1, "causal": False, "N": 8192}, True),  # non-causal
+    ("clustered4k", {"span": 128, "B": 1, "H": 2, "d": 32, "N": 8300}, True),       # d 32
     ("long", {"H": 2}, True),
-    ("iid", {"B": 1, "H": 4}, False),
+    ("iid", {"B": 1, "H": 2, "N": 8192}, False),
 ]
 
 
@@ -69,7 +71,7 @@ def test_bound_changes_work_not_results(name, change, skips, otilde, monkeypatch
 
 def test_forward_workspace_guard_bands():
     """The forward writes its key-block bounds inside the workspace it asked for, no further."""
-    w = inputs.WORKLOADS["clustered4k"].replace(span=128, B=1, H=3, N=700)
+    w = inputs.WORKLOADS["clustered4k"].replace(span=128, B=1, H=3, N=8300)
     q, k, v, _ = inputs.make_inputs(w, seed=9)
     qd, kd, vd = (to_dev(a, "bf16") for a in (q, k, v))
     need = capi.ent_attn_fwd_workspace_size(*w.shape, capi.ENT_BF16)

@@ -100,9 +100,10 @@ def test_otilde_small_bf16(N, d, causal, alpha):
     _check_otilde(gpu, q, k, v, alpha, causal, "bf16", np.arange(2 * N))
     dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, do, alpha, causal)
     check_grads(gpu, (dq, dk, dv))
-    # counters: one G.V product per live block
+    # counters: one G.V product per P.V block (the live blocks, and after an unevaluated
+    # downward stop the candidates at the final tau)
     live = int(gpu["mask"].sum())
-    assert gpu["cf"][5] == gpu["cf"][1] == live
+    assert gpu["cf"][5] == gpu["cf"][1] >= live
 
 
 @pytest.mark.parametrize("alpha", [1.5, 2.0])

@@ -77,8 +77,7 @@ struct Layout {
     static constexpr int kMisc = kBars + 8 * kNumBars;    // tmem base, decision, njobs, abort
     static constexpr int kPtab = kMisc + 32;              // 68 floats
     static constexpr int kMw = kPtab + 68 * 4;            // 8 floats: per-warp bound thresholds
-    static constexpr int kCnt = kMw + 8 * 4;              // 128 ints: support-list counts per row
-    static constexpr int kLive = kCnt + 128 * 4;          // live[T], cand[T] (bytes), list[T] (int),
+    static constexpr int kLive = kMw + 8 * 4;             // live[T], cand[T] (bytes), list[T] (int),
                                                           // per-warp block maxima [T][8] (bf16)
     __host__ __device__ static size_t r16(int T) { return (size_t)((T + 15) / 16) * 16; }
     static size_t bytes(int T) { return (size_t)kLive + 2 * r16(T) + 4 * (size_t)T + 16 * (size_t)T + 1024; }
@@ -220,8 +219,6 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tma_load_3d(smem + L::kQ + at * kAtom, &tm_q, at * 64, t * kBlk, bh, q_full);
     }
     for (int b = threadIdx.x; b < T; b += kThreads) { live[b] = 0; cand[b] = 0; }
-    int* lcnt = reinterpret_cast<int*>(smem + L::kCnt);    // support-list entries per row
-    if (threadIdx.x < kBlk) lcnt[threadIdx.x] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -768,6 +765,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int npass = pass;
         [[maybe_unused]] float2 sg2 = make_float2(0.f, 0.f);   // sum_j g of this half-row (OT)
         float2 fsum2 = make_float2(0.f, 0.f);                   // sum_j p of this half-row
+        int lnum = 0;                                           // support-list entries of this half-row
         if (ok) {
             named_bar(1, kEw);   // job_list / njobs of the P.V pass visible to the group
             nlive = misc->njobs;
@@ -823,7 +821,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     if (a.list_n && __any_sync(0xffffffffu, nzw != 0u)) {
                         // support list of the row: (key, u) for every p > 0 of these keys,
                         // found word by word (a packed pair is nonzero iff one of its p is);
-                        // the warp skips together every word that is zero in all its rows
+                        // the warp skips together every word that is zero in all its rows.
+                        // Each half-row counts its own entries (no shared counter on this
+                        // path): half 0 fills the list from the front, half 1 from the back,
+                        // and the epilogue closes the gap.
                         const size_t lbase = ((size_t)bh * N + i) * kListCap;
 #pragma unroll
                         for (int w = 0; w < 16; ++w) {
@@ -833,11 +834,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                 const int c = 32 * hc + 2 * w + e;
                                 const float u = __fmaf_rn(s[c], cx, -sv.tau);
                                 if (u > 0.f) {
-                                    const int slot = atomicAdd(&lcnt[row], 1);
-                                    if (slot < kListCap) {
+                                    if (lnum < kListCap) {
+                                        const int slot = half ? kListCap - 1 - lnum : lnum;
                                         a.list_key[lbase + slot] = b * kBlk + c0 + c;
                                         a.list_u[lbase + slot] = u;
                                     }
+                                    ++lnum;
                                 }
                             }
                         }
@@ -916,11 +918,22 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
         }
         if (a.list_n) {
-            named_bar(1, kEw);   // every half-row's entries are counted
-            if (row_valid && half == 0) {
-                const int n = lcnt[row];
-                a.list_n[(size_t)bh * N + i] = (ok && n <= kListCap) ? (uint8_t)n : kListOver;
+            // the row's list: half 0's entries at the front, half 1's at the back; half 1
+            // moves its entries to follow half 0's, in increasing order (each destination
+            // n0 + e lies at or below its source 16 - n1 + e and below every later source)
+            reinterpret_cast<int*>(xch)[(2 * 2 + half) * 128 + row] = lnum;
+            named_bar(1, kEw);
+            const int n0 = reinterpret_cast<int*>(xch)[(2 * 2 + 0) * 128 + row];
+            const int n1 = reinterpret_cast<int*>(xch)[(2 * 2 + 1) * 128 + row];
+            const bool fits = ok && n0 + n1 <= kListCap;
+            if (row_valid && half == 1 && fits) {
+                const size_t lbase = ((size_t)bh * N + i) * kListCap;
+                for (int e = 0; e < n1; ++e) {
+                    a.list_key[lbase + n0 + e] = a.list_key[lbase + kListCap - n1 + e];
+                    a.list_u[lbase + n0 + e] = a.list_u[lbase + kListCap - n1 + e];
+                }
             }
+            if (row_valid && half == 0) a.list_n[(size_t)bh * N + i] = fits ? (uint8_t)(n0 + n1) : kListOver;
         }
         // verification of the rows that stopped on an unevaluated step: f at the final tau
         // is sum_j p_ij - 1, summed above over a superset of the support; a tile where one

@@ -166,26 +166,32 @@ class EntmaxAttention(torch.autograd.Function):
     B*H*N*d*4 bytes kept for the backward) and the backward takes delta = dO . otilde
     instead of a delta pass over the keys (faster where most blocks are live);
     ``delta="recompute"`` keeps nothing extra and recomputes delta from the scores
-    (faster at high block sparsity, and the choice when activation memory is tight)."""
+    (faster at high block sparsity, and the choice when activation memory is tight);
+    ``delta="lists"`` keeps each row's support list (16 keys and u values, 128 bytes per
+    row, bf16 inputs) and the backward does every query tile whose rows all have lists
+    from them (faster where nearly every row has at most 16 nonzeros)."""
 
     @staticmethod
     def forward(ctx, q, k, v, alpha, causal, delta):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        ot = None
-        if delta == "otilde" and any(ctx.needs_input_grad[:3]):
-            ot = torch.empty(q.shape, dtype=torch.float32, device=q.device)
-        elif delta not in ("otilde", "recompute"):
-            raise ValueError(f"delta must be 'otilde' or 'recompute', not {delta!r}")
-        o, tau, mask, _ = entmax_attn_fwd(q, k, v, alpha, causal, otilde=ot)
-        ctx.save_for_backward(q, k, v, o, tau, mask, ot)
+        if delta not in ("otilde", "recompute", "lists"):
+            raise ValueError(f"delta must be 'otilde', 'recompute' or 'lists', not {delta!r}")
+        grad = any(ctx.needs_input_grad[:3])
+        ot = (torch.empty(q.shape, dtype=torch.float32, device=q.device)
+              if delta == "otilde" and grad else None)
+        lists = alloc_lists(q) if delta == "lists" and grad else None
+        o, tau, mask, _ = entmax_attn_fwd(q, k, v, alpha, causal, otilde=ot, lists=lists)
+        lk, lu, ln = lists if lists is not None else (None, None, None)
+        ctx.save_for_backward(q, k, v, o, tau, mask, ot, lk, lu, ln)
         ctx.alpha, ctx.causal = alpha, causal
         return o
 
     @staticmethod
     def backward(ctx, do):
-        q, k, v, o, tau, mask, ot = ctx.saved_tensors
+        q, k, v, o, tau, mask, ot, lk, lu, ln = ctx.saved_tensors
+        lists = (lk, lu, ln) if lk is not None else None
         dq, dk, dv = entmax_attn_bwd(q, k, v, o, do.contiguous(), tau, mask, ctx.alpha, ctx.causal,
-                                     otilde=ot)
+                                     otilde=ot, lists=lists)
         return dq, dk, dv, None, None, None
 
 

@@ -394,16 +394,17 @@ def combine_ranks(ms: float, units: float, world: int, device) -> tuple:
 
 def launches_per_step(dtype, delta, T):
     """Kernels of this library launched per step.  bf16: the key-block statistics (at
-    least 64 query tiles, unless ENTATTN_BOUND=0 or the histogram start is selected), the
-    forward and its second launch for tiles that failed verification (it returns at once
-    for the others), the support-list backward (lists only), dq and dkv.  float32: the
-    forward and three backward kernels."""
+    least 64 query tiles, unless ENTATTN_BOUND=0 or the histogram start is selected),
+    the forward (which also re-solves, in its last CTA, any tile that failed the check of
+    its unevaluated stops), the support-list backward (lists only), dq and dkv.  float32:
+    the forward and three backward kernels."""
     if dtype != "bf16":
         return 4
     hb = os.environ.get("ENTATTN_HIST_BUDGET")
     bound = (os.environ.get("ENTATTN_BOUND", "1") != "0" and (not hb or int(hb) == 0)
              and T >= 64)
-    return int(bound) + 2 + (1 if delta == "lists" else 0) + 2
+    return int(bound) + 1 + (1 if delta == "lists" else 0) + 2
+
 
 SWEEP = ([("iid", {"beta": b}) for b in (1.0, 2.0, 4.0, 8.0)]
          + [("alpha", {"alpha": a}) for a in (1.25, 1.5, 2.0)]

@@ -137,3 +137,17 @@ def test_lists_argument_errors():
     with pytest.raises(capi.EntAttnError) as e:
         A.entmax_attn_fwd(z, z, z, 1.5, True, lists=A.alloc_lists(z))
     assert e.value.status == capi.ENT_EUNSUPPORTED
+
+
+def test_autograd_lists_matches_recompute():
+    # beta 8: every query tile has lists, so the backward runs the list kernel alone
+    w, (q, k, v, do) = inputs.small_case(B=2, H=2, N=384, d=64, causal=True, alpha=1.5,
+                                         beta=8.0, seed=6)
+    grads = {}
+    for mode in ("lists", "recompute"):
+        qd, kd, vd = (to_dev(a, "bf16").requires_grad_() for a in (q, k, v))
+        o = A.entmax_attention(qd, kd, vd, 1.5, True, delta=mode)
+        o.backward(to_dev(do, "bf16"))
+        grads[mode] = [to_np(t.grad) for t in (qd, kd, vd)]
+    for a, b in zip(grads["lists"], grads["recompute"]):
+        assert rel_frob(a.astype(np.float64), b.astype(np.float64)) <= 1e-2

@@ -156,8 +156,9 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, N = a.N;
-    const int t = a.causal ? (T - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-    const int bh = blockIdx.y;
+    // grid (BH, T): every head's longest causal tile first
+    const int t = a.causal ? (T - 1 - (int)blockIdx.y) : (int)blockIdx.y;
+    const int bh = blockIdx.x;
     const int nblk = a.causal ? t + 1 : T;
     const Abort ab{&misc->abort, a.hdr};
     // a tile the support-list kernel covered (its dQ is written) is done
@@ -532,8 +533,9 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T, N = a.N;
-    const int b = blockIdx.x;
-    const int bh = blockIdx.y;
+    // grid (BH, T): every head's key block 0 (the most live query tiles when causal) first
+    const int b = blockIdx.y;
+    const int bh = blockIdx.x;
     const Abort ab{&misc->abort, a.hdr};
 
     if (threadIdx.x == 0) {
@@ -804,14 +806,14 @@ static cudaError_t launch_tc_bwd(const BwdArgs& a, cudaStream_t s, const CUtenso
         auto kern = tc_bwd_dq_kernel<D, GM>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
         if (e != cudaSuccess) return e;
-        kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(m[0], m[1], m[2], m[3], a);
+        kern<<<dim3(a.BH, a.T), kThreads, sm, s>>>(m[0], m[1], m[2], m[3], a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     const size_t sm = DkvLayout<D>::bytes(a.T);
     auto kern = tc_bwd_dkv_kernel<D, GM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(m[2], m[3], m[4], m[5], a);
+    kern<<<dim3(a.BH, a.T), kThreads, sm, s>>>(m[2], m[3], m[4], m[5], a);
     return cudaGetLastError();
 }
 

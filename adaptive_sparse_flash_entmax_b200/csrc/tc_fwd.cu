@@ -1,6 +1,6 @@
 // tc_fwd.cu -- the bf16 forward on sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
-// One CTA per 128-row query tile ("AdaSplash: Adaptive Sparse Flash Attention",
+// One CTA per 128-row query tile, grid (heads, tiles) ("AdaSplash: Adaptive Sparse Flash Attention",
 // Technical Deep Dive / AdaSplash: Fused GPU Kernel for Attention: the Q tile is
 // loaded once and stays on chip; K tiles stream for the tau passes; a final pass
 // streams K and V and accumulates O = P V).  Warp roles:
@@ -166,8 +166,10 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tmem_relinquish();
     }
     // This CTA's tile, then (last CTA of the grid only) the tiles on the failure list.
-    int cur_t = a.causal ? (T - 1 - (int)blockIdx.x) : (int)blockIdx.x;   // long tiles first
-    int cur_bh = blockIdx.y;
+    // grid (BH, T): the heads' longest causal tiles are dispatched first, all of them
+    // before any shorter one, so the last wave holds the shortest tiles
+    int cur_t = a.causal ? (T - 1 - (int)blockIdx.y) : (int)blockIdx.y;
+    int cur_bh = blockIdx.x;
     bool fixing = false;
     int fail_cursor = 0;
     for (int rep = 0;; ++rep) {
@@ -371,16 +373,17 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                         for (int kk = 0; kk < kBlk / 16; ++kk) {
                             // keys 16kk .. 16kk+15: the half (kk >> 2) that owns them wrote
-                            // their P, two per column, into its own first 32 columns
-                            const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
+                            // their P, two per column, at the start of the 32 columns of the
+                            // round ((kk >> 1) & 1) that held their scores
+                            const uint32_t acol = (kk >> 2) * 64 + ((kk >> 1) & 1) * 32 + (kk & 1) * 8;
                             umma_bf16_ts(tmem + 256, ap + acol, dv + ((kk * 16 * 128) >> 4), idesc_pv,
                                          (ip > 0 || kk > 0) ? 1u : 0u);
                         }
                         if constexpr (OT) {
-                            // G (bf16 pairs) sits in the 32 columns after each half's P
+                            // G (bf16 pairs) sits 16 columns after the P of the same keys
 #pragma unroll
                             for (int kk = 0; kk < kBlk / 16; ++kk) {
-                                const uint32_t acol = (kk >> 2) * 64 + 32 + (kk & 3) * 8;
+                                const uint32_t acol = (kk >> 2) * 64 + ((kk >> 1) & 1) * 32 + 16 + (kk & 1) * 8;
                                 umma_bf16_ts(tmem + kOtCol, ap + acol, dv + ((kk * 16 * 128) >> 4),
                                              idesc_pv, (ip > 0 || kk > 0) ? 1u : 0u);
                             }
@@ -774,27 +777,27 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const int sb = li % SB;   // the P.V pass counts its own jobs
                 if (!(ok = mbar_wait(&s_full[sb], (li / SB) & 1, ab, 9))) break;
                 tc_fence_after();
-                float s[64];
-                tmem_ld32(lane_base + sbuf_col(sb) + c0, &s[0]);
-                tmem_ld32(lane_base + sbuf_col(sb) + c0 + 32, &s[32]);
-                tmem_wait_ld();
-                reg_fence<64>(s);
-                const int nv = key_end - b * kBlk - c0;
-                if (!__all_sync(0xffffffffu, nv >= 64)) {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
-                }
+                const int nv = key_end - b * kBlk - c0;   // valid columns of this thread: c < nv
+                const bool full_blk = __all_sync(0xffffffffu, nv >= 64);
                 const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-sv.tau, -sv.tau);
                 uint32_t nzb = 0u;   // OR of this thread's bf16 p bits: nonzero iff some p > 0
-                // two rounds of 32 keys; P of keys c0 + 32 hc .. + 31 goes over this thread's
-                // own S columns c0 + 16 hc .. + 15 (G, with otilde, 32 columns further on)
-#pragma unroll
+                // two rounds of 32 keys, each loaded, turned into P (and G) and stored over its
+                // own 32 S columns: P of keys c0 + 32 hc + 2k, +1 in column c0 + 32 hc + k
+                // (k < 16), G with otilde 16 columns further on; one copy of the round's code
+#pragma unroll 1
                 for (int hc = 0; hc < 2; ++hc) {
+                    float s[32];
+                    tmem_ld32(lane_base + sbuf_col(sb) + c0 + 32 * hc, s);
+                    tmem_wait_ld();
+                    reg_fence<32>(s);
+                    if (!full_blk) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) s[c] = (32 * hc + c < nv) ? s[c] : -INFINITY;
+                    }
                     uint32_t pk[16];
                     [[maybe_unused]] uint32_t gk[16];
 #pragma unroll
-                    for (int c2 = 0; c2 < 32; c2 += 2) {
-                        const int c = 32 * hc + c2;
+                    for (int c = 0; c < 32; c += 2) {
                         const float2 u2 = __ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2);
                         if constexpr (OT) {
                             float2 p2, g2;
@@ -802,8 +805,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             fsum2 = __fadd2_rn(fsum2, p2);
                             const __nv_bfloat162 hp = __floats2bfloat162_rn(p2.x, p2.y);
                             const __nv_bfloat162 hg = __floats2bfloat162_rn(g2.x, g2.y);
-                            pk[c2 >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
-                            gk[c2 >> 1] = *reinterpret_cast<const uint32_t*>(&hg);
+                            pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&hp);
+                            gk[c >> 1] = *reinterpret_cast<const uint32_t*>(&hg);
                             // sum the rounded weights the G.V product uses: otilde is then
                             // a weighted mean whose weights sum to one
                             sg2 = __fadd2_rn(sg2, __bfloat1622float2(hg));
@@ -811,32 +814,37 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             const float2 p2 = entmax_p_x2<GM>(u2, gamma);
                             fsum2 = __fadd2_rn(fsum2, p2);
                             const __nv_bfloat162 h2 = __floats2bfloat162_rn(p2.x, p2.y);
-                            pk[c2 >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+                            pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
                         }
                     }
                     uint32_t nzw = 0u;
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) nzw |= pk[c];
+                    for (int w = 0; w < 16; ++w) nzw |= pk[w];
                     nzb |= nzw;
                     if (a.list_n && __any_sync(0xffffffffu, nzw != 0u)) {
-                        // support list of the row: (key, u) for every p > 0 of these keys,
-                        // found word by word (a packed pair is nonzero iff one of its p is);
-                        // the warp skips together every word that is zero in all its rows.
-                        // Each half-row counts its own entries (no shared counter on this
-                        // path): half 0 fills the list from the front, half 1 from the back,
-                        // and the epilogue closes the gap.
-                        const size_t lbase = ((size_t)bh * N + i) * kListCap;
+                        // support list of the row: (key, u) for every p > 0 of these keys (a
+                        // packed pair is nonzero iff one of its p is).  Compact on purpose: the
+                        // round's u go to this thread's column of the (by now idle) histogram
+                        // area and a loop visits the nonzero words only.  Each half-row counts
+                        // its own entries: half 0 fills the list from the front, half 1 from
+                        // the back, and the epilogue closes the gap.
+                        float* scr = reinterpret_cast<float*>(smem + L::kP) + ew;
 #pragma unroll
-                        for (int w = 0; w < 16; ++w) {
-                            if (!__any_sync(0xffffffffu, pk[w] != 0u)) continue;
+                        for (int c = 0; c < 32; ++c) scr[c * kEw] = __fmaf_rn(s[c], cx, -sv.tau);
+                        uint32_t wm = 0u;
+#pragma unroll
+                        for (int w = 0; w < 16; ++w) wm |= (pk[w] != 0u ? 1u : 0u) << w;
+                        const size_t lbase = ((size_t)bh * N + i) * kListCap;
+                        while (wm != 0u) {
+                            const int w = __ffs(wm) - 1;
+                            wm &= wm - 1u;
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
-                                const int c = 32 * hc + 2 * w + e;
-                                const float u = __fmaf_rn(s[c], cx, -sv.tau);
+                                const float u = scr[(2 * w + e) * kEw];
                                 if (u > 0.f) {
                                     if (lnum < kListCap) {
                                         const int slot = half ? kListCap - 1 - lnum : lnum;
-                                        a.list_key[lbase + slot] = b * kBlk + c0 + c;
+                                        a.list_key[lbase + slot] = b * kBlk + c0 + 32 * hc + 2 * w + e;
                                         a.list_u[lbase + slot] = u;
                                     }
                                     ++lnum;
@@ -844,8 +852,8 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             }
                         }
                     }
-                    tmem_st16(lane_base + sbuf_col(sb) + c0 + 16 * hc, pk);
-                    if constexpr (OT) tmem_st16(lane_base + sbuf_col(sb) + c0 + 32 + 16 * hc, gk);
+                    tmem_st16(lane_base + sbuf_col(sb) + c0 + 32 * hc, pk);
+                    if constexpr (OT) tmem_st16(lane_base + sbuf_col(sb) + c0 + 32 * hc + 16, gk);
                 }
                 // the block mask: some p > 0 in the block at the final tau (a bf16 p is
                 // nonzero exactly when its bits are)
@@ -1147,7 +1155,7 @@ static cudaError_t launch_tc_fwd(const CUtensorMap& mq, const CUtensorMap& mk,
     auto kern = a.otilde ? tc_fwd_kernel<D, GM, true> : tc_fwd_kernel<D, GM, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(a.T, a.BH), kThreads, sm, s>>>(mq, mk, mv, mc, a);
+    kern<<<dim3(a.BH, a.T), kThreads, sm, s>>>(mq, mk, mv, mc, a);
     return cudaGetLastError();
 }
 

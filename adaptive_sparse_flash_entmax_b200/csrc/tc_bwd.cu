@@ -316,43 +316,36 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         float* xch = reinterpret_cast<float*>(smem + L::kXch);   // [5][2][128]
         const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-tau, -tau);
         bool ok = true;
-        // S and dP of job j, columns [32r, 32r + 32) of this thread's 64 keys; the pair is
-        // released after the second round
-        auto load_round = [&](int j, int r, float* s, float* dp) -> void {
-            const int p = pair_of(j);
-            tmem_ld32(lane_base + p * 256 + r * 32, s);
-            tmem_ld32(lane_base + p * 256 + 128 + r * 32, dp);
-            tmem_wait_ld();
-            reg_fence<32>(s);
-            reg_fence<32>(dp);
-            if (r == 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[p]);
-            }
-            const int nv = key_end - list[j < nA ? j : j - nA] * kBlk - half * 64 - r * 32;
-            if (!__all_sync(0xffffffffu, nv >= 32)) {   // diagonal or ragged block
-#pragma unroll
-                for (int c = 0; c < 32; ++c) s[c] = (c < nv) ? s[c] : -INFINITY;
-            }
-        };
         // phase A: sum_j g and sum_j g dP
         float sg = 0.f, sgdp = 0.f;
         for (int j = 0; j < nA && ok; ++j) {
             if (!(ok = mbar_wait(&s_full[pair_of(j)], use_of(j) & 1, ab, 26))) break;
             tc_fence_after();
+            // both rounds in one go (the pair is free again after a single load latency)
+            float sa[64], dpa[64];
+            const int p = pair_of(j);
+            tmem_ld32(lane_base + p * 256, &sa[0]);
+            tmem_ld32(lane_base + p * 256 + 32, &sa[32]);
+            tmem_ld32(lane_base + p * 256 + 128, &dpa[0]);
+            tmem_ld32(lane_base + p * 256 + 128 + 32, &dpa[32]);
+            tmem_wait_ld();
+            reg_fence<64>(sa);
+            reg_fence<64>(dpa);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[p]);
+            const int nv = key_end - list[j] * kBlk - half * 64;
+            if (!__all_sync(0xffffffffu, nv >= 64)) {   // diagonal or ragged block
+#pragma unroll
+                for (int c = 0; c < 64; ++c) sa[c] = (c < nv) ? sa[c] : -INFINITY;
+            }
             float2 a0 = make_float2(0.f, 0.f), b0 = a0, a1 = a0, b1 = a0;
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                float s[32], dp[32];
-                load_round(j, r, s, dp);
-#pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    const float2 g0 = entmax_g_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma);
-                    const float2 g1 = entmax_g_x2<GM>(__ffma2_rn(make_float2(s[c + 2], s[c + 3]), cx2, nt2), gamma);
-                    a0 = __fadd2_rn(a0, g0); b0 = __ffma2_rn(g0, make_float2(dp[c], dp[c + 1]), b0);
-                    a1 = __fadd2_rn(a1, g1); b1 = __ffma2_rn(g1, make_float2(dp[c + 2], dp[c + 3]), b1);
-                }
+            for (int c = 0; c < 64; c += 4) {
+                const float2 g0 = entmax_g_x2<GM>(__ffma2_rn(make_float2(sa[c], sa[c + 1]), cx2, nt2), gamma);
+                const float2 g1 = entmax_g_x2<GM>(__ffma2_rn(make_float2(sa[c + 2], sa[c + 3]), cx2, nt2), gamma);
+                a0 = __fadd2_rn(a0, g0); b0 = __ffma2_rn(g0, make_float2(dpa[c], dpa[c + 1]), b0);
+                a1 = __fadd2_rn(a1, g1); b1 = __ffma2_rn(g1, make_float2(dpa[c + 2], dpa[c + 3]), b1);
             }
             a0 = __fadd2_rn(a0, a1); b0 = __fadd2_rn(b0, b1);
             sg += a0.x + a0.y;
@@ -408,11 +401,32 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (!(ok = mbar_wait(&s_full[0], use_of(j) & 1, ab, 26))) break;
             tc_fence_after();
             const int key0 = list[ib] * kBlk + half * 64;   // key of this thread's first column
+            // both rounds' S and dP in one go, so the pair is free for S(i+1), dP(i+1) after a
+            // single TMEM load latency
+            float sa[64], dpa[64];
+            {
+                const int p = pair_of(j);
+                tmem_ld32(lane_base + p * 256, &sa[0]);
+                tmem_ld32(lane_base + p * 256 + 32, &sa[32]);
+                tmem_ld32(lane_base + p * 256 + 128, &dpa[0]);
+                tmem_ld32(lane_base + p * 256 + 128 + 32, &dpa[32]);
+                tmem_wait_ld();
+                reg_fence<64>(sa);
+                reg_fence<64>(dpa);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[p]);
+                const int nv = key_end - key0;   // valid columns of this thread: c < nv
+                if (!__all_sync(0xffffffffu, nv >= 64)) {   // diagonal or ragged block
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) sa[c] = (c < nv) ? sa[c] : -INFINITY;
+                }
+            }
             uint32_t whi[32];
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                float s[32], dp[32];
-                load_round(j, r, s, dp);
+                const float* s = sa + 32 * r;
+                const float* dp = dpa + 32 * r;
                 float rmax = s[0];
 #pragma unroll
                 for (int c = 1; c < 32; ++c) rmax = fmaxf(rmax, s[c]);

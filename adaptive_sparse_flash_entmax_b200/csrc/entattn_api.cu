@@ -106,6 +106,13 @@ ent::AcceptRule accept_rule() {
     return r;
 }
 
+// Speculative first job of each score pass in the bf16 forward (on by default);
+// ENTATTN_SPEC=0 (environment, read per call) waits for each decision instead, for ablations.
+int spec_enabled() {
+    const char* v = getenv("ENTATTN_SPEC");
+    return (v && *v && atoi(v) == 0) ? 0 : 1;
+}
+
 float verify_tol() {
     const char* v = getenv("ENTATTN_VERIFY_TOL");
     return (v && *v) ? (float)atof(v) : 1e-4f;
@@ -251,6 +258,7 @@ ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, i
     if (dtype == ENT_BF16) {
         a.acc = accept_rule();
         a.verify_tol = verify_tol();
+        a.spec = spec_enabled();
         a.fail_list = reinterpret_cast<int*>(static_cast<char*>(ws) + FL.fix);
     }
     if (bound) {

@@ -36,6 +36,8 @@ struct FwdArgs {
     AcceptRule acc;
     float verify_tol;
     int* fail_list;
+    int spec;              // tensor-core path: load and multiply the next score pass's likely
+                           // first job before the decision after a pass (0: wait for it)
     float* otilde;         // nullable [BH][N][d] fp32: sum_j g_ij v_j / sum_j g_ij
     // Key-block bounds for skipping statistics-pass blocks (tensor-core path; all null:
     // no bound pass).  Per 64-key half-block hb of head bh (T2 = 2T of them):

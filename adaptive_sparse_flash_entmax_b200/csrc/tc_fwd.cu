@@ -115,6 +115,33 @@ __device__ __forceinline__ void warp_colmax_32(float* v, int lane) {
     }
 }
 
+// The speculative first job of the next score pass.  The decision after a pass (another
+// solver pass, with its candidate list, or the P.V pass) drains the tile's pipeline: its
+// first K blocks are loaded and multiplied only after it.  Instead, the blocks of this
+// pass's first job -- usually also the next pass's first candidates -- are loaded by the
+// producer and multiplied by the MMA issuer while the elementwise warps finish the pass;
+// if the next pass starts with the same job, its S is already in TMEM, otherwise the
+// elementwise warps drop it.  Every role arms it under the same condition from the same
+// list and checks it against the same published decision, so all agree on hit or miss.
+struct SpecJob {
+    int b0 = -1, b1 = -1;   // the guessed job's blocks (b1 < 0: a one-block job)
+    int use = 0;            // producer: the double-slot use that holds it
+    bool on = false, hit = false;
+    __device__ __forceinline__ void arm(bool want, bool all_blocks, int njobs, const int* jl) {
+        on = want;
+        if (want) {
+            b0 = all_blocks ? 0 : jl[0];
+            b1 = njobs > 1 ? (all_blocks ? 1 : jl[1]) : -1;
+        }
+    }
+    __device__ __forceinline__ bool matches(int njobs, const int* jl) const {
+        return njobs > 0 && jl[0] == b0 && (njobs > 1 ? jl[1] == b1 : b1 < 0);
+    }
+    __device__ __forceinline__ void check(bool solve, int njobs, const int* jl) {
+        hit = on && solve && matches(njobs, jl);
+    }
+};
+
 // Bounded wait that ignores the abort flag (used to drain in-flight copies).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = globaltimer_ns();
@@ -232,6 +259,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             int sj = 0, dj = 0, kind = kDecSolve;   // P.V-pass tiles, score-pass double slots loaded
             uint32_t dec_phase = 0;
             bool ok = true, first = !use_bound, bound = use_bound;
+            SpecJob spec;   // the next pass's first job, loaded before the decision
             // a score-pass job: K blocks b0 and b1 (b1 < 0: none) stacked in one double slot,
             // block h at rows 128h of each [256 rows x 64] atom (the bound pass loads blocks
             // of 128 centroids from `map` the same way)
@@ -265,12 +293,25 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int i = 0; i < njobs && ok; i += 2)
                         ok = load_pair(&tm_c, i, (i + 1 < njobs) ? i + 1 : -1);
                 } else if (!pv) {
-                    for (int i = 0; i < njobs && ok; i += 2) {
+                    // a hit: the first job is in the slot the speculative load filled.  The
+                    // guess for the next pass is read now, while this pass's list is stable
+                    // (the next decision needs every job of this pass loaded first).
+                    const int i0 = spec.hit ? 2 : 0;
+                    spec.arm(a.spec && njobs > 0, first, njobs, job_list);
+                    for (int i = i0; i < njobs && ok; i += 2) {
                         const int b0 = first ? i : job_list[i];
                         const int b1 = (i + 1 < njobs) ? (first ? i + 1 : job_list[i + 1]) : -1;
                         ok = load_pair(&tm_k, b0, b1);
                     }
+                    if (ok && spec.on) {
+                        ok = load_pair(&tm_k, spec.b0, spec.b1);
+                        spec.use = dj - 1;
+                    }
                 } else {
+                    // the P.V tiles reuse the ring's memory: the speculative job's K blocks
+                    // must have been read by its MMA first
+                    if (spec.on)
+                        ok = mbar_wait(&kempty2[spec.use % kDSlots], (spec.use / kDSlots) & 1, ab, 1);
                     for (int i = 0; i < njobs && ok; ++i) {
                         const int b = job_list[i];
                         ok = load_tile(&tm_k, b);
@@ -282,6 +323,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 if (!(ok = mbar_wait(dec_bar, dec_phase, ab, 2))) break;
                 dec_phase ^= 1;
                 kind = misc->decision;
+                spec.check(kind == kDecSolve, misc->njobs, job_list);
             }
             // Copies issued but possibly not consumed land before the CTA ends.
             drain_wait(q_full, 0);
@@ -304,6 +346,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             int sjob = 0, kind = kDecSolve;   // score-pass jobs issued (= double slots consumed)
             uint32_t dec_phase = 0;
             bool first = !use_bound, bound = use_bound;
+            SpecJob spec;   // the next pass's first job, issued before the decision
             auto wait_tile = [&](int tt) { return mbar_wait(&kfull[tt % kSlots], (tt / kSlots) & 1, ab, 4); };
             auto issue_s = [&](int sb, int tt) {
                 const uint64_t dk = dring + ((uint32_t)((tt % kSlots) * L::kTile) >> 4);
@@ -316,31 +359,41 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 umma_commit(&s_full[sb]);
                 umma_commit(&kempty[tt % kSlots]);
             };
+            // one score-pass job: S of one or two K blocks (one double slot) into an S buffer
+            auto issue_job = [&](bool two) -> bool {
+                const int sb = sjob & 1, ds = sjob % kDSlots;
+                if (!mbar_wait(&kfull2[ds], (sjob / kDSlots) & 1, ab, 4)) return false;
+                if (!mbar_wait(&s_empty2[sb], ((sjob >> 1) & 1) ^ 1, ab, 5)) return false;
+                tc_fence_after();
+                const uint32_t idesc = two ? idesc_qk2 : idesc_qk;
+                const uint64_t dk = dring + ((uint32_t)(ds * 2 * L::kTile) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t oa = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
+                    const uint32_t ob = ((kk >> 2) * 2 * kAtom + (kk & 3) * 32) >> 4;
+                    umma_bf16(tmem + sb * 256, dq + oa, dk + ob, idesc, kk > 0);
+                }
+                umma_commit(&s_full2[sb]);
+                umma_commit(&kempty2[ds]);
+                ++sjob;
+                return true;
+            };
             while (ok) {
                 const bool pv = kind == kDecPv;
                 const int njobs = bound ? nbj : first ? nblk : misc->njobs;
+                const bool was_bound = bound, was_first = first;
                 first = bound = false;
                 if (!pv) {
-                    for (int i = 0; i < njobs && ok; i += 2, ++sjob) {
-                        const int sb = sjob & 1, ds = sjob % kDSlots;
-                        if (!(ok = mbar_wait(&kfull2[ds], (sjob / kDSlots) & 1, ab, 4))) break;
-                        if (!(ok = mbar_wait(&s_empty2[sb], ((sjob >> 1) & 1) ^ 1, ab, 5))) break;
-                        tc_fence_after();
-                        const uint32_t idesc = (i + 1 < njobs) ? idesc_qk2 : idesc_qk;
-                        const uint64_t dk = dring + ((uint32_t)(ds * 2 * L::kTile) >> 4);
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t oa = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
-                            const uint32_t ob = ((kk >> 2) * 2 * kAtom + (kk & 3) * 32) >> 4;
-                            umma_bf16(tmem + sb * 256, dq + oa, dk + ob, idesc, kk > 0);
-                        }
-                        umma_commit(&s_full2[sb]);
-                        umma_commit(&kempty2[ds]);
-                    }
+                    // a hit: the first job was issued before the decision
+                    const int i0 = spec.hit ? 2 : 0;
+                    spec.arm(a.spec && njobs > 0 && !was_bound, was_first, njobs, job_list);
+                    for (int i = i0; i < njobs && ok; i += 2) ok = issue_job(i + 1 < njobs);
                     if (!ok) break;
+                    if (spec.on && !(ok = issue_job(spec.b1 >= 0))) break;
                     if (!(ok = mbar_wait(dec_bar, dec_phase, ab, 7))) break;
                     dec_phase ^= 1;
                     kind = misc->decision;
+                    spec.check(kind == kDecSolve, misc->njobs, job_list);
                     continue;
                 }
                 // P.V pass over the live blocks, with its own barriers and ring counters:
@@ -463,6 +516,18 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         int sjob = 0, pass = 0, nlive = 0;
         long long qk_blocks = use_bound ? nbj : nblk, skipped = 0;
         bool ok = true;
+        SpecJob spec;
+        // a speculative job that is not used: wait for its S, then free the buffer unread
+        auto drop_job = [&]() -> bool {
+            const int sb = sjob & 1;
+            if (!mbar_wait(&s_full2[sb], (sjob >> 1) & 1, ab, 14)) return false;
+            tc_fence_after();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty2[sb]);
+            ++sjob;
+            return true;
+        };
         if (use_bound) {
             // ---- bound pass: S_c = Q C^T over the tile's half-block centroids
             // |q| of this row from the swizzled Q tile (a sum of squares does not depend on
@@ -582,9 +647,16 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 qk_blocks += npj;
                 if (pass == 0) skipped = nblk - npj;
             }
+            // the speculative job issued after the previous pass: on a hit it is this pass's
+            // first job (the next S buffer in sequence); on a miss its S is dropped
+            if (spec.on && !spec.matches(npj, job_list)) {
+                ok = ok && drop_job();
+                qk_blocks += spec.b1 >= 0 ? 2 : 1;
+            }
+            spec.arm(a.spec && npj > 0, pass == 0 && !use_bound, npj, job_list);
             // jobs of two blocks (one 256-column S buffer); the buffer is released after
             // the second block's load
-            for (int jj = 0; jj < npj; jj += 2, ++sjob) {
+            for (int jj = 0; jj < npj && ok; jj += 2, ++sjob) {
                 const int sb = sjob & 1;
                 if (!(ok = mbar_wait(&s_full2[sb], (sjob >> 1) & 1, ab, 8))) break;
                 tc_fence_after();
@@ -664,10 +736,30 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         // two packed accumulator sets (columns c mod 4 < 2 and >= 2)
                         float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, b0 = a0, b1 = a0, b2 = a0;
                         const float2 cx2 = make_float2(cx, cx), nt2 = make_float2(-sv.tau, -sv.tau);
+                        if constexpr (GM == 2) {
+                            // F2 = #{u > 0} as 64 minus the sign bits: an integer add per
+                            // element instead of a compare and a float add (masked columns are
+                            // -inf; an exact u = +0 counts, which adds nothing to F0, F1 and
+                            // only makes the Halley step and the crossing bound more cautious)
+                            unsigned int neg = 0u;
 #pragma unroll
-                        for (int c = 0; c < 64; c += 4) {
-                            entmax_acc_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma, a0, a1, a2);
-                            entmax_acc_x2<GM>(__ffma2_rn(make_float2(s[c + 2], s[c + 3]), cx2, nt2), gamma, b0, b1, b2);
+                            for (int c = 0; c < 64; c += 4) {
+                                const float2 u0 = __ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2);
+                                const float2 u1 = __ffma2_rn(make_float2(s[c + 2], s[c + 3]), cx2, nt2);
+                                neg += (__float_as_uint(u0.x) >> 31) + (__float_as_uint(u0.y) >> 31) +
+                                       (__float_as_uint(u1.x) >> 31) + (__float_as_uint(u1.y) >> 31);
+                                const float2 p0 = make_float2(fmaxf(u0.x, 0.f), fmaxf(u0.y, 0.f));
+                                const float2 p1 = make_float2(fmaxf(u1.x, 0.f), fmaxf(u1.y, 0.f));
+                                a0 = __ffma2_rn(p0, p0, a0); a1 = __fadd2_rn(a1, p0);
+                                b0 = __ffma2_rn(p1, p1, b0); b1 = __fadd2_rn(b1, p1);
+                            }
+                            a2 = make_float2((float)(64u - neg), 0.f);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 64; c += 4) {
+                                entmax_acc_x2<GM>(__ffma2_rn(make_float2(s[c], s[c + 1]), cx2, nt2), gamma, a0, a1, a2);
+                                entmax_acc_x2<GM>(__ffma2_rn(make_float2(s[c + 2], s[c + 3]), cx2, nt2), gamma, b0, b1, b2);
+                            }
                         }
                         a0 = __fadd2_rn(a0, b0); a1 = __fadd2_rn(a1, b1); a2 = __fadd2_rn(a2, b2);
                         const float f1 = a1.x + a1.y;
@@ -764,6 +856,11 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
             if (all) break;
+        }
+        // the P.V pass follows: a speculative job issued after the last pass is dropped
+        if (spec.on) {
+            ok = ok && drop_job();
+            qk_blocks += spec.b1 >= 0 ? 2 : 1;
         }
         const int npass = pass;
         [[maybe_unused]] float2 sg2 = make_float2(0.f, 0.f);   // sum_j g of this half-row (OT)

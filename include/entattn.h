@@ -88,10 +88,20 @@ size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype);
  * the histogram start is selected), solver passes until every row of the
  * tile has converged, and one P.V pass over the live key blocks.  A row stops
  * when |f(tau)| <= 1e-5 (bf16; 1e-6 float32), when its next step is below
- * 1e-6 (4e-7) * max(1, |tau|), or after 24 passes; the bf16 path also stops on
- * an upward Halley step of at most 5e-4, taking that step unverified (the
- * support only shrinks, so the block mask still covers every p > 0 and may
- * differ from the exact one only on blocks with max(x - tau) > -5e-4).
+ * 1e-6 (4e-7) * max(1, |tau|), or after 24 passes.  The bf16 path also stops
+ * on a Halley step it does not evaluate when the step is at most 1e-2 and the
+ * support elements that can cross the boundary within it change f by at most
+ * 1e-5 (upward: F2 h^2 for gamma >= 2, F1 h below; downward: h^min(gamma,2));
+ * the P.V pass then checks |sum_j p_ij - 1| <= 1e-4 at the returned tau, and
+ * every query tile with a row that fails the check is solved again with
+ * evaluated stops only, by the last CTA of the same launch.  The block mask is
+ * written from p > 0 at the returned tau, so it is exact for that tau.
+ * Environment switches read at each call, for ablations: ENTATTN_ACCEPT=0 (no
+ * unevaluated stops), ENTATTN_VERIFY_TOL (the check's tolerance; negative:
+ * solve every such tile again), ENTATTN_BOUND=0 (no centroid bound pass),
+ * ENTATTN_SPEC=0 (no speculative first job: by default the K blocks of a score
+ * pass's first job are loaded and multiplied again before the decision that
+ * ends the pass, and used if the next pass starts with the same job).
  * bf16 inputs start every row's solver from the plain bracket [m-1, m - n^(1-alpha)]
  * (measured faster on B200 than the histogram start, whose inserts cost more than
  * the passes they save).  The environment variable ENTATTN_HIST_BUDGET, read at each
@@ -237,7 +247,8 @@ ent_status ent_attn_noalloc_read_status(long long *counters, void *stream);
  * Synchronises `stream` and reads the status word and the work counters of a
  * workspace that a forward or backward used.  counters (nullable, 8 entries):
  *   [0] block products (128x128xd, 2*128*128*d flops each) in the forward's
- *       statistics and solver passes (one S block per visited block and pass),
+ *       statistics and solver passes (one S block per visited block and pass,
+ *       plus the blocks of speculative first jobs that were not used),
  *   [1] live blocks in the forward P.V pass (two block products each: S, P V),
  *   [2] solver passes summed over query tiles,
  *   [3] query tiles processed,

@@ -99,8 +99,8 @@ struct RowSolver {
 // Unverified-step rules of solver_update (all 0: every stop is at an evaluated tau).
 struct AcceptRule {
     float step = 0.f;      // largest step, either way
-    float cert = 0.f;      // bound on the change in f from elements crossing the support
-                           // boundary within the step
+    float cert_up = 0.f;   // bound on the change in f from elements crossing the support
+    float cert_down = 0.f; // boundary within an upward / a downward step
 };
 
 // One Halley-bisection update after a pass evaluated F0 = sum u^gamma,
@@ -140,7 +140,7 @@ __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1,
         const float h = fabsf(dl);
         const float cross = (dl > 0.f) ? ((gamma >= 2.f) ? F2 * h * h : F1 * h)
                                        : ((gamma >= 2.f) ? h * h : exp2f(gamma * __log2f(h)));
-        if (cross <= acc.cert) {
+        if (cross <= (dl > 0.f ? acc.cert_up : acc.cert_down)) {
             st.tau = next; st.done = 1; st.unv = 1; st.down = dl < 0.f; st.iters = pass; return;
         }
     }

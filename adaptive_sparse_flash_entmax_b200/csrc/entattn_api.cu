@@ -92,7 +92,9 @@ bool bound_enabled() {
 
 // Unverified Halley steps of the bf16 forward (each checked in the P.V pass, see
 // solver_update): steps up to 1e-2 either way whose boundary crossings can change f by
-// at most 1e-5 (upward from the sums, downward per entering element).  ENTATTN_ACCEPT=0
+// at most 5e-5 upward (a bound on all leaving elements together, from the sums: half
+// the check's 1e-4) or 3e-5 per entering element downward (at least four would have to
+// enter within the step to miss the check).  ENTATTN_ACCEPT=0
 // (environment, read per call) stops every row at an evaluated tau instead, for
 // ablations.  ENTATTN_VERIFY_TOL sets the check's tolerance on |sum_j p - 1| (default
 // 1e-4; a negative value makes every tile with such a row be solved again, which
@@ -102,7 +104,8 @@ ent::AcceptRule accept_rule() {
     const char* v = getenv("ENTATTN_ACCEPT");
     if (v && *v && atoi(v) == 0) return r;
     r.step = 1e-2f;
-    r.cert = 1e-5f;
+    r.cert_up = 5e-5f;
+    r.cert_down = 3e-5f;
     return r;
 }
 

@@ -90,8 +90,9 @@ size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype);
  * when |f(tau)| <= 1e-5 (bf16; 1e-6 float32), when its next step is below
  * 1e-6 (4e-7) * max(1, |tau|), or after 24 passes.  The bf16 path also stops
  * on a Halley step it does not evaluate when the step is at most 1e-2 and the
- * support elements that can cross the boundary within it change f by at most
- * 1e-5 (upward: F2 h^2 for gamma >= 2, F1 h below; downward: h^min(gamma,2));
+ * elements that can cross the support boundary within it change f by at most
+ * 5e-5 upward (all leaving elements together: F2 h^2 for gamma >= 2, F1 h
+ * below) or 3e-5 per entering element downward (h^min(gamma,2));
  * the P.V pass then checks |sum_j p_ij - 1| <= 1e-4 at the returned tau, and
  * every query tile with a row that fails the check is solved again with
  * evaluated stops only, by the last CTA of the same launch.  The block mask is

@@ -1,8 +1,9 @@
 """Unevaluated Halley stops of the bf16 forward and their check.
 
 A row may stop on a Halley step it does not evaluate (up to 1e-2 either way, when the
-elements that can cross the support boundary within the step change f by at most
-1e-5); the P.V pass then sums p at the final tau, and a tile where such a row misses
+elements that can cross the support boundary within the step change f by at most 5e-5
+upward, all of them together, or 3e-5 each downward); the P.V pass then sums p at the
+final tau, and a tile where such a row misses
 |sum p - 1| <= 1e-4 goes on a failure list that the last CTA of the grid solves again,
 stopping only at evaluated points.  Checked here: the oracle parity of the default rule
 (every row of a head, every alpha), no more solver passes than with evaluated stops

@@ -135,8 +135,16 @@ __device__ __forceinline__ void hist_bracket_warp(const unsigned int* hist, int 
     tau0 = fminf(fmaxf(t0, lo), hi);
 }
 
-template <typename T, int E, int GM>
-__global__ void __launch_bounds__(kRowThreads) rows_fwd_kernel(const RowArgs a) {
+// HIST: the histogram start (ENT_SOLVE_HIST); the other solvers take a kernel without it.
+// The kernels are bound by the latency of each row's passes, so the rows in flight per SM
+// set their rate: the register caps below (CTAs per SM) are the fastest measured on
+// [16384, 1024], [16384, 4096] and [4096, 16384] bf16 rows (the forward at eight CTAs per
+// SM spills a few words and is still 16 % faster than at three).
+template <int E> constexpr int rows_fwd_ctas() { return E <= 16 ? 8 : 2; }
+template <int E> constexpr int rows_bwd_ctas() { return E <= 4 ? 8 : E <= 16 ? 5 : 1; }
+
+template <typename T, int E, int GM, bool HIST>
+__global__ void __launch_bounds__(kRowThreads, rows_fwd_ctas<E>()) rows_fwd_kernel(const RowArgs a) {
     __shared__ float red[3][kRowWarps];
     __shared__ unsigned int hist[kBins];
     __shared__ float ptab[68];
@@ -161,7 +169,7 @@ __global__ void __launch_bounds__(kRowThreads) rows_fwd_kernel(const RowArgs a) 
     sv.lo = m - 1.f;
     sv.hi = fmaxf(sv.lo, m - exp2f((1.f - a.alpha) * __log2f((float)a.n)));
     sv.tau = 0.5f * (sv.lo + sv.hi);
-    if (a.method == kSolveHist) {
+    if constexpr (HIST) {
         // 64 bins of width 1/63 on the absolute grid under the row max: [m-1, m]
         const int A = abs_bin(m);
         if (tid < kBins) hist[tid] = 0u;
@@ -216,7 +224,7 @@ __global__ void __launch_bounds__(kRowThreads) rows_fwd_kernel(const RowArgs a) 
 }
 
 template <typename T, int E, int GM>
-__global__ void __launch_bounds__(kRowThreads) rows_bwd_kernel(const RowArgs a) {
+__global__ void __launch_bounds__(kRowThreads, rows_bwd_ctas<E>()) rows_bwd_kernel(const RowArgs a) {
     __shared__ float red[3][kRowWarps];
     const int tid = threadIdx.x;
     const size_t off = (size_t)blockIdx.x * a.n;
@@ -251,10 +259,14 @@ cudaError_t rows_launch(const RowArgs& a, bool bwd, cudaStream_t s) {
         if (e <= 4) rows_bwd_kernel<T, 4, GM><<<grid, block, 0, s>>>(a);
         else if (e <= 16) rows_bwd_kernel<T, 16, GM><<<grid, block, 0, s>>>(a);
         else rows_bwd_kernel<T, 64, GM><<<grid, block, 0, s>>>(a);
+    } else if (a.method == kSolveHist) {
+        if (e <= 4) rows_fwd_kernel<T, 4, GM, true><<<grid, block, 0, s>>>(a);
+        else if (e <= 16) rows_fwd_kernel<T, 16, GM, true><<<grid, block, 0, s>>>(a);
+        else rows_fwd_kernel<T, 64, GM, true><<<grid, block, 0, s>>>(a);
     } else {
-        if (e <= 4) rows_fwd_kernel<T, 4, GM><<<grid, block, 0, s>>>(a);
-        else if (e <= 16) rows_fwd_kernel<T, 16, GM><<<grid, block, 0, s>>>(a);
-        else rows_fwd_kernel<T, 64, GM><<<grid, block, 0, s>>>(a);
+        if (e <= 4) rows_fwd_kernel<T, 4, GM, false><<<grid, block, 0, s>>>(a);
+        else if (e <= 16) rows_fwd_kernel<T, 16, GM, false><<<grid, block, 0, s>>>(a);
+        else rows_fwd_kernel<T, 64, GM, false><<<grid, block, 0, s>>>(a);
     }
     return cudaGetLastError();
 }

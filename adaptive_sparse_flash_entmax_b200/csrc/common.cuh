@@ -111,14 +111,15 @@ struct AcceptRule {
 // outside is clamped onto it: a root on a bracket end, such as tau = m - 1 for
 // a one-element support, must stay reachable); otherwise the bracket is bisected.
 // The rule `acc` may also stop a row on a Halley step it takes without evaluating
-// it: near the root Halley's error is cubic in the step while the support stays the
-// same, so what the step can miss is the change of support.  Each element that
-// crosses the boundary within a step h changes f by at most h^gamma.  Upward, only
-// elements of the support (u <= h) can leave: together at most h^2 F2 (gamma >= 2) or
-// h F1 (gamma < 2), from the sums just evaluated.  Downward, the elements that can
-// enter are not counted by the sums; the step is taken when h^min(gamma,2) alone is
-// below the bound (a handful of entering elements stays within the caller's check).
-// Either way the caller checks f at the new tau afterwards.
+// it, when f at the new point is small by two counts.  (1) With the support fixed, f
+// after the step is f + dl f' + dl^2 f''/2 (exact for gamma = 2, whose f is then a
+// quadratic, and for gamma = 1, a line; a Taylor estimate otherwise): Halley's own
+// miss, which is not small where f is not.  (2) Each element that crosses the
+// boundary within a step h changes f by at most h^gamma.  Upward, only elements of the
+// support (u <= h) can leave: together at most h^2 F2 (gamma >= 2) or h F1
+// (gamma < 2), from the sums just evaluated.  Downward, the elements that can enter
+// are not counted by the sums; h^min(gamma,2) per entering element is what the rule
+// bounds.  Either way the caller checks f at the new tau afterwards.
 __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1, float F2,
                                               float gamma, bool gamma_is_one, int pass,
                                               float ftol, float stol,
@@ -140,7 +141,8 @@ __device__ __forceinline__ void solver_update(RowSolver& st, float F0, float F1,
         const float h = fabsf(dl);
         const float cross = (dl > 0.f) ? ((gamma >= 2.f) ? F2 * h * h : F1 * h)
                                        : ((gamma >= 2.f) ? h * h : exp2f(gamma * __log2f(h)));
-        if (cross <= (dl > 0.f ? acc.cert_up : acc.cert_down)) {
+        const float miss = fabsf(f + dl * (fp + 0.5f * dl * fpp));   // fixed-support f after it
+        if (miss + cross <= (dl > 0.f ? acc.cert_up : acc.cert_down)) {
             st.tau = next; st.done = 1; st.unv = 1; st.down = dl < 0.f; st.iters = pass; return;
         }
     }

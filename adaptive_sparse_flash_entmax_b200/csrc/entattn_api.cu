@@ -66,7 +66,7 @@ int hist_budget() {
 // of the statistics pass: per head max |c| and min R (float bits), per 64-key
 // half-block {R, L} and the bf16 centroid.
 struct FwdLayout {
-    size_t maxc, minr, stats, cent, fix, total;
+    size_t maxc, minr, stats, cent, fix, gap, calib, total;
 };
 
 FwdLayout fwd_layout(int B, int H, int N, int d) {
@@ -77,8 +77,21 @@ FwdLayout fwd_layout(int B, int H, int N, int d) {
     L.stats = L.maxc + round_up(BH * 8, 256);
     L.cent = L.stats + round_up(BH * T2 * 8, 256);
     L.fix = L.cent + round_up(BH * T2 * (size_t)d * 2, 256);   // failure list, one int per tile
-    L.total = L.fix + round_up(BH * T2 / 2 * 4, 256);
+    L.gap = L.fix + round_up(BH * T2 / 2 * 4, 256);
+    // calibrated start (sequences of >= kBoundMinBlocks query tiles): the sampled rows'
+    // gaps and scores
+    const bool cal = n_tiles(N) >= ent::kBoundMinBlocks;
+    L.calib = L.gap + (cal ? round_up(BH * ent::kCalRows * 4, 256) : 0);
+    L.total = L.calib + (cal ? round_up(BH * ent::kCalRows * (size_t)N * 4, 256) : 0);
     return L;
+}
+
+// Calibrated solver start (bf16 path, sequences of >= kBoundMinBlocks query tiles), on by
+// default.  ENTATTN_CALIB=0 (environment, read per call) starts every row at the plain
+// bracket's midpoint instead, for ablations; the outputs meet the same stop rule either way.
+bool calib_enabled() {
+    const char* v = getenv("ENTATTN_CALIB");
+    return !(v && *v && atoi(v) == 0);
 }
 
 // Statistics-pass skipping by key-block bounds (bf16 path), on by default.
@@ -263,6 +276,11 @@ ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, i
         a.verify_tol = verify_tol();
         a.spec = spec_enabled();
         a.fail_list = reinterpret_cast<int*>(static_cast<char*>(ws) + FL.fix);
+    }
+    if (dtype == ENT_BF16 && hist_budget() == 0 && calib_enabled() && n_tiles(N) >= ent::kBoundMinBlocks) {
+        char* base = static_cast<char*>(ws);
+        a.gap = reinterpret_cast<float*>(base + FL.gap);
+        a.calib = reinterpret_cast<float*>(base + FL.calib);
     }
     if (bound) {
         // statistics-pass skipping by key-block bounds; off with the histogram start, whose

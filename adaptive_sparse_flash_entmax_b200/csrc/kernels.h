@@ -8,7 +8,8 @@
 namespace ent {
 
 constexpr int kListCap = 16;        // entries per row in the support lists
-constexpr int kBoundMinBlocks = 64; // shortest query tile (key blocks) that runs the bound pass
+constexpr int kBoundMinBlocks = 64;  // shortest query tile (key blocks) that runs the bound pass
+constexpr int kCalRows = 8;          // sampled rows per head of the calibrated start
 constexpr uint8_t kListOver = 255;  // list_n of a row with more than kListCap nonzeros
 
 struct FwdArgs {
@@ -51,6 +52,13 @@ struct FwdArgs {
     void* cent;
     float2* bstats;
     unsigned int* head_words;
+    // Calibrated start (tensor-core path; null: every row starts at the plain bracket's
+    // midpoint).  Per head, kCalRows sampled query rows p_s = (s+1) N / kCalRows - 1 are
+    // solved exactly before the forward: calib [BH][kCalRows][N] holds their scores x,
+    // gap [BH][kCalRows] their m - tau; a row then starts at m - gap of the nearest
+    // sample, clamped into its bracket.
+    float* calib;
+    float* gap;
     // Per-row support lists (nullable; tensor-core path): for each query row the keys j
     // with p_ij > 0 and their u_ij = x_ij - tau_i, up to kListCap of them, in list_key /
     // list_u [BH][N][kListCap]; list_n [BH][N] the count, kListOver when the row has more.

@@ -61,6 +61,7 @@ constexpr int kTmemCols = 512;     // score passes: S [0,256), [256,512); P.V pa
                                    // or, with otilde, G.V [256+D, 256+2D) (and S2 when D = 64)
 constexpr int kDecSolve = 1, kDecPv = 2;
 constexpr uint8_t kPvLive = 255;   // cand[] of a block with a nonzero p in the P.V pass
+constexpr float kCalMargin = 0.03f; // calibrated start: offset below the nearest sample's gap
 
 __host__ __device__ constexpr uint32_t sbuf_col(int sb) { return sb < 2 ? sb * 128 : 384; }
 
@@ -785,11 +786,21 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const int w_other = (int)X(2, half ^ 1);
                 const bool over = (wbins == 0) || (w_other == 0);
                 if (half == 0 && row_valid && over) {
-                    // plain bracket [m-1, m - n^(1-alpha)], start at its midpoint
+                    // plain bracket [m-1, m - n^(1-alpha)], start at its midpoint, or at
+                    // m - (the gap of the nearest sampled row) when the start is calibrated
                     const float mr = fmaxf(m, m_other);
                     sv.lo = mr - 1.f;
                     sv.hi = fmaxf(sv.lo, mr - exp2f((1.f - a.alpha) * __log2f((float)key_end)));
                     sv.tau = 0.5f * (sv.lo + sv.hi);
+                    if (a.gap) {
+                        const int sr = min(max((int)(((long long)(i + 1) * kCalRows + N / 2) / N) - 1, 0), kCalRows - 1);
+                        const float g = a.gap[(size_t)bh * kCalRows + sr];
+                        // kCalMargin below it: from below, Halley approaches the root with
+                        // upward steps, whose unevaluated stops have the rigorous crossing
+                        // bound (a start just above the root ends on a downward stop, which
+                        // on clustered keys can miss the check)
+                        if (g >= 0.f) sv.tau = fminf(fmaxf(mr - g - kCalMargin, sv.lo), sv.hi);
+                    }
                 }
                 named_bar(1, kEw);
                 if (half == 0 && row_valid && over) {
@@ -1232,6 +1243,132 @@ __global__ void __launch_bounds__(128) block_stats_kernel(const __nv_bfloat16* _
     }
 }
 
+// ---------------------------------------------------------------- calibrated start
+// Not on the pages.  A tile runs as many solver passes as its slowest row, and the plain
+// bracket's midpoint m - (1 + n^(1-alpha))/2 sits far from the root where the gap m - tau
+// is small (clustered keys: ~0.27 against ~0.5).  Before the forward, kCalRows query rows
+// per head are solved exactly; each row of the forward then starts at m - (the gap of the
+// nearest sampled row), inside its own bracket.  The result is a deterministic function of
+// the inputs; only the path of the solver changes, not its stop rule.
+//
+// calib_scores_kernel: grid (ceil(N / 256), BH), one key per thread: x = cx q_s . k_j for
+// every sampled row s with j in its (causal) range, q_s staged in shared memory as floats.
+constexpr int kCalThreads = 256;
+
+__global__ void __launch_bounds__(kCalThreads) calib_scores_kernel(const FwdArgs a) {
+    extern __shared__ float qs[];   // [kCalRows][dr]
+    const int bh = blockIdx.y, N = a.N, dr = a.dr;
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q) + (size_t)bh * N * dr;
+    for (int i = threadIdx.x; i < kCalRows * dr; i += kCalThreads) {
+        const int sidx = i / dr, c = i - sidx * dr;
+        const int p = (sidx + 1) * N / kCalRows - 1;
+        qs[i] = __bfloat162float(q[(size_t)p * dr + c]);
+    }
+    __syncthreads();
+    const int j = blockIdx.x * kCalThreads + threadIdx.x;
+    if (j >= N) return;
+    // causal: the sampled rows before this CTA's first key take none of its keys (the
+    // rows are in increasing order, so those are the first r0 of them)
+    int r0 = 0;
+    if (a.causal)
+        while (r0 < kCalRows && (r0 + 1) * N / kCalRows - 1 < (int)(blockIdx.x * kCalThreads)) ++r0;
+    const __nv_bfloat16* kr = static_cast<const __nv_bfloat16*>(a.k) + ((size_t)bh * N + j) * dr;
+    float acc[kCalRows];
+#pragma unroll
+    for (int r = 0; r < kCalRows; ++r) acc[r] = 0.f;
+    for (int c = 0; c < dr; c += 8) {
+        const uint4 w = *reinterpret_cast<const uint4*>(kr + c);
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+        float kv[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+            kv[2 * e] = f.x;
+            kv[2 * e + 1] = f.y;
+        }
+#pragma unroll
+        for (int r = 0; r < kCalRows; ++r) {
+            if (r < r0) continue;
+            const float4 qa = *reinterpret_cast<const float4*>(qs + r * dr + c);
+            const float4 qb = *reinterpret_cast<const float4*>(qs + r * dr + c + 4);
+            acc[r] = fmaf(qa.x, kv[0], acc[r]); acc[r] = fmaf(qa.y, kv[1], acc[r]);
+            acc[r] = fmaf(qa.z, kv[2], acc[r]); acc[r] = fmaf(qa.w, kv[3], acc[r]);
+            acc[r] = fmaf(qb.x, kv[4], acc[r]); acc[r] = fmaf(qb.y, kv[5], acc[r]);
+            acc[r] = fmaf(qb.z, kv[6], acc[r]); acc[r] = fmaf(qb.w, kv[7], acc[r]);
+        }
+    }
+    float* out = a.calib + (size_t)bh * kCalRows * N;
+#pragma unroll
+    for (int r = 0; r < kCalRows; ++r) {
+        const int p = (r + 1) * N / kCalRows - 1;
+        if (!a.causal || j <= p) out[(size_t)r * N + j] = a.cx * acc[r];
+    }
+}
+
+// calib_solve_kernel: grid (kCalRows, BH), one CTA per sampled row: the row maximum, then
+// Halley-bisection passes from the plain bracket with evaluated stops only (the forward's
+// stop rule), the sums reduced over the CTA; writes gap = m - tau.
+template <int GM>
+__global__ void __launch_bounds__(kCalThreads) calib_solve_kernel(const FwdArgs a) {
+    __shared__ float red[3][kCalThreads / 32];
+    __shared__ float bc[2];
+    const int r = blockIdx.x, bh = blockIdx.y, N = a.N;
+    const int p = (r + 1) * N / kCalRows - 1;
+    const int n = a.causal ? p + 1 : N;
+    const float* x = a.calib + ((size_t)bh * kCalRows + r) * N;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    auto reduce3 = [&](float& u, float& v, float& w, bool is_max) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            if (is_max) {
+                u = fmaxf(u, __shfl_xor_sync(0xffffffffu, u, o));
+            } else {
+                u += __shfl_xor_sync(0xffffffffu, u, o);
+                v += __shfl_xor_sync(0xffffffffu, v, o);
+                w += __shfl_xor_sync(0xffffffffu, w, o);
+            }
+        }
+        __syncthreads();   // the previous use of red is finished
+        if (lane == 0) { red[0][warp] = u; red[1][warp] = v; red[2][warp] = w; }
+        __syncthreads();
+        u = red[0][0]; v = red[1][0]; w = red[2][0];
+#pragma unroll
+        for (int i = 1; i < kCalThreads / 32; ++i) {
+            if (is_max) u = fmaxf(u, red[0][i]);
+            else { u += red[0][i]; v += red[1][i]; w += red[2][i]; }
+        }
+    };
+    float m = -INFINITY, d1 = 0.f, d2 = 0.f;
+    for (int j = threadIdx.x; j < n; j += kCalThreads) m = fmaxf(m, x[j]);
+    reduce3(m, d1, d2, true);
+    RowSolver sv;
+    sv.done = 0;
+    sv.iters = 0;
+    sv.lo = m - 1.f;
+    sv.hi = fmaxf(sv.lo, m - exp2f((1.f - a.alpha) * __log2f((float)n)));
+    sv.tau = 0.5f * (sv.lo + sv.hi);
+    const float gamma = a.gamma;
+    for (int pass = 1;; ++pass) {
+        float2 s0 = make_float2(0.f, 0.f), s1 = s0, s2 = s0;
+        const float2 nt2 = make_float2(-sv.tau, -sv.tau);
+        for (int j = 2 * threadIdx.x; j < n; j += 2 * kCalThreads) {
+            const float2 xx = make_float2(x[j], j + 1 < n ? x[j + 1] : -INFINITY);
+            entmax_acc_x2<GM>(__fadd2_rn(xx, nt2), gamma, s0, s1, s2);
+        }
+        float F0 = s0.x + s0.y, F1 = s1.x + s1.y, F2 = s2.x + s2.y;
+        reduce3(F0, F1, F2, false);
+        if (threadIdx.x == 0) {
+            solver_update(sv, F0, F1, F2, gamma, gamma == 1.f, pass, a.ftol, a.stol);
+            bc[0] = sv.tau;
+            bc[1] = sv.done ? 1.f : 0.f;
+        }
+        __syncthreads();
+        sv.tau = bc[0];
+        if (bc[1] != 0.f) break;
+    }
+    if (threadIdx.x == 0) a.gap[(size_t)bh * kCalRows + r] = m - sv.tau;
+}
+
 template <int D, int GM>
 static cudaError_t launch_tc_fwd(const CUtensorMap& mq, const CUtensorMap& mk,
                                  const CUtensorMap& mv, const CUtensorMap& mc, const FwdArgs& a,
@@ -1245,6 +1382,13 @@ static cudaError_t launch_tc_fwd(const CUtensorMap& mq, const CUtensorMap& mk,
             block_stats_kernel<32><<<grid, 128, 0, s>>>(kk, a.N, T2, cc, a.bstats, a.head_words);
         else
             block_stats_kernel<D><<<grid, 128, 0, s>>>(kk, a.N, T2, cc, a.bstats, a.head_words);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (a.gap) {
+        const size_t qsm = (size_t)kCalRows * a.dr * sizeof(float);
+        calib_scores_kernel<<<dim3((a.N + kCalThreads - 1) / kCalThreads, a.BH), kCalThreads, qsm, s>>>(a);
+        calib_solve_kernel<GM><<<dim3(kCalRows, a.BH), kCalThreads, 0, s>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

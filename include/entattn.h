@@ -73,6 +73,9 @@ int ent_attn_block_size(void);
 
 /*
  * Bytes of device workspace the forward / backward need for this shape.
+ * The forward's (bf16) holds the centroid bounds of the statistics pass, the list
+ * of query tiles to solve again and, for N of at least 64 query tiles, the scores
+ * of 8 sampled query rows per head (B*H*8*N floats) for the calibrated start.
  * The backward's is the 256-byte header plus delta, one float per query row:
  * 256 + round_up(B*H*N*4, 256).  A negative size gives 0.
  */
@@ -103,9 +106,11 @@ size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype);
  * ENTATTN_SPEC=0 (no speculative first job: by default the K blocks of a score
  * pass's first job are loaded and multiplied again before the decision that
  * ends the pass, and used if the next pass starts with the same job).
- * bf16 inputs start every row's solver from the plain bracket [m-1, m - n^(1-alpha)]
+ * bf16 inputs start every row's solver inside the plain bracket [m-1, m - n^(1-alpha)]
  * (measured faster on B200 than the histogram start, whose inserts cost more than
- * the passes they save).  The environment variable ENTATTN_HIST_BUDGET, read at each
+ * the passes they save): at its midpoint, or, for N of at least 64 query tiles, at
+ * m - g, g = m - tau of the nearest of 8 query rows per head that two small kernels
+ * solve exactly before the forward (ENTATTN_CALIB=0: the midpoint always).  The environment variable ENTATTN_HIST_BUDGET, read at each
  * call, selects the histogram start of the statistics pass instead: a tile builds
  * the histogram until it has made that many inserts after its first block (a
  * negative value: no limit).  float32 inputs always use the histogram start.  The

@@ -75,3 +75,22 @@ def test_resolved_tiles_match_evaluated_stops(name, change, otilde, monkeypatch)
         if a is not None:
             assert torch.equal(a, b)
     assert cf[3] > c0[3]                        # tiles were solved again
+
+
+@pytest.mark.parametrize("beta", [1.0, 2.0])
+def test_clustered_rows_need_no_second_solve(beta, monkeypatch):
+    """Clustered keys put many scores next to tau.  A Halley step stopped unevaluated must
+    account for its own miss on the fixed support, not only for the elements crossing the
+    boundary: without that term, about 3 % of the long workload's tiles at beta 1 failed
+    the P.V check and were solved a second time, serially, by the last CTA (a forward of
+    18 ms instead of 2.9)."""
+    from fullsize import check_forward
+    w = inputs.WORKLOADS["long"].replace(H=2, beta=beta)
+    q, k, v, _ = inputs.make_inputs(w, seed=10)
+    qd, kd, vd = (to_dev(a, "bf16") for a in (q, k, v))
+    for calib in ("0", "1"):
+        monkeypatch.setenv("ENTATTN_CALIB", calib)
+        (o, tau, mask, _, _), c = _fwd(w, qd, kd, vd)
+        assert c[3] == w.B * w.H * ((w.N + 127) // 128)   # every tile solved once
+        res = check_forward(qd, kd, vd, tau, mask, o, w.alpha, w.causal)
+        assert res["rows"] == w.B * w.H * w.N

@@ -30,7 +30,8 @@ struct WsHeader {
     unsigned int tile_counter;     // forward: CTAs finished (the last one re-solves failed tiles)
     unsigned int fail_count;       // forward: tiles on the failure list
     unsigned long long counters[8];
-    unsigned char pad1[256 - 16 - 64];
+    unsigned int claim;            // forward: failure-list entries taken for solving again
+    unsigned char pad1[256 - 16 - 64 - 4];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 

@@ -72,12 +72,12 @@ struct FwdLayout {
 FwdLayout fwd_layout(int B, int H, int N, int d) {
     const size_t BH = (size_t)B * H, T2 = 2 * (size_t)n_tiles(N);
     FwdLayout L;
-    L.maxc = kHdr;                       // [BH] words, then min R [BH] right after them
+    L.fix = kHdr;                        // failure list, one int per tile (zeroed with the header)
+    L.maxc = L.fix + round_up(BH * T2 / 2 * 4, 256);   // [BH] words, then min R [BH]
     L.minr = L.maxc + BH * 4;
     L.stats = L.maxc + round_up(BH * 8, 256);
     L.cent = L.stats + round_up(BH * T2 * 8, 256);
-    L.fix = L.cent + round_up(BH * T2 * (size_t)d * 2, 256);   // failure list, one int per tile
-    L.gap = L.fix + round_up(BH * T2 / 2 * 4, 256);
+    L.gap = L.cent + round_up(BH * T2 * (size_t)d * 2, 256);
     // calibrated start (sequences of >= kBoundMinBlocks query tiles): the sampled rows'
     // gaps and scores
     const bool cal = n_tiles(N) >= ent::kBoundMinBlocks;
@@ -250,8 +250,9 @@ ent_status fwd_impl(const void* q, const void* k, const void* v, int B, int H, i
     // (no tile of a shorter sequence runs the bound pass, so its statistics are not computed)
     const bool bound = dtype == ENT_BF16 && hist_budget() == 0 && bound_enabled() && !empty &&
                        n_tiles(N) >= ent::kBoundMinBlocks;
-    // header and the per-head max |c| start at 0, the per-head min R at all ones
-    cudaError_t e = cudaMemsetAsync(ws, 0, bound ? FL.minr : kHdr, s);
+    // header, failure list (entries are tile + 1, 0 until written) and the per-head max |c|
+    // start at 0, the per-head min R at all ones
+    cudaError_t e = cudaMemsetAsync(ws, 0, bound ? FL.minr : (dtype == ENT_BF16 ? FL.maxc : kHdr), s);
     if (e == cudaSuccess && bound) e = cudaMemsetAsync(static_cast<char*>(ws) + FL.minr, 0xFF, (size_t)B * H * 4, s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace header");
     if (empty) return ENT_OK;

@@ -32,8 +32,9 @@ struct FwdArgs {
                            // first block (0: no histogram, < 0: no limit)
     // Unverified Halley steps (tensor-core path): the rule, and the check in the P.V pass
     // (|sum_j p_ij - 1| <= verify_tol for every row that stopped on one).  A tile that
-    // fails it goes on the failure list fail_list [BH*T] (count in the workspace header);
-    // the last CTA of the grid to finish solves those tiles again with evaluated stops.
+    // fails it goes on the failure list fail_list [BH*T] (tile + 1; count and claim counter
+    // in the workspace header); CTAs that finished their own tile claim the entries and
+    // solve those tiles again with evaluated stops.
     AcceptRule acc;
     float verify_tol;
     int* fail_list;

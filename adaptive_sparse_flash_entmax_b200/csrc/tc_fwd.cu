@@ -193,13 +193,12 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tmem_alloc(&misc->tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    // This CTA's tile, then (last CTA of the grid only) the tiles on the failure list.
+    // This CTA's tile, then tiles from the failure list that it claims.
     // grid (BH, T): the heads' longest causal tiles are dispatched first, all of them
     // before any shorter one, so the last wave holds the shortest tiles
     int cur_t = a.causal ? (T - 1 - (int)blockIdx.y) : (int)blockIdx.y;
     int cur_bh = blockIdx.x;
     bool fixing = false;
-    int fail_cursor = 0;
     for (int rep = 0;; ++rep) {
     const int t = cur_t;
     const int bh = cur_bh;
@@ -1060,7 +1059,7 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const bool bad = ok && row_valid && sv.unv && !(fabsf(f_end) <= a.verify_tol);
         const bool tile_bad = !named_bar_and(1, kEw, !bad);
         if (tile_bad && ew == 0) {
-            a.fail_list[atomicAdd(&a.hdr->fail_count, 1u)] = bh * T + t;
+            a.fail_list[atomicAdd(&a.hdr->fail_count, 1u)] = bh * T + t + 1;   // 0: not written yet
             __threadfence();   // the entry is visible before this CTA counts itself finished
         }
         uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
@@ -1077,19 +1076,36 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     tc_fence_before();
     __syncthreads();
-    // next: for the last CTA of the grid to finish, the tiles on the failure list
+    // next: a tile from the failure list, claimed by whichever CTA is free.  A CTA that
+    // finishes its own tile takes the entries appended so far; the last CTA to finish
+    // its own tile sees every entry (each failing tile appends before it counts itself
+    // finished) and leaves only when all are claimed.  Re-solved tiles stop at evaluated
+    // points only, so they never append.  An entry holds its tile + 1 (the host zeroes the
+    // list), and a claimer waits (bounded) for its entry to be written.
     if (threadIdx.x == 0) {
         int next = -1;
         if (!misc->abort) {
-            bool last = fixing;
             if (!fixing) {
                 __threadfence();
-                last = atomicAdd(&a.hdr->tile_counter, 1u) == gridDim.x * gridDim.y - 1;
+                atomicAdd(&a.hdr->tile_counter, 1u);
                 __threadfence();
             }
-            if (last) {
-                const int nfail = (int)*reinterpret_cast<volatile unsigned int*>(&a.hdr->fail_count);
-                if (fail_cursor < nfail) next = reinterpret_cast<volatile int*>(a.fail_list)[fail_cursor];
+            volatile unsigned int* vcount = &a.hdr->fail_count;
+            volatile unsigned int* vclaim = &a.hdr->claim;
+            for (;;) {
+                const unsigned int c = *vclaim;
+                if (c >= *vcount) break;
+                if (atomicCAS(&a.hdr->claim, c, c + 1u) != c) continue;
+                const volatile int* entry = reinterpret_cast<volatile int*>(a.fail_list) + c;
+                const uint64_t t0 = globaltimer_ns();
+                int e = *entry;
+                while (e == 0 && globaltimer_ns() - t0 <= kWaitLimitNs) e = *entry;
+                if (e == 0) {   // never written: give up like any other bounded wait
+                    atomicExch(&a.hdr->status, 1u);
+                    atomicExch(&a.hdr->timeout_site, 15u);
+                }
+                next = e - 1;
+                break;
             }
         }
         misc->next = next;
@@ -1098,7 +1114,6 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int next = misc->next;
     if (next < 0) break;
     fixing = true;
-    ++fail_cursor;
     cur_bh = next / T;
     cur_t = next - cur_bh * T;
     tc_fence_after();

@@ -98,7 +98,7 @@ size_t ent_attn_bwd_workspace_size(int B, int H, int N, int d, int dtype);
  * below) or 3e-5 per entering element downward (h^min(gamma,2));
  * the P.V pass then checks |sum_j p_ij - 1| <= 1e-4 at the returned tau, and
  * every query tile with a row that fails the check is solved again with
- * evaluated stops only, by the last CTA of the same launch.  The block mask is
+ * evaluated stops only, by the CTAs of the same launch that are free.  The block mask is
  * written from p > 0 at the returned tau, so it is exact for that tau.
  * Environment switches read at each call, for ablations: ENTATTN_ACCEPT=0 (no
  * unevaluated stops), ENTATTN_VERIFY_TOL (the check's tolerance; negative:

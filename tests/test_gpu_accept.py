@@ -4,8 +4,8 @@ A row may stop on a Halley step it does not evaluate (up to 1e-2 either way, whe
 elements that can cross the support boundary within the step change f by at most 5e-5
 upward, all of them together, or 3e-5 each downward); the P.V pass then sums p at the
 final tau, and a tile where such a row misses
-|sum p - 1| <= 1e-4 goes on a failure list that the last CTA of the grid solves again,
-stopping only at evaluated points.  Checked here: the oracle parity of the default rule
+|sum p - 1| <= 1e-4 goes on a failure list whose tiles the CTAs that are free solve
+again, stopping only at evaluated points.  Checked here: the oracle parity of the default rule
 (every row of a head, every alpha), no more solver passes than with evaluated stops
 only, and the re-solve path: with a negative tolerance every such tile goes through
 it, and the outputs are then bit-identical to those of evaluated stops only
@@ -82,8 +82,8 @@ def test_clustered_rows_need_no_second_solve(beta, monkeypatch):
     """Clustered keys put many scores next to tau.  A Halley step stopped unevaluated must
     account for its own miss on the fixed support, not only for the elements crossing the
     boundary: without that term, about 3 % of the long workload's tiles at beta 1 failed
-    the P.V check and were solved a second time, serially, by the last CTA (a forward of
-    18 ms instead of 2.9)."""
+    the P.V check and were solved a second time (then serially, by the last CTA: a forward
+    of 18 ms instead of 2.9)."""
     from fullsize import check_forward
     w = inputs.WORKLOADS["long"].replace(H=2, beta=beta)
     q, k, v, _ = inputs.make_inputs(w, seed=10)

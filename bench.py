@@ -104,8 +104,11 @@ def config_of(w, n_gpus, extra=None):
     if w.kind == "clustered":
         c["cluster_span"] = w.span
     hb = os.environ.get("ENTATTN_HIST_BUDGET")
-    c["tau_start"] = ("plain bracket" if not hb or int(hb) == 0 else
-                      f"histogram (insert budget {hb})")
+    calib = (w.dtype == "bf16" and -(-w.N // 128) >= 64
+             and os.environ.get("ENTATTN_CALIB", "1") != "0")
+    c["tau_start"] = (f"histogram (insert budget {hb})" if hb and int(hb) != 0 else
+                      "plain bracket, calibrated (8 sampled rows per head)" if calib else
+                      "plain bracket midpoint")
     if hb:
         c["hist_budget"] = int(hb)
     if extra:
@@ -393,17 +396,19 @@ def combine_ranks(ms: float, units: float, world: int, device) -> tuple:
 
 
 def launches_per_step(dtype, delta, T):
-    """Kernels of this library launched per step.  bf16: the key-block statistics (at
-    least 64 query tiles, unless ENTATTN_BOUND=0 or the histogram start is selected),
-    the forward (which also re-solves, in its last CTA, any tile that failed the check of
-    its unevaluated stops), the support-list backward (lists only), dq and dkv.  float32:
-    the forward and three backward kernels."""
+    """Kernels of this library launched per step.  bf16: the key-block statistics and the
+    two kernels of the calibrated start (each at least 64 query tiles, unless
+    ENTATTN_BOUND=0 / ENTATTN_CALIB=0 or the histogram start is selected), the forward
+    (whose free CTAs also re-solve any tile that failed the check of its unevaluated
+    stops), the support-list backward (lists only), dq and dkv.  float32: the forward and
+    three backward kernels."""
     if dtype != "bf16":
         return 4
     hb = os.environ.get("ENTATTN_HIST_BUDGET")
-    bound = (os.environ.get("ENTATTN_BOUND", "1") != "0" and (not hb or int(hb) == 0)
-             and T >= 64)
-    return int(bound) + 1 + (1 if delta == "lists" else 0) + 2
+    plain = (not hb or int(hb) == 0) and T >= 64
+    bound = os.environ.get("ENTATTN_BOUND", "1") != "0" and plain
+    calib = os.environ.get("ENTATTN_CALIB", "1") != "0" and plain
+    return int(bound) + 2 * int(calib) + 1 + (1 if delta == "lists" else 0) + 2
 
 
 SWEEP = ([("iid", {"beta": b}) for b in (1.0, 2.0, 4.0, 8.0)]

@@ -62,6 +62,19 @@ int hist_budget() {
     return 0;
 }
 
+// A non-blocking stream per device for work forked from the caller's stream (created on
+// first use, kept for the life of the process); null if it cannot be created.
+cudaStream_t side_stream() {
+    static cudaStream_t streams[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+        streams[dev] = nullptr;
+    return streams[dev];
+}
+
 // Forward workspace layout: the 256-byte header, then (bf16 path) the key-block bounds
 // of the statistics pass: per head max |c| and min R (float bits), per 64-key
 // half-block {R, L} and the bf16 centroid.
@@ -360,9 +373,25 @@ ent_status bwd_impl(const void* q, const void* k, const void* v, const float* ot
         e = ent::simt_bwd_f32(a, d, gm, s);
     } else {
         const char* why = nullptr;
-        // the list kernel first: it decides which query tiles it covers
-        if (lists.want) e = ent::list_bwd(a, d, gm, s);
-        if (e == cudaSuccess) e = ent::tc_bwd(a, d, gm, s, &why);
+        if (lists.want) {
+            // the list kernel and dq take disjoint query tiles (both decide from the list
+            // counts) and run at the same time, the list kernel on a side stream forked
+            // from `s`; dkv, which adds the list kernel's accumulators, joins it
+            cudaStream_t side = side_stream();
+            cudaEvent_t fork = nullptr, join = nullptr;
+            if (!side) side = s;   // no side stream: the two run one after the other
+            e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventRecord(fork, s);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+            if (e == cudaSuccess) e = ent::list_bwd(a, d, gm, side);
+            if (e == cudaSuccess) e = cudaEventRecord(join, side);
+            if (e == cudaSuccess) e = ent::tc_bwd(a, d, gm, s, &why, join);
+            if (fork) cudaEventDestroy(fork);   // released once the recorded work is done
+            if (join) cudaEventDestroy(join);
+        } else {
+            e = ent::tc_bwd(a, d, gm, s, &why);
+        }
         if (e != cudaSuccess && why) return fail(ENT_ECUDA, "backward launch: %s", why);
     }
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");

@@ -122,7 +122,9 @@ cudaError_t simt_bwd_f32(const BwdArgs& a, int d, int gm, cudaStream_t s);
 
 // bf16 tensor-core path (tcgen05 + TMEM + TMA).  `why` names a host-side failure.
 cudaError_t tc_fwd(const FwdArgs& a, int d, int gm, cudaStream_t s, const char** why);
-cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char** why);
+// before_dkv (nullable): an event the dkv kernel waits for (the list kernel's end).
+cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char** why,
+                   cudaEvent_t before_dkv = nullptr);
 
 // Support-list backward of the query tiles whose rows all have lists (tc_lists.cu): dQ of
 // those rows, their dK / dV contributions added into dk_acc / dv_acc, and tile_list.

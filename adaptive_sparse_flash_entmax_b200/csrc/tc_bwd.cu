@@ -161,8 +161,15 @@ tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int bh = blockIdx.x;
     const int nblk = a.causal ? t + 1 : T;
     const Abort ab{&misc->abort, a.hdr};
-    // a tile the support-list kernel covered (its dQ is written) is done
-    if (a.tile_list && a.tile_list[(size_t)bh * T + t]) return;
+    // a tile every row of which has a support list is the list kernel's (it writes that
+    // dQ); the decision is the list kernel's own rule, taken here from the same list
+    // counts, so the two kernels can run at the same time
+    if (a.list_n) {
+        bool has = true;
+        if (threadIdx.x < kBlk && t * kBlk + (int)threadIdx.x < N)
+            has = a.list_n[(size_t)bh * N + t * kBlk + threadIdx.x] != kListOver;
+        if (__syncthreads_and(has)) return;
+    }
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < KS; ++i) { mbar_init(&kfull[i], 1); mbar_init(&kempty[i], 1); }
@@ -813,7 +820,8 @@ tc_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 
 // ------------------------------------------------------------------ host side
 template <int D, int GM>
-static cudaError_t launch_tc_bwd(const BwdArgs& a, cudaStream_t s, const CUtensorMap* m) {
+static cudaError_t launch_tc_bwd(const BwdArgs& a, cudaStream_t s, const CUtensorMap* m,
+                                 cudaEvent_t before_dkv) {
     // m: q128, do128, k128, v128, q64, do64
     {
         const size_t sm = DqLayout<D>::bytes(a.T);
@@ -822,6 +830,11 @@ static cudaError_t launch_tc_bwd(const BwdArgs& a, cudaStream_t s, const CUtenso
         if (e != cudaSuccess) return e;
         kern<<<dim3(a.BH, a.T), kThreads, sm, s>>>(m[0], m[1], m[2], m[3], a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    // dkv adds the list kernel's accumulators: it waits for that kernel here
+    if (before_dkv) {
+        cudaError_t e = cudaStreamWaitEvent(s, before_dkv, 0);
+        if (e != cudaSuccess) return e;
     }
     const size_t sm = DkvLayout<D>::bytes(a.T);
     auto kern = tc_bwd_dkv_kernel<D, GM>;
@@ -832,16 +845,18 @@ static cudaError_t launch_tc_bwd(const BwdArgs& a, cudaStream_t s, const CUtenso
 }
 
 template <int D>
-static cudaError_t tc_bwd_d(const BwdArgs& a, int gm, cudaStream_t s, const CUtensorMap* m) {
+static cudaError_t tc_bwd_d(const BwdArgs& a, int gm, cudaStream_t s, const CUtensorMap* m,
+                            cudaEvent_t before_dkv) {
     switch (gm) {
-        case 1: return launch_tc_bwd<D, 1>(a, s, m);
-        case 2: return launch_tc_bwd<D, 2>(a, s, m);
-        case 4: return launch_tc_bwd<D, 4>(a, s, m);
-        default: return launch_tc_bwd<D, 0>(a, s, m);
+        case 1: return launch_tc_bwd<D, 1>(a, s, m, before_dkv);
+        case 2: return launch_tc_bwd<D, 2>(a, s, m, before_dkv);
+        case 4: return launch_tc_bwd<D, 4>(a, s, m, before_dkv);
+        default: return launch_tc_bwd<D, 0>(a, s, m, before_dkv);
     }
 }
 
-cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char** why) {
+cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char** why,
+                   cudaEvent_t before_dkv) {
     CUtensorMap m[6];
     const bool ok = make_tmap_bf16_rows(&m[0], a.q, a.BH, a.N, d, 128) &&
                     make_tmap_bf16_rows(&m[1], a.dout, a.BH, a.N, d, 128) &&
@@ -854,7 +869,7 @@ cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char**
         return cudaErrorInvalidValue;
     }
     // d = 32 runs on the d = 64 kernels (zero-filled upper columns, see tc_fwd)
-    return d == 128 ? tc_bwd_d<128>(a, gm, s, m) : tc_bwd_d<64>(a, gm, s, m);
+    return d == 128 ? tc_bwd_d<128>(a, gm, s, m, before_dkv) : tc_bwd_d<64>(a, gm, s, m, before_dkv);
 }
 
 }  // namespace ent

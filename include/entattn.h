@@ -191,7 +191,11 @@ ent_status ent_attn_bwd_otilde(const void *q, const void *k, const void *v, cons
  * tiles by the block kernels of ent_attn_bwd.  Same outputs as ent_attn_bwd (up to
  * fp32 summation order: dK and dV collect the list contributions by atomic adds).
  * Its workspace: ent_attn_bwd_lists_workspace_size (ent_attn_bwd's plus one byte per
- * query tile and two float [B,H,N,d] accumulators).
+ * query tile and two float [B,H,N,d] accumulators).  The list kernel runs on a
+ * library-owned non-blocking stream (one per device) forked from `stream` by an
+ * event and joined back into it before the last kernel, so the work is ordered
+ * after everything enqueued on `stream` before the call and complete when `stream`
+ * passes the call (stream capture sees the same fork and join).
  */
 int ent_attn_list_cap(void);
 size_t ent_attn_bwd_lists_workspace_size(int B, int H, int N, int d, int dtype);

@@ -11,6 +11,23 @@
 #include "../../include/entattn.h"
 #include "kernels.h"
 
+namespace ent {
+
+// A non-blocking stream per device for work forked from the caller's stream (created on
+// first use, kept for the life of the process); null if it cannot be created.
+cudaStream_t side_stream() {
+    static cudaStream_t streams[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+        streams[dev] = nullptr;
+    return streams[dev];
+}
+
+}  // namespace ent
+
 namespace {
 
 thread_local std::string g_err;
@@ -60,19 +77,6 @@ int hist_budget() {
     const char* v = getenv("ENTATTN_HIST_BUDGET");
     if (v && *v) return atoi(v);
     return 0;
-}
-
-// A non-blocking stream per device for work forked from the caller's stream (created on
-// first use, kept for the life of the process); null if it cannot be created.
-cudaStream_t side_stream() {
-    static cudaStream_t streams[64] = {};
-    static std::mutex mu;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
-        streams[dev] = nullptr;
-    return streams[dev];
 }
 
 // Forward workspace layout: the 256-byte header, then (bf16 path) the key-block bounds
@@ -377,7 +381,7 @@ ent_status bwd_impl(const void* q, const void* k, const void* v, const float* ot
             // the list kernel and dq take disjoint query tiles (both decide from the list
             // counts) and run at the same time, the list kernel on a side stream forked
             // from `s`; dkv, which adds the list kernel's accumulators, joins it
-            cudaStream_t side = side_stream();
+            cudaStream_t side = ent::side_stream();
             cudaEvent_t fork = nullptr, join = nullptr;
             if (!side) side = s;   // no side stream: the two run one after the other
             e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);

@@ -122,6 +122,10 @@ cudaError_t simt_bwd_f32(const BwdArgs& a, int d, int gm, cudaStream_t s);
 
 // bf16 tensor-core path (tcgen05 + TMEM + TMA).  `why` names a host-side failure.
 cudaError_t tc_fwd(const FwdArgs& a, int d, int gm, cudaStream_t s, const char** why);
+// A non-blocking stream per device for work forked from the caller's stream (null if it
+// cannot be created); defined with the ABI.
+cudaStream_t side_stream();
+
 // before_dkv (nullable): an event the dkv kernel waits for (the list kernel's end).
 cudaError_t tc_bwd(const BwdArgs& a, int d, int gm, cudaStream_t s, const char** why,
                    cudaEvent_t before_dkv = nullptr);

@@ -1388,6 +1388,27 @@ template <int D, int GM>
 static cudaError_t launch_tc_fwd(const CUtensorMap& mq, const CUtensorMap& mk,
                                  const CUtensorMap& mv, const CUtensorMap& mc, const FwdArgs& a,
                                  cudaStream_t s) {
+    // the calibrated start's two kernels run beside the block statistics (both only read
+    // the inputs), on a stream forked from `s` and joined before the forward
+    cudaStream_t side = (a.gap && a.bstats) ? side_stream() : nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    if (side && (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
+                 cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess ||
+                 cudaEventRecord(fork, s) != cudaSuccess || cudaStreamWaitEvent(side, fork, 0) != cudaSuccess))
+        side = nullptr;   // then on `s`, one after the other
+    if (!side) {
+        if (fork) cudaEventDestroy(fork);
+        if (join) cudaEventDestroy(join);
+    }
+    if (a.gap) {
+        cudaStream_t cs = side ? side : s;
+        const size_t qsm = (size_t)kCalRows * a.dr * sizeof(float);
+        calib_scores_kernel<<<dim3((a.N + kCalThreads - 1) / kCalThreads, a.BH), kCalThreads, qsm, cs>>>(a);
+        calib_solve_kernel<GM><<<dim3(kCalRows, a.BH), kCalThreads, 0, cs>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e == cudaSuccess && side) e = cudaEventRecord(join, side);
+        if (e != cudaSuccess) return e;
+    }
     if (a.bstats) {
         const int T2 = 2 * a.T;
         const dim3 grid((T2 + 3) / 4, a.BH);
@@ -1400,11 +1421,10 @@ static cudaError_t launch_tc_fwd(const CUtensorMap& mq, const CUtensorMap& mk,
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    if (a.gap) {
-        const size_t qsm = (size_t)kCalRows * a.dr * sizeof(float);
-        calib_scores_kernel<<<dim3((a.N + kCalThreads - 1) / kCalThreads, a.BH), kCalThreads, qsm, s>>>(a);
-        calib_solve_kernel<GM><<<dim3(kCalRows, a.BH), kCalThreads, 0, s>>>(a);
-        cudaError_t e = cudaGetLastError();
+    if (side) {
+        cudaError_t e = cudaStreamWaitEvent(s, join, 0);
+        cudaEventDestroy(fork);
+        cudaEventDestroy(join);
         if (e != cudaSuccess) return e;
     }
     const size_t sm = Layout<D>::bytes(a.T);

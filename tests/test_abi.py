@@ -35,6 +35,12 @@ def test_sizes(lib):
         rows = B * H * N * 4
         assert capi.ent_attn_bwd_workspace_size(B, H, N, d, capi.ENT_BF16) == 256 + -(-rows // 256) * 256
     assert capi.ent_attn_bwd_workspace_size(-1, 1, 128, 64, capi.ENT_BF16) == 0
+    # sequences of >= 64 query tiles also hold the calibrated start's scores: 8 sampled rows
+    # of N floats per head, which shorter ones do not need
+    short = capi.ent_attn_fwd_workspace_size(2, 3, 63 * 128, 64, capi.ENT_BF16)
+    long_ = capi.ent_attn_fwd_workspace_size(2, 3, 64 * 128, 64, capi.ENT_BF16)
+    assert long_ - short >= 2 * 3 * 8 * 64 * 128 * 4
+    assert long_ % 256 == 0 and short % 256 == 0
 
 
 FAKE = 1 << 20   # a 16-byte-aligned non-null value; never dereferenced on argument errors

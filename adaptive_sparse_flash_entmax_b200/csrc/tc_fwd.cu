@@ -1058,12 +1058,18 @@ tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const float f_end = X(3, 0) + X(3, 1) - 1.f;
         const bool bad = ok && row_valid && sv.unv && !(fabsf(f_end) <= a.verify_tol);
         const bool tile_bad = !named_bar_and(1, kEw, !bad);
-        if (tile_bad && ew == 0) {
-            a.fail_list[atomicAdd(&a.hdr->fail_count, 1u)] = bh * T + t + 1;   // 0: not written yet
-            __threadfence();   // the entry is visible before this CTA counts itself finished
-        }
         uint8_t* mrow = a.mask + ((size_t)bh * T + t) * T;
         for (int bb = ew; bb < T; bb += kEw) mrow[bb] = (bb < nblk && cand[bb] == kPvLive) ? 1 : 0;
+        if (tile_bad) {
+            // every output of this tile is written before the entry is: a CTA that claims
+            // it writes them again, and its writes must land last
+            named_bar(1, kEw);
+            if (ew == 0) {
+                __threadfence();
+                a.fail_list[atomicAdd(&a.hdr->fail_count, 1u)] = bh * T + t + 1;   // 0: not written yet
+                __threadfence();
+            }
+        }
         if (ew == 0) {
             atomicAdd(&a.hdr->counters[kCtrQkBlocks], (unsigned long long)qk_blocks);
             atomicAdd(&a.hdr->counters[kCtrPvBlocks], (unsigned long long)nlive);

@@ -61,7 +61,7 @@ extern "C" {
 typedef enum {
     ENT_OK = 0,
     ENT_EINVAL = 1,        /* a bad argument (null pointer, bad size, alpha out of range) */
-    ENT_EUNSUPPORTED = 2,  /* a valid request this build does not implement (e.g. d = 96) */
+    ENT_EUNSUPPORTED = 2,  /* a valid request the library does not implement (e.g. d = 96) */
     ENT_ECUDA = 3,         /* a CUDA runtime call failed; see ent_attn_last_error() */
     ENT_ETIMEOUT = 4       /* a bounded device wait gave up (reported by ent_attn_read_status) */
 } ent_status;

@@ -26,7 +26,7 @@ int main(void) {
     CHECK(ent_attn_fwd(fake, fake, fake, 1, 1, 128, 64, ENT_BF16, 2.5f, 1, fake, ffake, bfake,
                        NULL, fake, 256, NULL) == ENT_EINVAL);
     CHECK(strlen(ent_attn_last_error()) > 0);
-    /* head dimension this build does not implement */
+    /* a head dimension the library does not implement */
     CHECK(ent_attn_bwd(fake, fake, fake, NULL, fake, ffake, bfake, 1, 1, 128, 96, ENT_BF16, 1.5f,
                        1, fake, fake, fake, fake, (size_t)1 << 30, NULL) == ENT_EUNSUPPORTED);
     /* the otilde pair wants its otilde pointer */
